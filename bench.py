@@ -1,0 +1,273 @@
+#!/usr/bin/env python
+"""Batch-1 decode benchmark of the persistent decode kernel.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kie|reference]
+
+One "step" is one decode token: one pass of the whole decode path (every
+layer, LM head, greedy argmax, token feedback).  The timed region is one
+kie_decode(K) call -- a single persistent launch that runs K steps -- after
+an untimed prefill of the workload's prompt and W untimed warm-up steps.
+
+Default workload: the 2.3B-class dense decoder (34 layers, d 2048, 16x128
+query heads / 8 KV heads, F 8192, V 32768, fp16 weights and KV cache), prompt
+128 -> decode 512, seeded synthetic weights and prompt.  Every step streams
+4.41 GB of weights, far more than the 126 MB L2, so no L2 flush is needed
+between steps.
+
+Multi-GPU: the path is one request's serial decode chain, so it does not
+shard; N GPUs run N independent replicas (one request each) and `value` is
+the sum of their tokens/s, timed as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "batch-1 decode tokens/s/request on 1 B200; % of HBM roofline (bytes/token)"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=512, help="timed decode steps (tokens)")
+    ap.add_argument("--warmup", type=int, default=3, help="untimed decode steps before timing")
+    ap.add_argument("--impl", choices=["kie", "reference"], default="kie")
+    ap.add_argument("--workload", type=int, default=1, help="workload id (see synth/configs.py)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="bounded CPU work for the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int, period: float = 0.02):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def workload_bytes(m, P, K, weight_bytes_per_step, kv_bytes_per_position):
+    """Algorithmic bytes of K decode steps after a P-token prompt: every weight
+    once per step plus K and V of all positions 0..p at step p."""
+    kv_positions = sum(P + k + 1 for k in range(K))
+    return K * weight_bytes_per_step + kv_positions * kv_bytes_per_position
+
+
+def oracle_decode_rate(w, bits, seconds, warmup=0, max_steps=None):
+    """Greedy decode tokens/s of the float64 oracle on this host (bounded sample)."""
+    from oracle import Oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count()
+    m = w.model
+    import synth
+    prompt = synth.prompt(w)
+    orc = Oracle(m, bits, w.prompt_len + 4096, cache_f64=True)
+    orc.prefill(prompt)
+    if warmup:
+        orc.decode(warmup)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        orc.decode(1)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_steps and n >= max_steps):
+            break
+    return n / el, n, el, cores
+
+
+def main():
+    args = parse()
+    import numpy as np
+    import torch
+
+    import synth
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = synth.WORKLOADS[args.workload]
+    m = w.model
+    P, K, W = w.prompt_len, args.steps, max(3, args.warmup)
+
+    if args.impl == "reference":
+        # the oracle as it stands, on this host's cores, rank 0 only
+        if rank != 0:
+            return
+        bits = synth.generate_weights(m, w.weight_seed)
+        budget = max(5.0, min(120.0, args.cpu_seconds * 4))
+        rate, n, el, cores = oracle_decode_rate(w, bits, budget, warmup=min(W, 3), max_steps=K)
+        line = {"metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": 0, "steps": n,
+                "warmup": min(W, 3), "ms_per_step": 1e3 / rate, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "impl": "reference",
+                "config": {"workload": w.name, "prompt": P, "decode_steps": K, "batch": 1},
+                "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores,
+                                 "kind": "oracle",
+                                 "sample": f"{n} greedy decode steps of the float64 numpy "
+                                           f"oracle after the {P}-token prompt ({el:.1f} s)"},
+                "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import decode_persistent_monokernel_b200 as kie
+    kie.load()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    bits = synth.generate_weights(m, w.weight_seed)
+    prompt = synth.prompt(w)
+    max_seq = P + max(K, W) + 8
+    wdev = torch.from_numpy(bits.view(np.int16)).cuda()
+    stream = torch.cuda.current_stream()
+    dec = kie.Decoder(kie.make_desc(m, max_seq), wdev, stream=stream)
+    del wdev
+    torch.cuda.empty_cache()
+    st = dec.kie_get_stats()
+
+    # warm-up: prompt + W steps, untimed
+    dec.kie_prefill(prompt)
+    dec.kie_decode(W)
+    # timed: K steps from the workload's own starting point (position P)
+    dec.kie_prefill(prompt)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        toks = dec.kie_decode(K)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    kernel_ms = dec.kie_get_stats().last_kernel_ms
+    # end to end through the C ABI with host buffers: prompt in, tokens out
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    dec.kie_prefill(prompt)
+    toks2 = dec.kie_decode(K)
+    e2e_s = time.perf_counter() - t0
+    barrier()
+    assert (toks == toks2).all(), "decode is not reproducible"
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_s, kernel_ms], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, e2e_s, kernel_ms = t.tolist()
+
+    total_bytes = workload_bytes(m, P, K, st.weight_bytes_per_step, st.kv_bytes_per_position)
+    peak, peak_kind = peak_hbm()
+    achieved = total_bytes / (kernel_ms * 1e-3) / 1e9
+    value = world * K / (ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 (fp16 weights/KV)" if m.dtype == "f16"
+        else "f32 (bf16 weights/KV)", "data": "synthetic (seeded weights and prompt)",
+        "config": {"workload": w.name, "prompt": P, "decode_steps": K, "batch": 1,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2: %.2f GB of weights streamed per step"
+                         % (st.weight_bytes_per_step / 1e9)},
+        "us_per_token": 1e3 * ms / K,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "frac_of_8TBps_nominal": achieved / 8000.0,
+                     "bytes_per_step": total_bytes / K, "traffic": None,
+                     "kernel_ms": kernel_ms},
+        "clocks": clk.summary(),
+        "gpu_launches": 1,
+        "e2e": {"value": world * K / e2e_s,
+                "unit": "tokens/s (decode tokens / wall time of kie_prefill(host prompt) + "
+                        "kie_decode(host tokens))",
+                "h2d_bytes_per_step": 4 * P / K,
+                "d2h_bytes_per_step": (4 * P + 4 * K + 8) / K},
+        "kernel": {"ctas": st.n_ctas, "threads": st.threads_per_cta, "ring_slots": st.ring_slots,
+                   "smem_bytes": st.smem_bytes},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dec.kie_destroy()
+        rate, n, el, cores = oracle_decode_rate(w, bits, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"{n} greedy decode steps of the float64 numpy oracle "
+                                          f"after the {P}-token prompt ({el:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

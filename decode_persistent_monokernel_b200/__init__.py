@@ -1,0 +1,185 @@
+"""Python binding of libkie.so, the persistent batch-1 decode library.
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels behind the C ABI declared in ``include/kie.h``.  PyTorch supplies
+device memory and streams.  There is no fallback: if the compiled library is
+missing, importing the binding's calls raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkie.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "kie.h")
+
+KIE_OK = 0
+KIE_ERR_INVALID = -1
+KIE_ERR_OOM = -2
+KIE_ERR_CUDA = -3
+KIE_ERR_CAPACITY = -4
+KIE_ERR_NOT_RESIDENT = -5
+KIE_ERR_DEVICE_TIMEOUT = -6
+KIE_ERR_POISONED = -7
+KIE_F16 = 0
+KIE_BF16 = 1
+
+
+class kie_model_desc(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int32), ("d_model", ctypes.c_int32),
+                ("n_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("ffn_dim", ctypes.c_int32),
+                ("vocab", ctypes.c_int32), ("rms_eps", ctypes.c_float),
+                ("rope_theta", ctypes.c_float), ("dtype", ctypes.c_int32),
+                ("n_lanes", ctypes.c_int32), ("lane_delay", ctypes.c_int32),
+                ("max_seq", ctypes.c_int32)]
+
+
+class kie_stats(ctypes.Structure):
+    _fields_ = [("n_ctas", ctypes.c_int32), ("threads_per_cta", ctypes.c_int32),
+                ("ring_slots", ctypes.c_int32), ("slot_bytes", ctypes.c_int32),
+                ("smem_bytes", ctypes.c_int32), ("pos", ctypes.c_int32),
+                ("weight_bytes_per_step", ctypes.c_int64),
+                ("kv_bytes_per_position", ctypes.c_int64),
+                ("last_kernel_ms", ctypes.c_float), ("last_launch_steps", ctypes.c_int32),
+                ("pending_token", ctypes.c_int32)]
+
+
+class KieError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{msg} (status {code})")
+        self.code = code
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libkie.so (built by ``build.py``); raises if it is not there."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libkie.so not built: {path} is missing (run "
+                           "decode_persistent_monokernel_b200/build.py)")
+    L = ctypes.CDLL(path)
+    sig = {
+        "kie_create": ([ctypes.POINTER(kie_model_desc), _P, _P, ctypes.POINTER(_P)], _I),
+        "kie_prefill": ([_P, _P, _I, ctypes.POINTER(_I)], _I),
+        "kie_decode": ([_P, _I, _P], _I),
+        "kie_decode_ex": ([_P, _I, _P, _P, _P], _I),
+        "kie_destroy": ([_P], _I),
+        "kie_strerror": ([_I], ctypes.c_char_p),
+        "kie_get_stats": ([_P, ctypes.POINTER(kie_stats)], _I),
+        "kie_copy_kv": ([_P, _I, _I, _I, _I, _P, _P], _I),
+        "kie_debug_set": ([_P, _I, _I], _I),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def header_functions(path: str = HEADER) -> list:
+    """Names of every function the C header declares."""
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kie_[a-z_]+)\s*\(", text)))
+
+
+def strerror(code: int) -> str:
+    return load().kie_strerror(code).decode()
+
+
+def _check(code: int) -> None:
+    if code != KIE_OK:
+        raise KieError(code, strerror(code))
+
+
+def make_desc(shape, max_seq: int) -> kie_model_desc:
+    """A descriptor from any object with the model-shape attributes."""
+    return kie_model_desc(shape.n_layers, shape.d_model, shape.n_heads, shape.n_kv_heads,
+                          shape.head_dim, shape.ffn_dim, shape.vocab, shape.rms_eps,
+                          shape.rope_theta, KIE_F16 if shape.dtype == "f16" else KIE_BF16,
+                          shape.n_lanes, shape.lane_delay if shape.n_lanes > 1 else 0, max_seq)
+
+
+def _ptr(buf):
+    """Address of a torch tensor or a numpy array (host buffers must be contiguous)."""
+    if buf is None:
+        return None
+    if hasattr(buf, "data_ptr"):
+        return buf.data_ptr()
+    return buf.ctypes.data
+
+
+class Decoder:
+    """Owns one kie_ctx.  Host-side token arrays are int32 numpy arrays."""
+
+    def __init__(self, desc: kie_model_desc, weights_dev, stream=None):
+        L = load()
+        self._h = _P()
+        st = None if stream is None else (stream.cuda_stream if hasattr(stream, "cuda_stream")
+                                          else stream)
+        _check(L.kie_create(ctypes.byref(desc), _ptr(weights_dev), st, ctypes.byref(self._h)))
+        self.desc = desc
+
+    def kie_prefill(self, tokens) -> int:
+        import numpy as np
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        nxt = _I()
+        _check(load().kie_prefill(self._h, t.ctypes.data, len(t), ctypes.byref(nxt)))
+        return nxt.value
+
+    def kie_decode(self, n_steps: int):
+        import numpy as np
+        out = np.empty(n_steps, dtype=np.int32)
+        _check(load().kie_decode(self._h, n_steps, out.ctypes.data))
+        return out
+
+    def kie_decode_ex(self, n_steps: int, forced=None, logits_out=None):
+        import numpy as np
+        out = np.empty(n_steps, dtype=np.int32)
+        f = None if forced is None else np.ascontiguousarray(forced, dtype=np.int32)
+        _check(load().kie_decode_ex(self._h, n_steps, None if f is None else f.ctypes.data,
+                                    out.ctypes.data, _ptr(logits_out)))
+        return out
+
+    def kie_get_stats(self) -> kie_stats:
+        s = kie_stats()
+        _check(load().kie_get_stats(self._h, ctypes.byref(s)))
+        return s
+
+    def kie_copy_kv(self, layer: int, kv_head: int, pos0: int, n: int):
+        import numpy as np
+        k = np.empty((n, self.desc.head_dim), dtype=np.uint16)
+        v = np.empty((n, self.desc.head_dim), dtype=np.uint16)
+        _check(load().kie_copy_kv(self._h, layer, kv_head, pos0, n, k.ctypes.data, v.ctypes.data))
+        return k, v
+
+    def kie_debug_set(self, watchdog_ms: int, skip_signal_cta: int = -1) -> None:
+        _check(load().kie_debug_set(self._h, watchdog_ms, skip_signal_cta))
+
+    def kie_destroy(self) -> None:
+        if self._h:
+            _check(load().kie_destroy(self._h))
+            self._h = _P()
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.kie_destroy()
+
+    def __del__(self):
+        try:
+            if self._h:
+                load().kie_destroy(self._h)
+        except Exception:
+            pass

@@ -1,0 +1,695 @@
+// Host side of libkie.so: the C ABI declared in include/kie.h.
+//
+// kie_create plans how the decode step's weight rows are split over the SMs,
+// copies the canonical weights into one contiguous stream per SM in the order
+// that SM consumes them (the per-SM weight stream the persistent kernel's
+// producer warp reads with bulk copies), and allocates the KV cache and
+// activation buffers.  kie_prefill / kie_decode launch the persistent kernel
+// once per call, cooperatively, with one CTA per SM.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <string>
+#include <vector>
+
+#include "../../include/kie.h"
+#include "kie_internal.h"
+
+namespace kie {
+size_t monokernel_smem_bytes(int ring_slots, int vbuf_floats, int part_floats);
+int monokernel_threads();
+const void *monokernel_fn(int dtype);
+cudaError_t launch_repack(const uint16_t *src, uint8_t *dst, const RepackJob *jobs, int njobs,
+                          cudaStream_t st);
+}  // namespace kie
+
+using namespace kie;
+
+static thread_local std::string g_last_error;
+
+static void set_error(const char *what, cudaError_t e) {
+  char buf[512];
+  snprintf(buf, sizeof buf, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+  g_last_error = buf;
+}
+
+// ---------------------------------------------------------------- canonical layout
+namespace {
+
+struct Piece {          // rows of one canonical matrix inside a stage's row space
+  int64_t src;          // element offset of the piece's first row in layer 0
+  int64_t src2;         // second source (up rows of a gate/up piece), or -1
+  int32_t rows, K, in_off;
+};
+
+struct Layout {
+  int64_t embed, final_norm, lm_head, total;
+  int64_t layer0, layer_stride, lane_stride;
+  // offsets inside one lane of layer 0 (relative to the lane's start)
+  int64_t attn_norm, wq, wk, wv, wo, ffn_norm, wg, wu, wd;
+  int64_t mix;  // relative to the layer start (lane models)
+};
+
+Layout make_layout(const kie_model_desc &m) {
+  Layout L{};
+  const int64_t d = m.d_model, V = m.vocab, dh = m.head_dim;
+  const int64_t nl = m.n_lanes, dl = d / nl, hq = m.n_heads / nl, hkv = m.n_kv_heads / nl,
+                fl = m.ffn_dim / nl;
+  int64_t o = 0;
+  L.embed = o; o += V * d;
+  L.layer0 = o;
+  int64_t q = 0;
+  L.attn_norm = q; q += dl;
+  L.wq = q; q += hq * dh * dl;
+  L.wk = q; q += hkv * dh * dl;
+  L.wv = q; q += hkv * dh * dl;
+  L.wo = q; q += dl * hq * dh;
+  L.ffn_norm = q; q += dl;
+  L.wg = q; q += fl * dl;
+  L.wu = q; q += fl * dl;
+  L.wd = q; q += dl * fl;
+  L.lane_stride = q;
+  L.mix = nl * q;
+  L.layer_stride = nl * q + (nl > 1 ? d * d : 0);
+  o += m.n_layers * L.layer_stride;
+  L.final_norm = o; o += d;
+  L.lm_head = o; o += V * d;
+  L.total = o;
+  return L;
+}
+
+struct Plan {
+  int n_ctas = 0;
+  StageShape shape[ST_COUNT]{};
+  std::vector<StageCta> stage_cta;   // [ST_COUNT][n_ctas]
+  std::vector<Block> blocks;
+  std::vector<int32_t> cta_blk_begin;
+  std::vector<int64_t> cta_stream_off;
+  std::vector<RepackJob> jobs;
+  int64_t stream_bytes = 0;
+  int vbuf_floats = 0, part_floats = 0, ring_slots = 0;
+  size_t smem = 0;
+  int max_split = 0;
+  int64_t weight_bytes_per_step = 0;
+};
+
+StageShape make_shape(int K, int in_len, int out_len) {
+  StageShape s{};
+  s.K = K;
+  int nseg = (K + 2047) / 2048;
+  while (K % nseg != 0 || (K / nseg) % 8 != 0) ++nseg;
+  s.nseg = nseg;
+  s.KT = K / nseg;
+  int R = 16;
+  while (R > 1 && R * s.KT * 2 > kSlotBytes) R >>= 1;
+  s.R = R;
+  s.in_len = in_len;
+  s.out_len = out_len;
+  return s;
+}
+
+// Row pieces of each stage in the stage's output order.
+void stage_pieces(const kie_model_desc &m, const Layout &Ly, int k, std::vector<Piece> &out) {
+  out.clear();
+  const int nl = m.n_lanes, d = m.d_model, dh = m.head_dim;
+  const int dl = d / nl, hq = m.n_heads / nl, hkv = m.n_kv_heads / nl, fl = m.ffn_dim / nl;
+  auto lane = [&](int ln) { return Ly.layer0 + int64_t(ln) * Ly.lane_stride; };
+  switch (k) {
+    case ST_QKV:
+      for (int ln = 0; ln < nl; ++ln) out.push_back({lane(ln) + Ly.wq, -1, hq * dh, dl, ln * dl});
+      for (int ln = 0; ln < nl; ++ln) out.push_back({lane(ln) + Ly.wk, -1, hkv * dh, dl, ln * dl});
+      for (int ln = 0; ln < nl; ++ln) out.push_back({lane(ln) + Ly.wv, -1, hkv * dh, dl, ln * dl});
+      break;
+    case ST_O:
+      for (int ln = 0; ln < nl; ++ln)
+        out.push_back({lane(ln) + Ly.wo, -1, dl, hq * dh, ln * hq * dh});
+      break;
+    case ST_GU:
+      for (int ln = 0; ln < nl; ++ln)
+        out.push_back({lane(ln) + Ly.wg, lane(ln) + Ly.wu, fl, dl, ln * dl});
+      break;
+    case ST_D:
+      for (int ln = 0; ln < nl; ++ln) out.push_back({lane(ln) + Ly.wd, -1, dl, fl, ln * fl});
+      break;
+    case ST_MIX:
+      out.push_back({Ly.layer0 + Ly.mix, -1, d, d, 0});
+      break;
+    case ST_LM:
+      out.push_back({Ly.lm_head, -1, m.vocab, d, 0});
+      break;
+  }
+}
+
+// Blocks of one CTA's row range [r0, r1) of a stage; `up` selects the second
+// source of gate/up pieces.  Returns (src offsets of layer 0) per block.
+void cut_blocks(const std::vector<Piece> &pieces, int r0, int r1, bool up, int lrow_base,
+                const StageShape &sh, int &tile, std::vector<Block> &blk,
+                std::vector<int64_t> &src) {
+  int base = 0;
+  for (const Piece &pc : pieces) {
+    const int a = std::max(r0, base), b = std::min(r1, base + pc.rows);
+    if (a < b) {
+      Block B{};
+      B.lrow0 = lrow_base + (a - r0);
+      B.nrows = b - a;
+      B.in_off = pc.in_off;
+      B.tile0 = tile;
+      tile += ((B.nrows + sh.R - 1) / sh.R) * sh.nseg;
+      blk.push_back(B);
+      src.push_back((up ? pc.src2 : pc.src) + int64_t(a - base) * pc.K);
+    }
+    base += pc.rows;
+  }
+}
+
+const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Plan &P) {
+  const Layout Ly = make_layout(m);
+  const int nl = m.n_lanes, d = m.d_model, dh = m.head_dim;
+  const bool lanes = nl > 1;
+  P.n_ctas = n_ctas;
+  P.shape[ST_QKV] = make_shape(d / nl, d, (m.n_heads + 2 * m.n_kv_heads) * dh);
+  P.shape[ST_O] = make_shape(m.n_heads / nl * dh, m.n_heads * dh, d);
+  P.shape[ST_GU] = make_shape(d / nl, d, m.ffn_dim);
+  P.shape[ST_D] = make_shape(m.ffn_dim / nl, m.ffn_dim, d);
+  P.shape[ST_MIX] = make_shape(d, d, d);
+  P.shape[ST_LM] = make_shape(d, d, m.vocab);
+
+  // per-CTA blocks of every stage kind (same for every layer)
+  P.stage_cta.assign(size_t(ST_COUNT) * n_ctas, StageCta{});
+  std::vector<std::vector<int64_t>> src_of_cta(n_ctas);   // per CTA, per block: layer-0 source
+  P.cta_blk_begin.assign(n_ctas + 1, 0);
+  std::vector<Piece> pieces;
+  int part_max = 4;
+  for (int c = 0; c < n_ctas; ++c) {
+    P.cta_blk_begin[c] = int(P.blocks.size());
+    int local_blk = 0;
+    for (int k = 0; k < ST_COUNT; ++k) {
+      StageCta &sc = P.stage_cta[size_t(k) * n_ctas + c];
+      if (k == ST_MIX && !lanes) continue;
+      stage_pieces(m, Ly, k, pieces);
+      const StageShape &sh = P.shape[k];
+      const int N = sh.out_len;
+      const int r0 = int(int64_t(N) * c / n_ctas), r1 = int(int64_t(N) * (c + 1) / n_ctas);
+      sc.row0 = r0;
+      sc.nout = r1 - r0;
+      sc.blk_begin = local_blk;
+      int tile = 0;
+      std::vector<Block> blk;
+      std::vector<int64_t> src;
+      cut_blocks(pieces, r0, r1, false, 0, sh, tile, blk, src);
+      if (k == ST_GU) cut_blocks(pieces, r0, r1, true, sc.nout, sh, tile, blk, src);
+      sc.nlocal = (k == ST_GU) ? 2 * sc.nout : sc.nout;
+      sc.ntiles = tile;
+      sc.nblk = int(blk.size());
+      int64_t bytes = 0;
+      for (const Block &B : blk) bytes += int64_t(B.nrows) * sh.K * 2;
+      sc.bytes = bytes;
+      part_max = std::max(part_max, sc.nlocal * sh.nseg);
+      for (size_t i = 0; i < blk.size(); ++i) {
+        P.blocks.push_back(blk[i]);
+        src_of_cta[c].push_back(src[i]);
+      }
+      local_blk += int(blk.size());
+    }
+    if (local_blk > kMaxBlocksPerCta) return "too many row blocks per CTA for this shape";
+  }
+  P.cta_blk_begin[n_ctas] = int(P.blocks.size());
+
+  // per-CTA streams in consumption order, and the repack jobs that fill them
+  int64_t off = 0;
+  for (int c = 0; c < n_ctas; ++c) {
+    P.cta_stream_off.push_back(off);
+    auto emit = [&](int k, int64_t layer_off) {
+      const StageCta &sc = P.stage_cta[size_t(k) * n_ctas + c];
+      const StageShape &sh = P.shape[k];
+      for (int b = 0; b < sc.nblk; ++b) {
+        const Block &B = P.blocks[P.cta_blk_begin[c] + sc.blk_begin + b];
+        RepackJob j{};
+        j.src_elem = src_of_cta[c][sc.blk_begin + b] + layer_off;
+        j.dst_byte = off;
+        j.nrows = B.nrows;
+        j.K = sh.K;
+        j.KT = sh.KT;
+        j.R = sh.R;
+        P.jobs.push_back(j);
+        off += int64_t(B.nrows) * sh.K * 2;
+      }
+    };
+    for (int l = 0; l < m.n_layers; ++l) {
+      const int64_t lo = int64_t(l) * Ly.layer_stride;
+      emit(ST_QKV, lo);
+      if (lanes && l >= 1) emit(ST_MIX, lo - Ly.layer_stride);
+      emit(ST_O, lo);
+      emit(ST_GU, lo);
+      emit(ST_D, lo);
+    }
+    if (lanes) emit(ST_MIX, int64_t(m.n_layers - 1) * Ly.layer_stride);
+    emit(ST_LM, 0);
+    off = (off + 255) / 256 * 256;
+  }
+  P.stream_bytes = off;
+
+  // shared memory: input vector / attention scratch, partial sums, ring
+  const int G = m.n_heads / m.n_kv_heads;
+  int vb = 0;
+  for (int k = 0; k < ST_COUNT; ++k) vb = std::max(vb, P.shape[k].in_len);
+  vb = std::max(vb, (G + 2) * dh + kConsumerWarps * G * (dh + 2));
+  P.vbuf_floats = (vb + 3) / 4 * 4;
+  P.part_floats = (part_max + 3) / 4 * 4;
+  const size_t fixed = monokernel_smem_bytes(0, P.vbuf_floats, P.part_floats);
+  if (fixed + 4 * (kSlotBytes + 16) > smem_cap) return "shape needs more shared memory than the SM has";
+  int slots = int((smem_cap - fixed) / (kSlotBytes + 16));
+  slots = std::min(slots, 32);
+  P.ring_slots = slots;
+  P.smem = monokernel_smem_bytes(slots, P.vbuf_floats, P.part_floats);
+  P.max_split = (n_ctas + m.n_kv_heads - 1) / m.n_kv_heads;
+
+  // weights streamed by one decode step: all matrices, norms, one embedding row
+  const int64_t esz = 2;
+  P.weight_bytes_per_step = (Ly.total - int64_t(m.vocab) * d + d) * esz;
+  return nullptr;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- context
+struct kie_ctx {
+  kie_model_desc m{};
+  int device = 0;
+  cudaStream_t stream = nullptr;
+  Plan plan;
+  int pos = 0;
+  int pending = -1;
+  int poisoned = 0;   // sticky error code
+  uint64_t watchdog_ns = 2000000000ull;
+  int skip_signal_cta = -1;
+  float last_ms = 0.f;
+  int last_steps = 0;
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  // device buffers
+  uint8_t *wstream = nullptr;
+  uint16_t *embed = nullptr;
+  float *gains = nullptr;  // [2L + 1, d]
+  float2 *rope = nullptr;
+  uint16_t *kcache = nullptr, *vcache = nullptr;
+  float *act = nullptr;    // x, qkv, attn_o, h, u, dsum, attn_part
+  uint32_t *sync = nullptr;
+  unsigned long long *keys = nullptr;
+  int32_t *tokens_in = nullptr, *tokens_out = nullptr;
+  StageCta *d_stage_cta = nullptr;
+  Block *d_blocks = nullptr;
+  int32_t *d_blk_begin = nullptr;
+  int64_t *d_stream_off = nullptr;
+  size_t off_x, off_qkv, off_o, off_h, off_u, off_dsum, off_part, act_floats;
+  size_t kv_elems = 0;
+  std::vector<int32_t> host_tokens;
+};
+
+static const char *validate(const kie_model_desc *m) {
+  if (!m) return "null descriptor";
+  if (m->n_layers < 1 || m->d_model < 8 || m->n_heads < 1 || m->n_kv_heads < 1 ||
+      m->ffn_dim < 8 || m->vocab < 1 || m->max_seq < 1)
+    return "sizes must be positive";
+  if (m->head_dim != 64 && m->head_dim != 128) return "head_dim must be 64 or 128";
+  if (m->dtype != KIE_F16 && m->dtype != KIE_BF16) return "dtype must be KIE_F16 or KIE_BF16";
+  if (m->n_lanes < 1) return "n_lanes must be >= 1";
+  if (m->n_heads % m->n_kv_heads) return "n_heads must be a multiple of n_kv_heads";
+  if (m->n_heads / m->n_kv_heads > 4) return "at most 4 query heads per KV head";
+  const int nl = m->n_lanes;
+  if (m->d_model % nl || m->n_heads % nl || m->n_kv_heads % nl || m->ffn_dim % nl)
+    return "lane count must divide d_model, heads, kv heads and ffn_dim";
+  if (m->n_heads * m->head_dim != m->d_model) return "n_heads * head_dim must equal d_model";
+  if ((m->d_model / nl) % 8 || (m->ffn_dim / nl) % 8) return "lane width and lane ffn must be multiples of 8";
+  if (nl > 1 && m->lane_delay < 2) return "lane_delay must be >= 2";
+  if (nl > 64) return "at most 64 lanes";
+  if (!(m->rms_eps >= 0.f) || !(m->rope_theta > 0.f)) return "bad rms_eps or rope_theta";
+  return nullptr;
+}
+
+static int cuda_fail(kie_ctx *c, const char *what, cudaError_t e) {
+  set_error(what, e);
+  if (c) c->poisoned = KIE_ERR_CUDA;
+  return KIE_ERR_CUDA;
+}
+
+#define CK(call)                                                    \
+  do {                                                              \
+    cudaError_t e_ = (call);                                        \
+    if (e_ != cudaSuccess) return cuda_fail(ctx, #call, e_);        \
+  } while (0)
+
+static void free_ctx(kie_ctx *c) {
+  if (!c) return;
+  void *ptrs[] = {c->wstream, c->embed, c->gains, c->rope, c->kcache, c->vcache, c->act,
+                  c->sync, c->keys, c->tokens_in, c->tokens_out, c->d_stage_cta, c->d_blocks,
+                  c->d_blk_begin, c->d_stream_off};
+  for (void *p : ptrs)
+    if (p) cudaFree(p);
+  if (c->ev0) cudaEventDestroy(c->ev0);
+  if (c->ev1) cudaEventDestroy(c->ev1);
+  delete c;
+}
+
+static int alloc(kie_ctx *ctx, void **p, size_t bytes, const char *what) {
+  cudaError_t e = cudaMalloc(p, bytes ? bytes : 16);
+  if (e == cudaErrorMemoryAllocation) {
+    cudaGetLastError();
+    set_error(what, e);
+    return KIE_ERR_OOM;
+  }
+  if (e != cudaSuccess) return cuda_fail(ctx, what, e);
+  return KIE_OK;
+}
+
+extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void *stream,
+                          kie_ctx **out) {
+  if (!out) return KIE_ERR_INVALID;
+  *out = nullptr;
+  if (const char *why = validate(desc)) {
+    g_last_error = why;
+    return KIE_ERR_INVALID;
+  }
+  if (!weights || (reinterpret_cast<uintptr_t>(weights) & 15)) {
+    g_last_error = "weights must be a 16-byte aligned device pointer";
+    return KIE_ERR_INVALID;
+  }
+  kie_ctx *ctx = new kie_ctx();
+  ctx->m = *desc;
+  ctx->stream = static_cast<cudaStream_t>(stream);
+  const kie_model_desc &m = ctx->m;
+  int rc;
+  auto fail = [&](int code) {
+    free_ctx(ctx);
+    return code;
+  };
+  if (const char *env = getenv("KIE_WATCHDOG_MS")) {
+    long v = atol(env);
+    if (v > 0) ctx->watchdog_ns = uint64_t(v) * 1000000ull;
+  }
+  cudaError_t e = cudaGetDevice(&ctx->device);
+  if (e != cudaSuccess) return fail(cuda_fail(nullptr, "cudaGetDevice", e));
+  cudaPointerAttributes pa{};
+  e = cudaPointerGetAttributes(&pa, weights);
+  if (e != cudaSuccess || (pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged)) {
+    cudaGetLastError();
+    g_last_error = "weights is not a device pointer";
+    return fail(KIE_ERR_INVALID);
+  }
+  int n_sm = 0, smem_optin = 0, coop = 0;
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, ctx->device);
+  cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, ctx->device);
+  cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, ctx->device);
+  if (!coop) {
+    g_last_error = "device lacks cooperative launch";
+    return fail(KIE_ERR_NOT_RESIDENT);
+  }
+  if (n_sm < m.n_kv_heads) {
+    g_last_error = "fewer SMs than KV heads";
+    return fail(KIE_ERR_NOT_RESIDENT);
+  }
+  if (const char *why = build_plan(m, n_sm, size_t(smem_optin), ctx->plan)) {
+    g_last_error = why;
+    return fail(KIE_ERR_INVALID);
+  }
+  Plan &P = ctx->plan;
+  const void *fn = monokernel_fn(m.dtype);
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(P.smem));
+  if (e != cudaSuccess) return fail(cuda_fail(nullptr, "cudaFuncSetAttribute", e));
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, monokernel_threads(), P.smem);
+  if (e != cudaSuccess) return fail(cuda_fail(nullptr, "occupancy query", e));
+  if (per_sm < 1) {
+    g_last_error = "persistent CTA does not fit on an SM";
+    return fail(KIE_ERR_NOT_RESIDENT);
+  }
+
+  const Layout Ly = make_layout(m);
+  const int d = m.d_model, L = m.n_layers, dh = m.head_dim;
+  // ---- allocations
+  if ((rc = alloc(ctx, (void **)&ctx->wstream, P.stream_bytes, "weight stream"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->embed, size_t(m.vocab) * d * 2, "embedding"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->gains, size_t(2 * L + 1) * d * 4, "gains"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->rope, size_t(m.max_seq) * (dh / 2) * 8, "rope"))) return fail(rc);
+  ctx->kv_elems = size_t(L) * m.n_kv_heads * m.max_seq * dh;
+  if ((rc = alloc(ctx, (void **)&ctx->kcache, ctx->kv_elems * 2, "K cache"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->vcache, ctx->kv_elems * 2, "V cache"))) return fail(rc);
+  size_t o = 0;
+  auto take = [&](size_t n) { size_t r = o; o += (n + 63) / 64 * 64; return r; };
+  ctx->off_x = take(d);
+  ctx->off_qkv = take(size_t(m.n_heads + 2 * m.n_kv_heads) * dh);
+  ctx->off_o = take(size_t(m.n_heads) * dh);
+  ctx->off_h = take(m.ffn_dim);
+  ctx->off_u = take(size_t(2) * d);
+  ctx->off_dsum = take(size_t(std::max(1, m.lane_delay)) * d);
+  ctx->off_part = take(size_t(m.n_heads) * P.max_split * (dh + 2));
+  ctx->act_floats = o;
+  if ((rc = alloc(ctx, (void **)&ctx->act, o * 4, "activations"))) return fail(rc);
+  const size_t sync_words = size_t(SY_ATTN0 + m.n_kv_heads) * kSyncStride;
+  if ((rc = alloc(ctx, (void **)&ctx->sync, sync_words * 4, "sync"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->keys, size_t(m.max_seq) * 8, "keys"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->tokens_in, size_t(m.max_seq) * 4, "tokens"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->tokens_out, size_t(m.max_seq) * 4, "tokens"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->d_stage_cta, P.stage_cta.size() * sizeof(StageCta), "plan"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->d_blocks, std::max<size_t>(1, P.blocks.size()) * sizeof(Block), "plan"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->d_blk_begin, P.cta_blk_begin.size() * 4, "plan"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->d_stream_off, P.cta_stream_off.size() * 8, "plan"))) return fail(rc);
+  RepackJob *d_jobs = nullptr;
+  if ((rc = alloc(ctx, (void **)&d_jobs, P.jobs.size() * sizeof(RepackJob), "repack jobs"))) return fail(rc);
+
+  cudaStream_t st = ctx->stream;
+  auto ck = [&](cudaError_t er, const char *what) {
+    if (er != cudaSuccess) { cuda_fail(nullptr, what, er); return false; }
+    return true;
+  };
+  bool ok = true;
+  ok = ok && ck(cudaMemcpyAsync(ctx->d_stage_cta, P.stage_cta.data(), P.stage_cta.size() * sizeof(StageCta), cudaMemcpyHostToDevice, st), "plan copy");
+  if (!P.blocks.empty())
+    ok = ok && ck(cudaMemcpyAsync(ctx->d_blocks, P.blocks.data(), P.blocks.size() * sizeof(Block), cudaMemcpyHostToDevice, st), "plan copy");
+  ok = ok && ck(cudaMemcpyAsync(ctx->d_blk_begin, P.cta_blk_begin.data(), P.cta_blk_begin.size() * 4, cudaMemcpyHostToDevice, st), "plan copy");
+  ok = ok && ck(cudaMemcpyAsync(ctx->d_stream_off, P.cta_stream_off.data(), P.cta_stream_off.size() * 8, cudaMemcpyHostToDevice, st), "plan copy");
+  ok = ok && ck(cudaMemcpyAsync(d_jobs, P.jobs.data(), P.jobs.size() * sizeof(RepackJob), cudaMemcpyHostToDevice, st), "plan copy");
+  const uint16_t *w = static_cast<const uint16_t *>(weights);
+  ok = ok && ck(launch_repack(w, ctx->wstream, d_jobs, int(P.jobs.size()), st), "repack");
+  ok = ok && ck(cudaMemcpyAsync(ctx->embed, w + Ly.embed, size_t(m.vocab) * d * 2, cudaMemcpyDeviceToDevice, st), "embedding copy");
+  // norm gains: widen to fp32 on the host (exact) from a host copy of the gain words
+  std::vector<uint16_t> gbits(size_t(2 * L + 1) * d);
+  const int nl = m.n_lanes, dl = d / nl;
+  for (int l = 0; l < L && ok; ++l)
+    for (int ln = 0; ln < nl && ok; ++ln) {
+      const int64_t lane0 = Ly.layer0 + int64_t(l) * Ly.layer_stride + int64_t(ln) * Ly.lane_stride;
+      ok = ck(cudaMemcpyAsync(&gbits[size_t(l) * d + size_t(ln) * dl], w + lane0 + Ly.attn_norm, size_t(dl) * 2, cudaMemcpyDeviceToHost, st), "gain copy") &&
+           ck(cudaMemcpyAsync(&gbits[size_t(L + l) * d + size_t(ln) * dl], w + lane0 + Ly.ffn_norm, size_t(dl) * 2, cudaMemcpyDeviceToHost, st), "gain copy");
+    }
+  ok = ok && ck(cudaMemcpyAsync(&gbits[size_t(2 * L) * d], w + Ly.final_norm, size_t(d) * 2, cudaMemcpyDeviceToHost, st), "gain copy");
+  ok = ok && ck(cudaStreamSynchronize(st), "create sync");
+  if (!ok) { cudaFree(d_jobs); return fail(KIE_ERR_CUDA); }
+  std::vector<float> gains(gbits.size());
+  for (size_t i = 0; i < gbits.size(); ++i) {
+    const uint32_t b = gbits[i];
+    if (m.dtype == KIE_BF16) {
+      uint32_t u = b << 16;
+      memcpy(&gains[i], &u, 4);
+    } else {  // binary16 -> binary32, from the format definition
+      const uint32_t s = (b >> 15) & 1, ex = (b >> 10) & 31, fr = b & 1023;
+      float v;
+      if (ex == 0) v = ldexpf(float(fr), -24);
+      else if (ex == 31) v = fr ? NAN : INFINITY;
+      else v = ldexpf(float(fr | 1024), int(ex) - 25);
+      gains[i] = s ? -v : v;
+    }
+  }
+  // RoPE table: angle p * theta^(-2i/dh) and its cos/sin in double, stored fp32
+  std::vector<float2> rope(size_t(m.max_seq) * (dh / 2));
+  for (int p = 0; p < m.max_seq; ++p)
+    for (int i = 0; i < dh / 2; ++i) {
+      const double ang = double(p) * pow(double(m.rope_theta), -2.0 * i / dh);
+      rope[size_t(p) * (dh / 2) + i] = make_float2(float(cos(ang)), float(sin(ang)));
+    }
+  ok = ck(cudaMemcpyAsync(ctx->gains, gains.data(), gains.size() * 4, cudaMemcpyHostToDevice, st), "gain upload") &&
+       ck(cudaMemcpyAsync(ctx->rope, rope.data(), rope.size() * 8, cudaMemcpyHostToDevice, st), "rope upload") &&
+       ck(cudaMemsetAsync(ctx->kcache, 0xff, ctx->kv_elems * 2, st), "cache poison") &&
+       ck(cudaMemsetAsync(ctx->vcache, 0xff, ctx->kv_elems * 2, st), "cache poison") &&
+       ck(cudaMemsetAsync(ctx->act, 0, ctx->act_floats * 4, st), "act clear") &&
+       ck(cudaEventCreate(&ctx->ev0), "event") && ck(cudaEventCreate(&ctx->ev1), "event") &&
+       ck(cudaStreamSynchronize(st), "create sync");
+  cudaFree(d_jobs);
+  if (!ok) return fail(KIE_ERR_CUDA);
+  *out = ctx;
+  return KIE_OK;
+}
+
+// Run the persistent kernel for n steps from position pos0.
+static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int first_token,
+               bool logits_every_step, float *logits_out, int32_t *out_host) {
+  const kie_model_desc &m = ctx->m;
+  const Plan &P = ctx->plan;
+  cudaStream_t st = ctx->stream;
+  KernelArgs a{};
+  a.n_layers = m.n_layers; a.d_model = m.d_model; a.n_heads = m.n_heads;
+  a.n_kv_heads = m.n_kv_heads; a.head_dim = m.head_dim; a.ffn_dim = m.ffn_dim; a.vocab = m.vocab;
+  a.n_lanes = m.n_lanes; a.lane_delay = m.n_lanes > 1 ? m.lane_delay : 1;
+  a.lane_width = m.d_model / m.n_lanes; a.lane_heads = m.n_heads / m.n_lanes;
+  a.lane_kv_heads = m.n_kv_heads / m.n_lanes; a.lane_ffn = m.ffn_dim / m.n_lanes;
+  a.rms_eps = m.rms_eps;
+  a.attn_scale = float(1.0 / sqrt(double(m.head_dim)));
+  a.max_seq = m.max_seq;
+  a.n_ctas = P.n_ctas; a.ring_slots = P.ring_slots;
+  a.vbuf_floats = P.vbuf_floats; a.part_floats = P.part_floats;
+  for (int k = 0; k < ST_COUNT; ++k) a.shape[k] = P.shape[k];
+  a.stage_cta = ctx->d_stage_cta; a.blocks = ctx->d_blocks;
+  a.cta_blk_begin = ctx->d_blk_begin; a.cta_stream_off = ctx->d_stream_off;
+  a.wstream = ctx->wstream; a.embed = ctx->embed;
+  a.gain_attn = ctx->gains; a.gain_ffn = ctx->gains + size_t(m.n_layers) * m.d_model;
+  a.gain_final = ctx->gains + size_t(2 * m.n_layers) * m.d_model;
+  a.rope_cs = ctx->rope; a.kcache = ctx->kcache; a.vcache = ctx->vcache;
+  a.x = ctx->act + ctx->off_x; a.qkv = ctx->act + ctx->off_qkv; a.attn_o = ctx->act + ctx->off_o;
+  a.hbuf = ctx->act + ctx->off_h; a.ubuf = ctx->act + ctx->off_u; a.dsum = ctx->act + ctx->off_dsum;
+  a.attn_part = ctx->act + ctx->off_part; a.max_split = P.max_split;
+  a.sync = ctx->sync; a.keys = ctx->keys;
+  a.pos0 = pos0; a.n_steps = n; a.first_token = first_token;
+  a.forced = forced_host ? ctx->tokens_in : nullptr;
+  a.logits_every_step = logits_every_step ? 1 : 0;
+  a.out_tokens = ctx->tokens_out; a.logits_out = logits_out;
+  a.watchdog_ns = ctx->watchdog_ns;
+  a.skip_signal_cta = ctx->skip_signal_cta;
+  ctx->skip_signal_cta = -1;
+
+  const size_t sync_words = size_t(SY_ATTN0 + m.n_kv_heads) * kSyncStride;
+  if (forced_host)
+    CK(cudaMemcpyAsync(ctx->tokens_in, forced_host, size_t(n) * 4, cudaMemcpyHostToDevice, st));
+  CK(cudaMemsetAsync(ctx->sync, 0, sync_words * 4, st));
+  CK(cudaMemsetAsync(ctx->keys, 0, size_t(n) * 8, st));
+  void *args[] = {&a};
+  CK(cudaEventRecord(ctx->ev0, st));
+  CK(cudaLaunchCooperativeKernel(monokernel_fn(m.dtype), dim3(P.n_ctas), dim3(monokernel_threads()),
+                                 args, P.smem, st));
+  CK(cudaEventRecord(ctx->ev1, st));
+  uint32_t status = 0;
+  CK(cudaMemcpyAsync(&status, ctx->sync + SY_STATUS * kSyncStride, 4, cudaMemcpyDeviceToHost, st));
+  ctx->host_tokens.resize(n);
+  CK(cudaMemcpyAsync(ctx->host_tokens.data(), ctx->tokens_out, size_t(n) * 4, cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  CK(cudaEventElapsedTime(&ctx->last_ms, ctx->ev0, ctx->ev1));
+  ctx->last_steps = n;
+  if (status != 0) {
+    char buf[160];
+    snprintf(buf, sizeof buf, "device watchdog: a bounded wait ran out (code 0x%x)", status);
+    g_last_error = buf;
+    ctx->poisoned = KIE_ERR_DEVICE_TIMEOUT;
+    return KIE_ERR_DEVICE_TIMEOUT;
+  }
+  if (out_host) memcpy(out_host, ctx->host_tokens.data(), size_t(n) * 4);
+  return KIE_OK;
+}
+
+extern "C" int kie_prefill(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_token) {
+  if (!ctx || !tokens || !next_token || n < 1) return KIE_ERR_INVALID;
+  if (ctx->poisoned) return KIE_ERR_POISONED;
+  if (n > ctx->m.max_seq) return KIE_ERR_CAPACITY;
+  for (int i = 0; i < n; ++i)
+    if (tokens[i] < 0 || tokens[i] >= ctx->m.vocab) return KIE_ERR_INVALID;
+  CK(cudaMemsetAsync(ctx->kcache, 0xff, ctx->kv_elems * 2, ctx->stream));
+  CK(cudaMemsetAsync(ctx->vcache, 0xff, ctx->kv_elems * 2, ctx->stream));
+  ctx->pos = 0;
+  ctx->pending = -1;
+  std::vector<int32_t> out(n);
+  int rc = run(ctx, 0, n, tokens, 0, false, nullptr, out.data());
+  if (rc) return rc;
+  ctx->pos = n;
+  ctx->pending = out[n - 1];
+  *next_token = ctx->pending;
+  return KIE_OK;
+}
+
+extern "C" int kie_decode_ex(kie_ctx *ctx, int32_t n_steps, const int32_t *forced_tokens,
+                             int32_t *out_tokens, float *logits_out) {
+  if (!ctx || !out_tokens || n_steps < 1) return KIE_ERR_INVALID;
+  if (ctx->poisoned) return KIE_ERR_POISONED;
+  if (!forced_tokens && ctx->pending < 0) return KIE_ERR_INVALID;
+  if (int64_t(ctx->pos) + n_steps > ctx->m.max_seq) return KIE_ERR_CAPACITY;
+  if (forced_tokens)
+    for (int i = 0; i < n_steps; ++i)
+      if (forced_tokens[i] < 0 || forced_tokens[i] >= ctx->m.vocab) return KIE_ERR_INVALID;
+  int rc = run(ctx, ctx->pos, n_steps, forced_tokens, ctx->pending, true, logits_out, out_tokens);
+  if (rc) return rc;
+  ctx->pos += n_steps;
+  ctx->pending = out_tokens[n_steps - 1];
+  return KIE_OK;
+}
+
+extern "C" int kie_decode(kie_ctx *ctx, int32_t n_steps, int32_t *out_tokens) {
+  return kie_decode_ex(ctx, n_steps, nullptr, out_tokens, nullptr);
+}
+
+extern "C" int kie_destroy(kie_ctx *ctx) {
+  if (!ctx) return KIE_ERR_INVALID;
+  if (ctx->stream) cudaStreamSynchronize(ctx->stream);
+  free_ctx(ctx);
+  return KIE_OK;
+}
+
+extern "C" const char *kie_strerror(int status) {
+  static thread_local std::string msg;
+  const char *base = "unknown status";
+  switch (status) {
+    case KIE_OK: base = "ok"; break;
+    case KIE_ERR_INVALID: base = "invalid argument"; break;
+    case KIE_ERR_OOM: base = "out of device memory"; break;
+    case KIE_ERR_CUDA: base = "CUDA error"; break;
+    case KIE_ERR_CAPACITY: base = "KV capacity exceeded"; break;
+    case KIE_ERR_NOT_RESIDENT: base = "persistent grid cannot be co-resident"; break;
+    case KIE_ERR_DEVICE_TIMEOUT: base = "device watchdog timeout"; break;
+    case KIE_ERR_POISONED: base = "context poisoned by an earlier device error"; break;
+  }
+  msg = base;
+  if (!g_last_error.empty() && status != KIE_OK) msg += ": " + g_last_error;
+  return msg.c_str();
+}
+
+extern "C" int kie_get_stats(const kie_ctx *ctx, kie_stats *out) {
+  if (!ctx || !out) return KIE_ERR_INVALID;
+  const Plan &P = ctx->plan;
+  memset(out, 0, sizeof *out);
+  out->n_ctas = P.n_ctas;
+  out->threads_per_cta = monokernel_threads();
+  out->ring_slots = P.ring_slots;
+  out->slot_bytes = kSlotBytes;
+  out->smem_bytes = int32_t(P.smem);
+  out->pos = ctx->pos;
+  out->weight_bytes_per_step = P.weight_bytes_per_step;
+  out->kv_bytes_per_position = int64_t(2) * ctx->m.n_layers * ctx->m.n_kv_heads * ctx->m.head_dim * 2;
+  out->last_kernel_ms = ctx->last_ms;
+  out->last_launch_steps = ctx->last_steps;
+  out->pending_token = ctx->pending;
+  return KIE_OK;
+}
+
+extern "C" int kie_copy_kv(const kie_ctx *ctx, int32_t layer, int32_t kv_head, int32_t pos0,
+                           int32_t n, uint16_t *k_out, uint16_t *v_out) {
+  if (!ctx) return KIE_ERR_INVALID;
+  const kie_model_desc &m = ctx->m;
+  if (layer < 0 || layer >= m.n_layers || kv_head < 0 || kv_head >= m.n_kv_heads || pos0 < 0 ||
+      n < 0 || int64_t(pos0) + n > m.max_seq)
+    return KIE_ERR_INVALID;
+  const size_t off = ((size_t(layer) * m.n_kv_heads + kv_head) * m.max_seq + pos0) * m.head_dim;
+  const size_t bytes = size_t(n) * m.head_dim * 2;
+  kie_ctx *c = const_cast<kie_ctx *>(ctx);
+  cudaError_t e = cudaSuccess;
+  if (k_out && e == cudaSuccess) e = cudaMemcpyAsync(k_out, ctx->kcache + off, bytes, cudaMemcpyDeviceToHost, ctx->stream);
+  if (v_out && e == cudaSuccess) e = cudaMemcpyAsync(v_out, ctx->vcache + off, bytes, cudaMemcpyDeviceToHost, ctx->stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(ctx->stream);
+  if (e != cudaSuccess) return cuda_fail(c, "kv copy", e);
+  return KIE_OK;
+}
+
+extern "C" int kie_debug_set(kie_ctx *ctx, int32_t watchdog_ms, int32_t skip_signal_cta) {
+  if (!ctx || watchdog_ms < 1) return KIE_ERR_INVALID;
+  ctx->watchdog_ns = uint64_t(watchdog_ms) * 1000000ull;
+  ctx->skip_signal_cta = skip_signal_cta;
+  return KIE_OK;
+}

@@ -1,0 +1,144 @@
+/*
+ * kie.h -- C ABI of the persistent batch-1 decode library (libkie.so).
+ *
+ * What it computes.  One single-request decode path of a pre-norm decoder,
+ * run as ONE persistent kernel: every layer of every step back to back, with
+ * no kernel launch between layers or tokens, the sampled token fed straight
+ * back on the device ("monokernel" bullet of the Kog Inference Engine
+ * write-ups: the entire decode path as one persistent kernel with no launches
+ * between layers; "Software versus silicon" section: prefill, decode and
+ * LM-head sampling in one go, with grid synchronisations and per-launch
+ * overhead removed).  Per step: embedding gather, RMSNorm, fused QKV GEMV,
+ * rotate-half RoPE, KV-cache append, grouped-query attention over the cache,
+ * O GEMV + residual, RMSNorm, gate/up GEMV + SwiGLU, down GEMV + residual,
+ * final RMSNorm, LM-head GEMV, greedy argmax (lowest index on ties).  Lane
+ * models (lane-structured transformer bullet: 8 parallel lanes; Delayed Tensor
+ * Parallelism bullet: each cross-lane sum delayed by delta layers) run every
+ * sublayer per lane slice and add  M_i u_i  to the residual at the start of
+ * layer i + delta (pending sums are added before the final norm).
+ *
+ * Precision: weights and KV cache in the storage dtype (FP16 per the pages'
+ * results table, or bfloat16); activations, accumulators and logits fp32.
+ *
+ * Conventions for every call:
+ *   - returns KIE_OK (0) or a negative kie_status; kie_strerror() names it;
+ *   - calls are synchronous: they return after the work queued on the
+ *     context's stream has finished;
+ *   - after KIE_ERR_DEVICE_TIMEOUT or KIE_ERR_CUDA the context is poisoned:
+ *     every later call except kie_destroy returns the same error.
+ *   - a context is not thread-safe; use one per host thread.
+ */
+#ifndef KIE_H
+#define KIE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KIE_OK = 0,
+  KIE_ERR_INVALID = -1,        /* bad descriptor, null pointer or argument */
+  KIE_ERR_OOM = -2,            /* device allocation failed */
+  KIE_ERR_CUDA = -3,           /* a CUDA call failed (message via kie_strerror) */
+  KIE_ERR_CAPACITY = -4,       /* pos + n would exceed max_seq */
+  KIE_ERR_NOT_RESIDENT = -5,   /* the persistent grid cannot be co-resident */
+  KIE_ERR_DEVICE_TIMEOUT = -6, /* a bounded in-kernel wait ran out (watchdog) */
+  KIE_ERR_POISONED = -7        /* an earlier device error poisoned this context */
+} kie_status;
+
+typedef enum { KIE_F16 = 0, KIE_BF16 = 1 } kie_dtype;
+
+/* Model shape.  Dense models: n_lanes = 1 and n_heads * head_dim == d_model.
+ * Lane models: every per-lane size is the total divided by n_lanes
+ * (lane width d_model/n_lanes, n_heads/n_lanes query heads, n_kv_heads/n_lanes
+ * KV heads, ffn_dim/n_lanes hidden units), lane_delay >= 2.
+ * Requirements: n_heads % n_kv_heads == 0; head_dim in {64, 128};
+ * d_model, ffn_dim (per lane) multiples of 8. */
+typedef struct {
+  int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, ffn_dim, vocab;
+  float rms_eps, rope_theta;
+  int32_t dtype;      /* kie_dtype: weights and KV cache */
+  int32_t n_lanes;    /* 1 = dense */
+  int32_t lane_delay; /* delta, layers; used when n_lanes > 1 */
+  int32_t max_seq;    /* KV capacity in positions (prompt + decode) */
+} kie_model_desc;
+
+typedef struct kie_ctx kie_ctx;
+
+/* Build a context on the current CUDA device.
+ *   weights: DEVICE pointer to all weights in the canonical layout (storage
+ *     dtype, row-major [out, in], concatenated, no padding):
+ *       embed[V,d];
+ *       per layer, per lane: attn_norm[dl], wq[Hql*dh,dl], wk[Hkvl*dh,dl],
+ *         wv[Hkvl*dh,dl], wo[dl,Hql*dh], ffn_norm[dl], w_gate[Fl,dl],
+ *         w_up[Fl,dl], w_down[dl,Fl];  lane models then mix[d,d];
+ *       final_norm[d], lm_head[V,d].
+ *     Borrowed for this call only: the library copies the weights into its
+ *     own per-SM streaming layout, so the caller may free them on return.
+ *   stream: cudaStream_t to run on (NULL = legacy default stream).
+ *   out: receives the context (owner: caller, release with kie_destroy). */
+int kie_create(const kie_model_desc *desc, const void *weights, void *stream, kie_ctx **out);
+
+/* Process a prompt from position 0 (the KV cache is reset and its unused
+ * slots filled with NaN) and return the greedy next token, the argmax of the
+ * logits at position n-1.
+ *   tokens: HOST array of n ids in [0, vocab); next_token: HOST out. */
+int kie_prefill(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_token);
+
+/* Greedy decode: step k feeds the pending token at position pos+k, appends
+ * its K/V, and the argmax of its logits becomes out_tokens[k] and the next
+ * pending token.  The first pending token is kie_prefill's next_token.
+ *   out_tokens: HOST array of n_steps. */
+int kie_decode(kie_ctx *ctx, int32_t n_steps, int32_t *out_tokens);
+
+/* kie_decode with options:
+ *   forced_tokens: HOST array of n_steps ids, or NULL.  When given, step k
+ *     feeds forced_tokens[k] instead of the pending token (teacher forcing);
+ *     out_tokens still receives each step's argmax.
+ *   logits_out: DEVICE fp32 array [n_steps, vocab], or NULL. */
+int kie_decode_ex(kie_ctx *ctx, int32_t n_steps, const int32_t *forced_tokens,
+                  int32_t *out_tokens, float *logits_out);
+
+/* Release every resource of the context (valid on a poisoned context). */
+int kie_destroy(kie_ctx *ctx);
+
+/* Static text for a kie_status; for KIE_ERR_CUDA and KIE_ERR_DEVICE_TIMEOUT
+ * it includes the detail of the most recent error in this process. */
+const char *kie_strerror(int status);
+
+/* Facts about a context, for measurement. */
+typedef struct {
+  int32_t n_ctas;             /* persistent CTAs (one per SM) */
+  int32_t threads_per_cta;
+  int32_t ring_slots;         /* shared-memory weight ring depth */
+  int32_t slot_bytes;
+  int32_t smem_bytes;         /* dynamic shared memory per CTA */
+  int32_t pos;                /* next position to be written */
+  int64_t weight_bytes_per_step; /* weights one decode step streams (incl. LM head) */
+  int64_t kv_bytes_per_position; /* K+V bytes per cached position, all layers */
+  float last_kernel_ms;       /* device time of the most recent launch (CUDA events) */
+  int32_t last_launch_steps;  /* steps run by that launch */
+  int32_t pending_token;
+} kie_stats;
+
+int kie_get_stats(const kie_ctx *ctx, kie_stats *out);
+
+/* Copy n cached positions [pos0, pos0 + n) of one layer and KV head to the
+ * host, as raw storage words: k_out and v_out are HOST arrays of n*head_dim
+ * uint16 (either may be NULL).  Positions never written hold NaN words. */
+int kie_copy_kv(const kie_ctx *ctx, int32_t layer, int32_t kv_head, int32_t pos0, int32_t n,
+                uint16_t *k_out, uint16_t *v_out);
+
+/* Test hooks for the device watchdog (no effect unless called).
+ *   watchdog_ms: limit of every in-kernel wait (default 2000, env KIE_WATCHDOG_MS).
+ *   skip_signal_cta: if >= 0, that CTA never signals the first stage of the
+ *     next launch, so the other CTAs' waits must run out and the call must
+ *     return KIE_ERR_DEVICE_TIMEOUT.  Reset to -1 after one launch. */
+int kie_debug_set(kie_ctx *ctx, int32_t watchdog_ms, int32_t skip_signal_cta);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KIE_H */

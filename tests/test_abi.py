@@ -1,0 +1,77 @@
+"""The C-ABI library loads, exports every function include/kie.h declares, and
+rejects bad descriptors on the host (no GPU needed: validation runs before any
+CUDA call)."""
+import ctypes
+import subprocess
+
+import pytest
+
+import decode_persistent_monokernel_b200 as kie
+from decode_persistent_monokernel_b200 import build as kbuild
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kie.load()
+
+
+def test_exports_every_declared_function(lib):
+    names = kie.header_functions()
+    assert {"kie_create", "kie_prefill", "kie_decode", "kie_decode_ex", "kie_destroy",
+            "kie_strerror"} <= set(names)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", kie.LIB_PATH], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(lib, n)
+
+
+def test_build_targets_sm100a_only():
+    flags = " ".join(kbuild.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+    assert flags.count("-gencode") == 1
+
+
+def _desc(**kw):
+    base = dict(n_layers=2, d_model=256, n_heads=4, n_kv_heads=4, head_dim=64, ffn_dim=704,
+                vocab=4096, rms_eps=1e-5, rope_theta=1e4, dtype=0, n_lanes=1, lane_delay=0,
+                max_seq=64)
+    base.update(kw)
+    return kie.kie_model_desc(*[base[f] for f, _ in kie.kie_model_desc._fields_])
+
+
+@pytest.mark.parametrize("bad", [
+    dict(head_dim=96, d_model=384),      # head_dim must be 64 or 128
+    dict(n_kv_heads=3),                  # heads not a multiple of kv heads
+    dict(d_model=264),                   # n_heads * head_dim != d_model
+    dict(dtype=7),
+    dict(n_lanes=2, lane_delay=1),       # delay must be >= 2
+    dict(n_lanes=3),                     # lanes must divide the sizes
+    dict(ffn_dim=700),                   # not a multiple of 8
+    dict(max_seq=0),
+    dict(n_heads=8, n_kv_heads=1, d_model=512),  # more than 4 q heads per kv head
+])
+def test_invalid_descriptors_rejected(lib, bad):
+    h = ctypes.c_void_p()
+    rc = lib.kie_create(ctypes.byref(_desc(**bad)), ctypes.c_void_p(16), None, ctypes.byref(h))
+    assert rc == kie.KIE_ERR_INVALID
+    assert not h.value
+
+
+def test_null_and_misaligned_weights_rejected(lib):
+    h = ctypes.c_void_p()
+    assert lib.kie_create(ctypes.byref(_desc()), None, None, ctypes.byref(h)) == kie.KIE_ERR_INVALID
+    assert lib.kie_create(ctypes.byref(_desc()), ctypes.c_void_p(18), None,
+                          ctypes.byref(h)) == kie.KIE_ERR_INVALID
+    assert lib.kie_create(None, ctypes.c_void_p(16), None, ctypes.byref(h)) == kie.KIE_ERR_INVALID
+
+
+def test_null_context_calls_rejected(lib):
+    assert lib.kie_prefill(None, None, 1, None) == kie.KIE_ERR_INVALID
+    assert lib.kie_decode(None, 1, None) == kie.KIE_ERR_INVALID
+    assert lib.kie_destroy(None) == kie.KIE_ERR_INVALID
+    assert lib.kie_get_stats(None, None) == kie.KIE_ERR_INVALID
+    assert "invalid" in kie.strerror(kie.KIE_ERR_INVALID)
+    assert "watchdog" in kie.strerror(kie.KIE_ERR_DEVICE_TIMEOUT)

@@ -1,0 +1,272 @@
+"""CUDA path vs the float64 oracle, element by element, through the C ABI.
+
+Acceptance (per step): logits relative L2 <= 1e-3 and max-abs <= 2e-2; the
+greedy token equal to the oracle's wherever the oracle's top-2 margin is at
+least 2e-2 (free runs compare up to the first near tie; teacher-forced runs
+compare every step); the KV cache written at exactly positions [0, pos) and
+NaN beyond.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import synth
+from oracle import Oracle
+from oracle.numerics import storage_to_f64
+from synth.configs import ModelShape
+from tests.gpu_util import (check_argmax, check_logits, free_run_prefix, make_decoder)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import decode_persistent_monokernel_b200 as kie
+    kie.load()
+    return torch
+
+
+def _gpu_logits(dec, n, vocab, forced):
+    import torch
+    z = torch.empty((n, vocab), dtype=torch.float32, device="cuda")
+    toks = dec.kie_decode_ex(n, forced=forced, logits_out=z)
+    torch.cuda.synchronize()
+    return toks, z.cpu().numpy()
+
+
+def _check_kv(dec, orc, m, upto, max_seq):
+    """Positions [0, upto) hold the oracle's rounded K/V (to rounding), the
+    rest still hold the NaN poison."""
+    for l in range(m.n_layers):
+        for g in range(m.n_kv_heads):
+            k, v = dec.kie_copy_kv(l, g, 0, max_seq)
+            kf, vf = storage_to_f64(k, m.dtype), storage_to_f64(v, m.dtype)
+            assert np.isfinite(kf[:upto]).all() and np.isfinite(vf[:upto]).all()
+            assert np.isnan(kf[upto:]).all() and np.isnan(vf[upto:]).all()
+            for got, want in ((kf[:upto], orc.K[l, g, :upto]), (vf[:upto], orc.V[l, g, :upto])):
+                scale = np.abs(want).max() + 1e-30
+                assert np.abs(got - want).max() <= 4e-3 * scale, (l, g)
+
+
+def _teacher_forced(m, bits, prompt, forced, label, cache_f64=False):
+    """Prefill + teacher-forced decode on the GPU, logits compared every step."""
+    P, N = len(prompt), len(forced)
+    dec = make_decoder(m, bits, P + N + 4)
+    t0 = dec.kie_prefill(prompt)
+    toks, z = _gpu_logits(dec, N, m.vocab, forced)
+    orc = Oracle(m, bits, P + N + 4, cache_f64=cache_f64)
+    z_ora = orc.teacher_forced_logits(prompt, forced)
+    rel, mab = check_logits(z, z_ora, label)
+    near = check_argmax(toks, z_ora, label)
+    return dec, orc, t0, rel, mab, near
+
+
+# ------------------------------------------------------------ tiny decoder, full protocol
+def test_tiny_free_run_teacher_forced_and_cache():
+    w = synth.WORKLOADS[0]
+    m = w.model
+    bits = synth.generate_weights(m, w.weight_seed)
+    prompt = synth.prompt(w)
+    P, N = w.prompt_len, w.decode_len
+    max_seq = P + N + 8
+    orc = Oracle(m, bits, max_seq)
+    t0, z0 = orc.prefill(prompt)
+    toks, zs = orc.decode(N)
+    dec = make_decoder(m, bits, max_seq)
+    g0 = dec.kie_prefill(prompt)
+    check_argmax([g0], z0, "prefill")
+    gt = dec.kie_decode(N)
+    free_run_prefix(np.concatenate([[g0], gt]), np.concatenate([[t0], toks]),
+                    np.vstack([z0, zs]), "tiny free run")
+    st = dec.kie_get_stats()
+    assert st.pos == P + N and st.pending_token == gt[-1]
+    # teacher-forced along the oracle's own greedy path, logits every step
+    forced = np.concatenate([[t0], toks[:-1]]).astype(np.int32)
+    assert dec.kie_prefill(prompt) == g0
+    gt2, z = _gpu_logits(dec, N, m.vocab, forced)
+    check_logits(z, zs, "tiny teacher-forced")
+    check_argmax(gt2, zs, "tiny teacher-forced")
+    orc2 = Oracle(m, bits, max_seq)
+    orc2.teacher_forced_logits(prompt, forced)
+    _check_kv(dec, orc2, m, P + N, max_seq)
+    dec.kie_destroy()
+
+
+def test_tiny_is_deterministic():
+    w = synth.WORKLOADS[0]
+    m = w.model
+    bits = synth.generate_weights(m, w.weight_seed)
+    prompt = synth.prompt(w)
+    forced = synth.forced_tokens(w, 24)
+    runs = []
+    for _ in range(2):
+        dec = make_decoder(m, bits, 64)
+        dec.kie_prefill(prompt)
+        runs.append(_gpu_logits(dec, 24, m.vocab, forced)[1])
+        dec.kie_destroy()
+    np.testing.assert_array_equal(runs[0].view(np.uint32), runs[1].view(np.uint32))
+
+
+_TINY = synth.WORKLOADS[0].model
+_VARIANTS = {
+    "gqa2_gains": _TINY.replace(n_kv_heads=2, gain_std=0.1, n_layers=3),
+    "gqa4": _TINY.replace(n_heads=4, n_kv_heads=1, n_layers=2),
+    "bf16": _TINY.replace(dtype="bf16", rope_theta=500000.0),
+    "lanes2_d2": _TINY.replace(n_lanes=2, lane_delay=2, n_layers=4, mix_std=0.02, gain_std=0.1),
+    "lanes4_d3": _TINY.replace(n_lanes=4, lane_delay=3, n_layers=5, mix_std=0.02),
+    "dh128": ModelShape(n_layers=2, d_model=512, n_heads=4, n_kv_heads=2, head_dim=128,
+                        ffn_dim=1376, vocab=5000, dtype="f16"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(_VARIANTS))
+def test_small_variants(name):
+    m = _VARIANTS[name]
+    bits = synth.generate_weights(m, 31)
+    prompt = synth.generate_tokens(13, m.vocab, 5)
+    forced = synth.generate_tokens(40, m.vocab, 6)
+    _teacher_forced(m, bits, prompt, forced, name)
+    # free run against the oracle's greedy path
+    dec = make_decoder(m, bits, 64)
+    orc = Oracle(m, bits, 64)
+    t0, z0 = orc.prefill(prompt)
+    toks, zs = orc.decode(20)
+    g0 = dec.kie_prefill(prompt)
+    gt = dec.kie_decode(20)
+    free_run_prefix(np.concatenate([[g0], gt]), np.concatenate([[t0], toks]),
+                    np.vstack([z0, zs]), name)
+
+
+# ------------------------------------------------------------ full-size workloads
+@pytest.fixture(scope="module")
+def dense_2b():
+    w = synth.WORKLOADS[1]
+    return synth.generate_weights(w.model, w.weight_seed)
+
+
+@pytest.mark.parametrize("cid", [1, 2])
+def test_full_size_teacher_forced(cid, dense_2b):
+    """Every step of the benchmarked launch shape (prompt P, N decode steps in
+    one launch) compared with the oracle on a seeded forced-token sequence."""
+    w = synth.WORKLOADS[cid]
+    m = w.model
+    bits = dense_2b if cid == 1 else synth.generate_weights(m, w.weight_seed)
+    prompt = synth.prompt(w)
+    forced = synth.forced_tokens(w, w.decode_len)
+    dec, orc, t0, rel, mab, near = _teacher_forced(m, bits, prompt, forced, f"cfg{cid}",
+                                                   cache_f64=True)
+    print(f"cfg{cid}: rel-L2 {rel:.3g} max-abs {mab:.3g} near ties {near}/{w.decode_len}")
+    # free run: the first steps against the oracle's own greedy path
+    n_free = 6
+    g0 = dec.kie_prefill(prompt)
+    gt = dec.kie_decode(n_free)
+    ot0, oz0 = orc.prefill(prompt)
+    otoks, ozs = orc.decode(n_free)
+    free_run_prefix(np.concatenate([[g0], gt]), np.concatenate([[ot0], otoks]),
+                    np.vstack([oz0, ozs]), f"cfg{cid} free run")
+    dec.kie_destroy()
+
+
+def _first_layers(m: ModelShape, bits: np.ndarray, n_layers: int):
+    """Weights of the same model truncated to its first n_layers layers."""
+    spec = {t.name: t for t in synth.tensor_table(m)}
+    first_after = spec["final_norm"].offset
+    sub = m.replace(n_layers=n_layers)
+    layer_end = synth.tensor_table(sub)[-3].offset + synth.tensor_table(sub)[-3].numel
+    out = np.concatenate([bits[:layer_end], bits[first_after:]])
+    assert out.size == synth.total_elements(sub)
+    return sub, out
+
+
+def test_long_context_two_layers(dense_2b):
+    """The long-context workload's shapes (8192-token prompt, 256 decode steps)
+    on the first two layers of the 2.3B-class model."""
+    w = synth.WORKLOADS[3]
+    m, bits = _first_layers(w.model, dense_2b, 2)
+    prompt = synth.prompt(w)
+    forced = synth.forced_tokens(w, w.decode_len)
+    _, _, _, rel, mab, near = _teacher_forced(m, bits, prompt, forced, "long-2L")
+    print(f"long-2L: rel-L2 {rel:.3g} max-abs {mab:.3g} near ties {near}")
+
+
+def test_long_context_full_model_properties(dense_2b):
+    """The full long-context workload: 8192-token prefill then 256 greedy steps.
+    Layer 0's cached K/V depend only on each token and its position, so the
+    oracle checks them at every position; the rest must be finite and the
+    cache must be written exactly up to the current position."""
+    w = synth.WORKLOADS[3]
+    m = w.model
+    prompt = synth.prompt(w)
+    P, N = w.prompt_len, w.decode_len
+    max_seq = P + N + 16
+    dec = make_decoder(m, dense_2b, max_seq)
+    t0 = dec.kie_prefill(prompt)
+    toks = dec.kie_decode(N)
+    assert 0 <= t0 < m.vocab and ((toks >= 0) & (toks < m.vocab)).all()
+    seq = np.concatenate([prompt, [t0], toks[:-1]])
+    m1, b1 = _first_layers(m, dense_2b, 1)
+    orc = Oracle(m1, b1, max_seq)
+    orc.forward(list(seq), logits="none")
+    for g in range(m.n_kv_heads):
+        k, v = dec.kie_copy_kv(0, g, 0, max_seq)
+        kf, vf = storage_to_f64(k, m.dtype), storage_to_f64(v, m.dtype)
+        L = P + N
+        assert np.isnan(kf[L:]).all() and np.isnan(vf[L:]).all()
+        for got, want in ((kf[:L], orc.K[0, g, :L]), (vf[:L], orc.V[0, g, :L])):
+            assert np.abs(got - want).max() <= 4e-3 * np.abs(want).max()
+    for l in (1, m.n_layers // 2, m.n_layers - 1):
+        k, v = dec.kie_copy_kv(l, 3, 0, max_seq)
+        assert np.isfinite(storage_to_f64(k[:P + N], m.dtype)).all()
+        assert np.isnan(storage_to_f64(k[P + N:], m.dtype)).all()
+    dec.kie_destroy()
+
+
+def test_8b_class_two_layers():
+    """The 8B-class workload's shapes (bf16, d 4096, 32x128 / 8 KV heads,
+    F 14336, V 128256; prompt 1024 -> 256 steps) on its first two layers."""
+    w = synth.WORKLOADS[4]
+    m = w.model.replace(n_layers=2)
+    bits = synth.generate_weights(m, w.weight_seed)
+    prompt = synth.prompt(w)
+    forced = synth.forced_tokens(w, w.decode_len)
+    _, _, _, rel, mab, near = _teacher_forced(m, bits, prompt, forced, "8b-2L", cache_f64=True)
+    print(f"8b-2L: rel-L2 {rel:.3g} max-abs {mab:.3g} near ties {near}")
+
+
+@pytest.mark.skipif(os.environ.get("KIE_SLOW") != "1", reason="set KIE_SLOW=1 (minutes of CPU)")
+def test_8b_class_full_model():
+    w = synth.WORKLOADS[4]
+    m = w.model
+    bits = synth.generate_weights(m, w.weight_seed)
+    prompt = synth.prompt(w)
+    forced = synth.forced_tokens(w, 16)
+    _teacher_forced(m, bits, prompt, forced, "8b-full", cache_f64=False)
+
+
+# ------------------------------------------------------------ host-side errors
+def test_errors_and_capacity():
+    import decode_persistent_monokernel_b200 as kie
+    w = synth.WORKLOADS[0]
+    m = w.model
+    bits = synth.generate_weights(m, w.weight_seed)
+    dec = make_decoder(m, bits, 20)
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_decode(1)                          # nothing prefilled yet
+    assert e.value.code == kie.KIE_ERR_INVALID
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_prefill(np.array([1, 2, m.vocab], dtype=np.int32))
+    assert e.value.code == kie.KIE_ERR_INVALID
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_prefill(np.zeros(21, dtype=np.int32))
+    assert e.value.code == kie.KIE_ERR_CAPACITY
+    dec.kie_prefill(np.arange(15, dtype=np.int32))
+    dec.kie_decode(5)
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_decode(1)
+    assert e.value.code == kie.KIE_ERR_CAPACITY
+    # the context is still usable after host-side rejections
+    assert dec.kie_prefill(np.arange(3, dtype=np.int32)) >= 0
+    dec.kie_destroy()
