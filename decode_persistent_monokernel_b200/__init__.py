@@ -72,6 +72,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kie_prefill": ([_P, _P, _I, ctypes.POINTER(_I)], _I),
         "kie_decode": ([_P, _I, _P], _I),
         "kie_decode_ex": ([_P, _I, _P, _P, _P], _I),
+        "kie_decode_ex_static": ([_P, _I, _P, _P, _P], _I),
         "kie_destroy": ([_P], _I),
         "kie_strerror": ([_I], ctypes.c_char_p),
         "kie_get_stats": ([_P, ctypes.POINTER(kie_stats)], _I),
@@ -149,6 +150,15 @@ class Decoder:
         f = None if forced is None else np.ascontiguousarray(forced, dtype=np.int32)
         _check(load().kie_decode_ex(self._h, n_steps, None if f is None else f.ctypes.data,
                                     out.ctypes.data, _ptr(logits_out)))
+        return out
+
+    def kie_decode_ex_static(self, n_steps: int, forced=None, logits_out=None):
+        """kie_decode_ex with the kernel scratch in the library's fixed device array."""
+        import numpy as np
+        out = np.empty(n_steps, dtype=np.int32)
+        f = None if forced is None else np.ascontiguousarray(forced, dtype=np.int32)
+        _check(load().kie_decode_ex_static(self._h, n_steps, None if f is None else f.ctypes.data,
+                                           out.ctypes.data, _ptr(logits_out)))
         return out
 
     def kie_get_stats(self) -> kie_stats:

@@ -14,6 +14,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -691,5 +692,142 @@ extern "C" int kie_debug_set(kie_ctx *ctx, int32_t watchdog_ms, int32_t skip_sig
   if (!ctx || watchdog_ms < 1) return KIE_ERR_INVALID;
   ctx->watchdog_ns = uint64_t(watchdog_ms) * 1000000ull;
   ctx->skip_signal_cta = skip_signal_cta;
+  return KIE_OK;
+}
+
+// ---------------------------------------------------------------- decode without allocation
+// kie_decode_ex_static: the same decode as kie_decode_ex, but the persistent
+// kernel's per-launch scratch (activation vectors, attention partials, the
+// epoch counters, argmax keys, token staging) lives in this fixed array that
+// the library's device image carries, instead of in buffers of the context.
+// The call itself makes no device or host allocation: it only copies, sets
+// memory and launches.  One array per GPU, held from module load until the
+// process exits; every call on that GPU reuses it.
+namespace {
+constexpr size_t kStaticScratchBytes = size_t(1) << 20;   // 1 MiB
+constexpr int kStaticMaxDevices = 64;
+}  // namespace
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+static void *g_static_scratch_dev[kStaticMaxDevices];
+static std::mutex g_static_scratch_mu;
+
+// Device address of g_static_scratch on `device` (the current device).  The
+// symbol's name is only a host-side handle, so the address is looked up once
+// per device with cudaGetSymbolAddress and cached.
+static int static_scratch_address(int device, void **out) {
+  if (device < 0 || device >= kStaticMaxDevices) {
+    g_last_error = "device index beyond the static scratch table";
+    return KIE_ERR_INVALID;
+  }
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_dev[device]) {
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p) {
+      set_error("cudaGetSymbolAddress(static scratch)", e);
+      return KIE_ERR_CUDA;
+    }
+    g_static_scratch_dev[device] = p;
+  }
+  *out = g_static_scratch_dev[device];
+  return KIE_OK;
+}
+
+extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t *forced_tokens,
+                                    int32_t *out_tokens, float *logits_out) {
+  if (!ctx || !out_tokens || n_steps < 1) return KIE_ERR_INVALID;
+  if (ctx->poisoned) return KIE_ERR_POISONED;
+  if (!forced_tokens && ctx->pending < 0) return KIE_ERR_INVALID;
+  if (int64_t(ctx->pos) + n_steps > ctx->m.max_seq) return KIE_ERR_CAPACITY;
+  if (forced_tokens)
+    for (int i = 0; i < n_steps; ++i)
+      if (forced_tokens[i] < 0 || forced_tokens[i] >= ctx->m.vocab) return KIE_ERR_INVALID;
+  const kie_model_desc &m = ctx->m;
+  const Plan &P = ctx->plan;
+  // carve the scratch: counters | keys | forced tokens | out tokens | activations
+  auto up = [](size_t b) { return (b + 255) / 256 * 256; };
+  const size_t sync_bytes = size_t(SY_ATTN0 + m.n_kv_heads) * kSyncStride * 4;
+  const size_t o_keys = up(sync_bytes);
+  const size_t o_tin = o_keys + up(size_t(n_steps) * 8);
+  const size_t o_tout = o_tin + up(size_t(n_steps) * 4);
+  const size_t o_act = o_tout + up(size_t(n_steps) * 4);
+  const size_t need = o_act + ctx->act_floats * 4;
+  if (need > kStaticScratchBytes) {
+    char buf[200];
+    snprintf(buf, sizeof buf,
+             "static scratch too small: this model and %d steps need %zu bytes, the fixed "
+             "maximum is %zu",
+             n_steps, need, kStaticScratchBytes);
+    g_last_error = buf;
+    return KIE_ERR_CAPACITY;
+  }
+  void *base = nullptr;
+  int device = -1;
+  cudaError_t e = cudaGetDevice(&device);
+  if (e != cudaSuccess) return cuda_fail(ctx, "cudaGetDevice", e);
+  if (device != ctx->device) {
+    g_last_error = "the context's device is not the current device";
+    return KIE_ERR_INVALID;
+  }
+  if (int rc = static_scratch_address(device, &base)) return rc;
+  uint8_t *s = static_cast<uint8_t *>(base);
+  float *act = reinterpret_cast<float *>(s + o_act);
+
+  KernelArgs a{};
+  a.n_layers = m.n_layers; a.d_model = m.d_model; a.n_heads = m.n_heads;
+  a.n_kv_heads = m.n_kv_heads; a.head_dim = m.head_dim; a.ffn_dim = m.ffn_dim; a.vocab = m.vocab;
+  a.n_lanes = m.n_lanes; a.lane_delay = m.n_lanes > 1 ? m.lane_delay : 1;
+  a.lane_width = m.d_model / m.n_lanes; a.lane_heads = m.n_heads / m.n_lanes;
+  a.lane_kv_heads = m.n_kv_heads / m.n_lanes; a.lane_ffn = m.ffn_dim / m.n_lanes;
+  a.rms_eps = m.rms_eps;
+  a.attn_scale = float(1.0 / sqrt(double(m.head_dim)));
+  a.max_seq = m.max_seq;
+  a.n_ctas = P.n_ctas; a.ring_slots = P.ring_slots;
+  a.vbuf_floats = P.vbuf_floats; a.part_floats = P.part_floats;
+  for (int k = 0; k < ST_COUNT; ++k) a.shape[k] = P.shape[k];
+  a.stage_cta = ctx->d_stage_cta; a.blocks = ctx->d_blocks;
+  a.cta_blk_begin = ctx->d_blk_begin; a.cta_stream_off = ctx->d_stream_off;
+  a.wstream = ctx->wstream; a.embed = ctx->embed;
+  a.gain_attn = ctx->gains; a.gain_ffn = ctx->gains + size_t(m.n_layers) * m.d_model;
+  a.gain_final = ctx->gains + size_t(2 * m.n_layers) * m.d_model;
+  a.rope_cs = ctx->rope; a.kcache = ctx->kcache; a.vcache = ctx->vcache;
+  a.x = act + ctx->off_x; a.qkv = act + ctx->off_qkv; a.attn_o = act + ctx->off_o;
+  a.hbuf = act + ctx->off_h; a.ubuf = act + ctx->off_u; a.dsum = act + ctx->off_dsum;
+  a.attn_part = act + ctx->off_part; a.max_split = P.max_split;
+  a.sync = reinterpret_cast<uint32_t *>(s);
+  a.keys = reinterpret_cast<unsigned long long *>(s + o_keys);
+  a.pos0 = ctx->pos; a.n_steps = n_steps; a.first_token = ctx->pending;
+  a.forced = forced_tokens ? reinterpret_cast<const int32_t *>(s + o_tin) : nullptr;
+  a.logits_every_step = 1;
+  a.out_tokens = reinterpret_cast<int32_t *>(s + o_tout);
+  a.logits_out = logits_out;
+  a.watchdog_ns = ctx->watchdog_ns;
+  a.skip_signal_cta = -1;
+
+  cudaStream_t st = ctx->stream;
+  // the counters and the argmax keys must start at zero on every call
+  if (forced_tokens)
+    CK(cudaMemcpyAsync(s + o_tin, forced_tokens, size_t(n_steps) * 4, cudaMemcpyHostToDevice, st));
+  CK(cudaMemsetAsync(s, 0, o_tin, st));
+  void *args[] = {&a};
+  CK(cudaEventRecord(ctx->ev0, st));
+  CK(cudaLaunchCooperativeKernel(monokernel_fn(m.dtype), dim3(P.n_ctas), dim3(monokernel_threads()),
+                                 args, P.smem, st));
+  CK(cudaEventRecord(ctx->ev1, st));
+  uint32_t status = 0;
+  CK(cudaMemcpyAsync(&status, s + SY_STATUS * kSyncStride * 4, 4, cudaMemcpyDeviceToHost, st));
+  CK(cudaMemcpyAsync(out_tokens, s + o_tout, size_t(n_steps) * 4, cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  CK(cudaEventElapsedTime(&ctx->last_ms, ctx->ev0, ctx->ev1));
+  ctx->last_steps = n_steps;
+  if (status != 0) {
+    char buf[160];
+    snprintf(buf, sizeof buf, "device watchdog: a bounded wait ran out (code 0x%x)", status);
+    g_last_error = buf;
+    ctx->poisoned = KIE_ERR_DEVICE_TIMEOUT;
+    return KIE_ERR_DEVICE_TIMEOUT;
+  }
+  ctx->pos += n_steps;
+  ctx->pending = out_tokens[n_steps - 1];
   return KIE_OK;
 }

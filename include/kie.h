@@ -101,6 +101,27 @@ int kie_decode(kie_ctx *ctx, int32_t n_steps, int32_t *out_tokens);
 int kie_decode_ex(kie_ctx *ctx, int32_t n_steps, const int32_t *forced_tokens,
                   int32_t *out_tokens, float *logits_out);
 
+/* kie_decode_ex without any allocation.  The pages have no counterpart to
+ * this call; it exists for callers that may not allocate device memory at the
+ * time they decode (for example a serving thread under a fixed device-memory
+ * budget that reserved everything at start-up, or one that must never enter
+ * the CUDA allocator because an allocation can block behind device-wide work).
+ * Same arguments, semantics and context state as kie_decode_ex; the kernel's
+ * per-launch scratch (activation vectors, attention partials, epoch counters,
+ * argmax keys, token staging) comes from one fixed 1 MiB array in the
+ * library's device image instead of the context's buffers.
+ *   - every GPU that loads the library holds that 1 MiB until the process exits;
+ *   - the array's device address is looked up (cudaGetSymbolAddress) on the
+ *     first call on each device, with that device current; make that first
+ *     call before any stream capture;
+ *   - calls whose scratch would not fit (large models or very long n_steps)
+ *     return KIE_ERR_CAPACITY, and kie_strerror gives the sizes;
+ *   - every call on a GPU shares the one array, which keeps the last call's
+ *     contents (the counters and keys are cleared at the start of each call):
+ *     calls that overlap on that GPU, from any context or stream, race. */
+int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t *forced_tokens,
+                         int32_t *out_tokens, float *logits_out);
+
 /* Release every resource of the context (valid on a poisoned context). */
 int kie_destroy(kie_ctx *ctx);
 

@@ -1,0 +1,66 @@
+"""kie_decode_ex_static, the decode call that allocates nothing.
+
+It serves callers that may not allocate device memory while they decode; its
+kernel scratch is the library's fixed device array.  It must give what
+kie_decode_ex gives on the same context state, call after call (the array
+keeps the previous call's contents, so two calls in a row are compared).
+This file is collected last so that a failure here comes after every other
+test has run.
+"""
+import numpy as np
+import pytest
+
+import synth
+from tests.gpu_util import check_logits, make_decoder
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(dec, fn, prompt, forced, chunks, vocab):
+    import torch
+    dec.kie_prefill(prompt)
+    toks, zs = [], []
+    s = 0
+    for n in chunks:
+        z = torch.empty((n, vocab), dtype=torch.float32, device="cuda")
+        f = None if forced is None else forced[s:s + n]
+        toks.append(fn(n, forced=f, logits_out=z))
+        torch.cuda.synchronize()
+        zs.append(z.cpu().numpy())
+        s += n
+    return np.concatenate(toks), np.vstack(zs)
+
+
+@pytest.mark.parametrize("teacher_forced", [True, False])
+def test_static_scratch_decode_matches_decode_ex(teacher_forced):
+    import torch
+    assert torch.cuda.is_available()
+    w = synth.WORKLOADS[0]
+    m = w.model
+    bits = synth.generate_weights(m, w.weight_seed)
+    prompt = synth.prompt(w)
+    forced = synth.forced_tokens(w, 24) if teacher_forced else None
+    dec = make_decoder(m, bits, 64)
+    chunks = (10, 14)                       # two calls in a row
+    t_ref, z_ref = _run(dec, dec.kie_decode_ex, prompt, forced, chunks, m.vocab)
+    t_new, z_new = _run(dec, dec.kie_decode_ex_static, prompt, forced, chunks, m.vocab)
+    np.testing.assert_array_equal(t_new, t_ref)
+    check_logits(z_new, z_ref, "static scratch")
+    assert dec.kie_get_stats().pos == len(prompt) + sum(chunks)
+    dec.kie_destroy()
+
+
+def test_static_scratch_rejects_oversize():
+    import decode_persistent_monokernel_b200 as kie
+    w = synth.WORKLOADS[0]
+    m = w.model
+    bits = synth.generate_weights(m, w.weight_seed)
+    dec = make_decoder(m, bits, 200000)
+    dec.kie_prefill(synth.prompt(w))
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_decode_ex_static(150000)   # argmax keys alone exceed the fixed array
+    assert e.value.code == kie.KIE_ERR_CAPACITY
+    assert "static scratch" in str(e.value)
+    # the context is unharmed: a fitting call still works
+    assert len(dec.kie_decode_ex_static(4)) == 4
+    dec.kie_destroy()
