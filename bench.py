@@ -45,7 +45,36 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="bounded CPU work for the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="run the profiling build (libkie_prof.so) and report where each "
+                         "SM's time goes; its timings are not the benchmark value")
     return ap.parse_args()
+
+
+PROF_NAMES = ["total", "wait_other_sms", "gemv", "wait_tiles", "attention", "staging_norm",
+              "stage_barrier", "lm_head", "producer_ring_full", "producer_total"]
+
+
+def profile_summary(prof, steps, mhz):
+    """Per-step microseconds per activity: mean and max over SMs."""
+    import numpy as np
+    cyc = prof.astype(np.float64)
+    us = cyc / (mhz * 1e6) * 1e6 / steps
+    out = {}
+    for i, name in enumerate(PROF_NAMES):
+        out[name] = {"mean_us": round(float(us[:, i].mean()), 2),
+                     "max_us": round(float(us[:, i].max()), 2)}
+    tot = us[:, 0].mean()
+    out["sync_share"] = round(float(us[:, 1].mean() / tot), 4) if tot > 0 else None
+    out["dependency_waits_per_step"] = round(float(prof[:, 11].mean() / steps), 1)
+    stages = ["qkv", "o", "gate_up", "down", "mix", "lm_head"]
+    out["gemv_by_stage_us"] = {n: round(float(us[:, 12 + i].mean()), 1) for i, n in enumerate(stages)}
+    gates = ["qkv_done", "attn_merged", "o_done", "gate_up_done", "down_done", "mix_flush", "token"]
+    out["wait_by_counter_us"] = {n: round(float(us[:, 18 + i].mean()), 1) for i, n in enumerate(gates)}
+    out["wait_by_counter_min_us"] = {n: round(float(us[:, 18 + i].min()), 1) for i, n in enumerate(gates)}
+    out["tiles_per_step"] = round(float(prof[:, 10].mean() / steps), 1)
+    out["clock_mhz_used"] = mhz
+    return out
 
 
 def peak_hbm():
@@ -175,7 +204,7 @@ def main():
         return
 
     import decode_persistent_monokernel_b200 as kie
-    kie.load()
+    kie.load(kie.PROF_LIB_PATH if args.profile else kie.LIB_PATH)
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
@@ -256,7 +285,11 @@ def main():
         "kernel": {"ctas": st.n_ctas, "threads": st.threads_per_cta, "ring_slots": st.ring_slots,
                    "smem_bytes": st.smem_bytes},
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if args.profile:
+        mhz = line["clocks"]["sm_mhz"] or 1965
+        line["profile"] = profile_summary(dec.kie_get_profile(), K, mhz)
+        line["profile_build"] = "libkie_prof.so (activity counters on): not the benchmark value"
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         dec.kie_destroy()
         rate, n, el, cores = oracle_decode_rate(w, bits, args.cpu_seconds)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,

@@ -13,6 +13,7 @@ import re
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libkie.so")
+PROF_LIB_PATH = os.path.join(HERE, "libkie_prof.so")   # built with -DKIE_PROFILE
 HEADER = os.path.join(os.path.dirname(HERE), "include", "kie.h")
 
 KIE_OK = 0
@@ -78,6 +79,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kie_get_stats": ([_P, ctypes.POINTER(kie_stats)], _I),
         "kie_copy_kv": ([_P, _I, _I, _I, _I, _P, _P], _I),
         "kie_debug_set": ([_P, _I, _I], _I),
+        "kie_get_profile": ([_P, _P, _I], _I),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -172,6 +174,14 @@ class Decoder:
         v = np.empty((n, self.desc.head_dim), dtype=np.uint16)
         _check(load().kie_copy_kv(self._h, layer, kv_head, pos0, n, k.ctypes.data, v.ctypes.data))
         return k, v
+
+    def kie_get_profile(self):
+        """Per-SM activity counters [n_ctas, 32] of the last launch (profiling build)."""
+        import numpy as np
+        n = self.kie_get_stats().n_ctas
+        out = np.zeros((n, 32), dtype=np.uint64)
+        _check(load().kie_get_profile(self._h, out.ctypes.data, out.size))
+        return out
 
     def kie_debug_set(self, watchdog_ms: int, skip_signal_cta: int = -1) -> None:
         _check(load().kie_debug_set(self._h, watchdog_ms, skip_signal_cta))

@@ -11,6 +11,7 @@ CSRC = os.path.join(HERE, "csrc")
 SOURCES = ["kie_api.cu", "monokernel.cu"]
 HEADERS = ["kie_internal.h", os.path.join("..", "..", "include", "kie.h")]
 LIB = os.path.join(HERE, "libkie.so")
+PROF_LIB = os.path.join(HERE, "libkie_prof.so")  # activity counters compiled in
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -27,28 +28,37 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, s) for s in SOURCES + HEADERS]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"),
+def _build_one(lib: str, extra, force: bool, verbose: bool) -> str:
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"),
            *[os.path.join(CSRC, s) for s in SOURCES], "-o", tmp]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         sys.stderr.write(res.stderr)
-    os.replace(tmp, LIB)
-    with open(os.path.join(HERE, "ptxas_info.txt"), "w") as f:
-        f.write(res.stderr)
+    os.replace(tmp, lib)
+    if lib == LIB:
+        with open(os.path.join(HERE, "ptxas_info.txt"), "w") as f:
+            f.write(res.stderr)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False, profile: bool = True) -> str:
+    """Builds libkie.so and (unless profile=False) the profiling libkie_prof.so."""
+    _build_one(LIB, [], force, verbose)
+    if profile:
+        _build_one(PROF_LIB, ["-DKIE_PROFILE"], force, False)
     return LIB
 
 

@@ -24,6 +24,7 @@
 namespace kie {
 size_t monokernel_smem_bytes(int ring_slots, int vbuf_floats, int part_floats);
 int monokernel_threads();
+bool monokernel_profiled();
 const void *monokernel_fn(int dtype);
 cudaError_t launch_repack(const uint16_t *src, uint8_t *dst, const RepackJob *jobs, int njobs,
                           cudaStream_t st);
@@ -99,19 +100,33 @@ struct Plan {
   int64_t weight_bytes_per_step = 0;
 };
 
-StageShape make_shape(int K, int in_len, int out_len) {
-  StageShape s{};
+// Tile shape of a stage whose rows have K elements (see StageShape).  Rows
+// longer than one slot, or splits that would give a lane more than 4 chunks,
+// are rejected.
+const char *make_shape(int K, int in_len, int out_len, StageShape &s) {
+  s = StageShape{};
   s.K = K;
-  int nseg = (K + 2047) / 2048;
-  while (K % nseg != 0 || (K / nseg) % 8 != 0) ++nseg;
-  s.nseg = nseg;
-  s.KT = K / nseg;
-  int R = 16;
-  while (R > 1 && R * s.KT * 2 > kSlotBytes) R >>= 1;
-  s.R = R;
   s.in_len = in_len;
   s.out_len = out_len;
-  return s;
+  const int max_rows = kSlotBytes / (2 * K);
+  if (K % 8 || max_rows < 1) return "a weight row must be a multiple of 8 elements and fit one 32 KB slot";
+  const int limit = (K % 256 == 0) ? 64 : 16;
+  int R = 1;
+  while (R * 2 <= std::min(limit, max_rows)) R *= 2;
+  s.R = R;
+  if (R >= kConsumerWarps) {
+    s.nseg = 1;
+    s.rpw = R / kConsumerWarps;
+  } else {
+    int S = kConsumerWarps / R;
+    while (S > 1 && (K / 8) % S) S >>= 1;
+    s.nseg = S;
+    s.rpw = 1;
+  }
+  s.cps = K / 8 / s.nseg;
+  if (s.rpw * s.cps > 128) return "row split leaves more than 4 chunks per lane";
+  if (s.rpw > 1 && s.cps % 32) return "multi-row warps need rows of a multiple of 256 elements";
+  return nullptr;
 }
 
 // Row pieces of each stage in the stage's output order.
@@ -160,7 +175,7 @@ void cut_blocks(const std::vector<Piece> &pieces, int r0, int r1, bool up, int l
       B.nrows = b - a;
       B.in_off = pc.in_off;
       B.tile0 = tile;
-      tile += ((B.nrows + sh.R - 1) / sh.R) * sh.nseg;
+      tile += (B.nrows + sh.R - 1) / sh.R;
       blk.push_back(B);
       src.push_back((up ? pc.src2 : pc.src) + int64_t(a - base) * pc.K);
     }
@@ -173,12 +188,14 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
   const int nl = m.n_lanes, d = m.d_model, dh = m.head_dim;
   const bool lanes = nl > 1;
   P.n_ctas = n_ctas;
-  P.shape[ST_QKV] = make_shape(d / nl, d, (m.n_heads + 2 * m.n_kv_heads) * dh);
-  P.shape[ST_O] = make_shape(m.n_heads / nl * dh, m.n_heads * dh, d);
-  P.shape[ST_GU] = make_shape(d / nl, d, m.ffn_dim);
-  P.shape[ST_D] = make_shape(m.ffn_dim / nl, m.ffn_dim, d);
-  P.shape[ST_MIX] = make_shape(d, d, d);
-  P.shape[ST_LM] = make_shape(d, d, m.vocab);
+  const char *err = nullptr;
+  if ((err = make_shape(d / nl, d, (m.n_heads + 2 * m.n_kv_heads) * dh, P.shape[ST_QKV])) ||
+      (err = make_shape(m.n_heads / nl * dh, m.n_heads * dh, d, P.shape[ST_O])) ||
+      (err = make_shape(d / nl, d, m.ffn_dim, P.shape[ST_GU])) ||
+      (err = make_shape(m.ffn_dim / nl, m.ffn_dim, d, P.shape[ST_D])) ||
+      (err = make_shape(d, d, d, P.shape[ST_MIX])) ||
+      (err = make_shape(d, d, m.vocab, P.shape[ST_LM])))
+    return err;
 
   // per-CTA blocks of every stage kind (same for every layer)
   P.stage_cta.assign(size_t(ST_COUNT) * n_ctas, StageCta{});
@@ -235,7 +252,7 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
         j.dst_byte = off;
         j.nrows = B.nrows;
         j.K = sh.K;
-        j.KT = sh.KT;
+        j.KT = sh.K;   // tiles are whole rows: the block is copied as is
         j.R = sh.R;
         P.jobs.push_back(j);
         off += int64_t(B.nrows) * sh.K * 2;
@@ -257,15 +274,14 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
 
   // shared memory: input vector / attention scratch, partial sums, ring
   const int G = m.n_heads / m.n_kv_heads;
-  int vb = 0;
-  for (int k = 0; k < ST_COUNT; ++k) vb = std::max(vb, P.shape[k].in_len);
+  int vb = 2 * d;   // normalised inputs (and their gains) are staged in shared memory
   vb = std::max(vb, (G + 2) * dh + kConsumerWarps * G * (dh + 2));
   P.vbuf_floats = (vb + 3) / 4 * 4;
   P.part_floats = (part_max + 3) / 4 * 4;
   const size_t fixed = monokernel_smem_bytes(0, P.vbuf_floats, P.part_floats);
-  if (fixed + 4 * (kSlotBytes + 16) > smem_cap) return "shape needs more shared memory than the SM has";
+  if (fixed + 3 * (kSlotBytes + 16) > smem_cap) return "shape needs more shared memory than the SM has";
   int slots = int((smem_cap - fixed) / (kSlotBytes + 16));
-  slots = std::min(slots, 32);
+  slots = std::min(slots, 16);
   P.ring_slots = slots;
   P.smem = monokernel_smem_bytes(slots, P.vbuf_floats, P.part_floats);
   P.max_split = (n_ctas + m.n_kv_heads - 1) / m.n_kv_heads;
@@ -288,6 +304,7 @@ struct kie_ctx {
   int pending = -1;
   int poisoned = 0;   // sticky error code
   uint64_t watchdog_ns = 2000000000ull;
+  int l2_prefetch_tiles = 0;
   int skip_signal_cta = -1;
   float last_ms = 0.f;
   int last_steps = 0;
@@ -306,6 +323,7 @@ struct kie_ctx {
   Block *d_blocks = nullptr;
   int32_t *d_blk_begin = nullptr;
   int64_t *d_stream_off = nullptr;
+  unsigned long long *prof = nullptr;  // [n_ctas][kProfSlots] (profiling build)
   size_t off_x, off_qkv, off_o, off_h, off_u, off_dsum, off_part, act_floats;
   size_t kv_elems = 0;
   std::vector<int32_t> host_tokens;
@@ -326,6 +344,8 @@ static const char *validate(const kie_model_desc *m) {
     return "lane count must divide d_model, heads, kv heads and ffn_dim";
   if (m->n_heads * m->head_dim != m->d_model) return "n_heads * head_dim must equal d_model";
   if ((m->d_model / nl) % 8 || (m->ffn_dim / nl) % 8) return "lane width and lane ffn must be multiples of 8";
+  if ((m->d_model / nl) % 128) return "lane width (d_model / n_lanes) must be a multiple of 128";
+  if (m->d_model > 8192) return "d_model above 8192 is not supported";
   if (nl > 1 && m->lane_delay < 2) return "lane_delay must be >= 2";
   if (nl > 64) return "at most 64 lanes";
   if (!(m->rms_eps >= 0.f) || !(m->rope_theta > 0.f)) return "bad rms_eps or rope_theta";
@@ -348,7 +368,7 @@ static void free_ctx(kie_ctx *c) {
   if (!c) return;
   void *ptrs[] = {c->wstream, c->embed, c->gains, c->rope, c->kcache, c->vcache, c->act,
                   c->sync, c->keys, c->tokens_in, c->tokens_out, c->d_stage_cta, c->d_blocks,
-                  c->d_blk_begin, c->d_stream_off};
+                  c->d_blk_begin, c->d_stream_off, c->prof};
   for (void *p : ptrs)
     if (p) cudaFree(p);
   if (c->ev0) cudaEventDestroy(c->ev0);
@@ -391,6 +411,10 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
   if (const char *env = getenv("KIE_WATCHDOG_MS")) {
     long v = atol(env);
     if (v > 0) ctx->watchdog_ns = uint64_t(v) * 1000000ull;
+  }
+  if (const char *env = getenv("KIE_L2_PREFETCH_TILES")) {
+    long v = atol(env);
+    if (v >= 0 && v <= 64) ctx->l2_prefetch_tiles = int(v);
   }
   cudaError_t e = cudaGetDevice(&ctx->device);
   if (e != cudaSuccess) return fail(cuda_fail(nullptr, "cudaGetDevice", e));
@@ -459,6 +483,7 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
   if ((rc = alloc(ctx, (void **)&ctx->d_blocks, std::max<size_t>(1, P.blocks.size()) * sizeof(Block), "plan"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->d_blk_begin, P.cta_blk_begin.size() * 4, "plan"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->d_stream_off, P.cta_stream_off.size() * 8, "plan"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->prof, size_t(P.n_ctas) * kProfSlots * 8, "profile"))) return fail(rc);
   RepackJob *d_jobs = nullptr;
   if ((rc = alloc(ctx, (void **)&d_jobs, P.jobs.size() * sizeof(RepackJob), "repack jobs"))) return fail(rc);
 
@@ -559,6 +584,8 @@ static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int fi
   a.watchdog_ns = ctx->watchdog_ns;
   a.skip_signal_cta = ctx->skip_signal_cta;
   ctx->skip_signal_cta = -1;
+  a.l2_prefetch_tiles = ctx->l2_prefetch_tiles;
+  a.prof = ctx->prof;
 
   const size_t sync_words = size_t(SY_ATTN0 + m.n_kv_heads) * kSyncStride;
   if (forced_host)
@@ -688,6 +715,19 @@ extern "C" int kie_copy_kv(const kie_ctx *ctx, int32_t layer, int32_t kv_head, i
   return KIE_OK;
 }
 
+extern "C" int kie_get_profile(const kie_ctx *ctx, uint64_t *out, int32_t n_words) {
+  if (!ctx || !out) return KIE_ERR_INVALID;
+  if (!monokernel_profiled()) {
+    g_last_error = "not a profiling build";
+    return KIE_ERR_INVALID;
+  }
+  const int32_t need = ctx->plan.n_ctas * kProfSlots;
+  if (n_words < need) return KIE_ERR_INVALID;
+  cudaError_t e = cudaMemcpy(out, ctx->prof, size_t(need) * 8, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(const_cast<kie_ctx *>(ctx), "profile copy", e);
+  return KIE_OK;
+}
+
 extern "C" int kie_debug_set(kie_ctx *ctx, int32_t watchdog_ms, int32_t skip_signal_cta) {
   if (!ctx || watchdog_ms < 1) return KIE_ERR_INVALID;
   ctx->watchdog_ns = uint64_t(watchdog_ms) * 1000000ull;
@@ -803,6 +843,7 @@ extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t
   a.logits_out = logits_out;
   a.watchdog_ns = ctx->watchdog_ns;
   a.skip_signal_cta = -1;
+  a.l2_prefetch_tiles = ctx->l2_prefetch_tiles;
 
   cudaStream_t st = ctx->stream;
   // the counters and the argmax keys must start at zero on every call

@@ -32,12 +32,16 @@ enum SyncSlot : int {
 };
 constexpr int kSyncStride = 32;  // uint32 words per counter (128 bytes)
 
-// Per-stage constants shared by every CTA.
+// Per-stage constants shared by every CTA.  A tile is R whole rows (at most
+// kSlotBytes).  All consumer warps share every tile: warp w takes row group
+// w / nseg (rpw consecutive rows) and column split w % nseg (cps 8-element
+// chunks of each of those rows), so each lane holds at most 4 chunks.
 struct StageShape {
   int32_t K;       // reduction length of every row
-  int32_t KT;      // columns per tile segment (K % KT == 0, KT % 8 == 0)
-  int32_t nseg;    // K / KT
-  int32_t R;       // rows per tile (power of two, <= 16)
+  int32_t R;       // rows per tile (power of two)
+  int32_t nseg;    // column splits per row = partial sums per row
+  int32_t rpw;     // rows per warp (1 unless R > 16)
+  int32_t cps;     // 8-element chunks per (row, split) = K / 8 / nseg
   int32_t in_len;  // length of the stage input vector
   int32_t out_len; // length of the stage output vector
 };
@@ -67,8 +71,27 @@ struct RepackJob {
   int32_t nrows, K, KT, R;
 };
 
+// Per-SM activity counters of the profiling build (SM clock cycles).
+enum ProfSlot : int {
+  PF_TOTAL = 0,       // consumer thread 0: whole launch
+  PF_GATE = 1,        // waiting for other SMs (epoch counters)
+  PF_GEMV = 2,        // GEMV stages except the LM head (incl. ring waits)
+  PF_FULLWAIT = 3,    // warp 0: waiting for weight tiles to land (ring empty)
+  PF_ATTN = 4,        // attention (incl. the merge)
+  PF_STAGE = 5,       // input staging and RMSNorm
+  PF_SIGNAL = 6,      // end-of-stage barrier + release
+  PF_LM = 7,          // LM-head GEMV
+  PF_PROD_EMPTY = 8,  // (unused: the copy pump never blocks)
+  PF_PROD_TOTAL = 9,  // (unused)
+  PF_TILES = 10,      // weight tiles issued
+  PF_NGATE = 11,      // number of dependency waits
+  PF_GEMV_K = 12,     // 12..17: GEMV time per stage kind
+  PF_GATE_K = 18,     // 18..24: dependency-wait time per counter (SyncSlot order)
+};
+constexpr int kProfSlots = 32;
+
 constexpr int kMaxBlocksPerCta = 64;
-constexpr int kSlotBytes = 8192;
+constexpr int kSlotBytes = 32768;  // one bulk copy per tile: >= 16 KB keeps HBM saturated
 constexpr int kConsumerWarps = 16;
 
 struct KernelArgs {
@@ -113,6 +136,8 @@ struct KernelArgs {
   float *logits_out;            // device [n_steps, V] or nullptr
   uint64_t watchdog_ns;
   int32_t skip_signal_cta;      // test hook, -1 = off
+  int32_t l2_prefetch_tiles;    // tiles the producer pulls into L2 beyond the ring
+  unsigned long long *prof;     // [n_ctas][kProfSlots] (profiling build), or nullptr
 };
 
 }  // namespace kie

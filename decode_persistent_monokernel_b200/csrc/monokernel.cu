@@ -17,7 +17,7 @@
 //     attention.
 // Cross-CTA dependencies use monotonically increasing epoch counters in
 // global memory (release add / acquire load), never a full grid barrier
-// primitive.  Every spin is bounded by a %globaltimer watchdog; on expiry
+// primitive.  Every spin is bounded by an SM-clock watchdog; on expiry
 // the CTA records an error, raises the abort flag and every CTA leaves
 // after draining its in-flight copies.
 #include <cuda_bf16.h>
@@ -32,6 +32,7 @@ namespace kie {
 
 constexpr int kNC = kConsumerWarps * 32;  // consumer threads
 constexpr int kThreads = kNC + 32;        // + one producer warp
+static_assert(kNC * 4 == 2048, "staging indexes warp partial sums by element / 2048");
 
 // Device error codes written to the status word (low byte: kind).
 enum DevErr : uint32_t {
@@ -78,6 +79,9 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
@@ -137,15 +141,39 @@ __device__ __forceinline__ float dot8(uint4 w, float4 a, float4 b, float acc) {
   return acc;
 }
 
+// ------------------------------------------------------------------ profiling build
+// With -DKIE_PROFILE every SM accumulates SM-clock cycles per activity and
+// writes them to KernelArgs::prof[cta * kProfSlots + slot] at exit.
+#ifdef KIE_PROFILE
+#define KP_BEGIN(var) long long var = (tid == 0) ? clock64() : 0ll
+#define KP_END(var, slot) \
+  do { if (tid == 0) s.misc->prof[slot] += clock64() - var; } while (0)
+#else
+#define KP_BEGIN(var) do {} while (0)
+#define KP_END(var, slot) do {} while (0)
+#endif
+
 // ------------------------------------------------------------------ shared state
+// Position of the next weight tile to issue (thread 0's copy pump).
+struct PumpState {
+  const uint8_t *cur;        // next byte of this CTA's weight stream
+  uint32_t T;                // tiles issued
+  int32_t step, l, si, bi, r0, nseq;
+  int32_t seq[6];            // stage kinds of the current layer (or tail)
+  int32_t done;
+};
+
 struct Misc {
   StageCta sc[ST_COUNT];
   Block blk[kMaxBlocksPerCta];
-  float rinv[64];          // per-lane 1/rms of the staged input
+  float red_sq[4 * kConsumerWarps];  // per-warp sums of squares while staging
   float red_v[kConsumerWarps];
   int32_t red_i[kConsumerWarps];
   volatile int32_t abort;  // a consumer saw a failed wait
   int32_t flag;            // broadcast slot
+  long long prof[kProfSlots];
+  PumpState pump;   // next tile to copy into the ring
+  PumpState pf;     // next tile to prefetch into L2 (runs ahead of `pump`)
 };
 
 struct Smem {
@@ -164,17 +192,28 @@ __device__ void raise_error(const KernelArgs &a, uint32_t code) {
   atomicExch(sync_at(a, SY_ABORT), 1u);
 }
 
+// Watchdog arithmetic uses the SM cycle counter (cheap to read); the limit in
+// cycles assumes at most 2 GHz, so a wait gives up after at least watchdog_ns.
+// The shared abort flag (a global load, about a microsecond) is polled only
+// every ~64K cycles so that it never delays noticing a completed wait.
+constexpr long long kAbortPollCycles = 1 << 16;
+
 // Bounded wait until *ctr >= target.  False on watchdog expiry or abort.
+template <typename PumpT>
 __device__ bool wait_counter(const KernelArgs &a, const uint32_t *ctr, uint32_t target,
-                             uint32_t where) {
+                             uint32_t where, PumpT &&pump) {
   if (ld_acquire(ctr) >= target) return true;
-  const uint64_t t0 = globaltimer();
+  const long long t0 = clock64(), limit = (long long)a.watchdog_ns * 2;
+  long long next_poll = kAbortPollCycles;
   const uint32_t *abortp = sync_at(a, SY_ABORT);
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (ld_acquire(ctr) >= target) return true;
-    if ((it & 15) == 0) {
+    pump();
+    const long long el = clock64() - t0;
+    if (el > next_poll) {
+      next_poll = el + kAbortPollCycles;
       if (ld_relaxed(abortp)) return false;
-      if (globaltimer() - t0 > a.watchdog_ns) {
+      if (el > limit) {
         raise_error(a, DE_TIMEOUT_COUNTER | (where << 8));
         return false;
       }
@@ -183,15 +222,21 @@ __device__ bool wait_counter(const KernelArgs &a, const uint32_t *ctr, uint32_t 
 }
 
 // Bounded wait on an mbarrier phase.
-__device__ bool wait_mbar(const KernelArgs &a, uint64_t *bar, uint32_t parity, uint32_t code) {
+template <typename PumpT>
+__device__ bool wait_mbar(const KernelArgs &a, uint64_t *bar, uint32_t parity, uint32_t code,
+                          PumpT &&pump) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  const long long t0 = clock64(), limit = (long long)a.watchdog_ns * 2;
+  long long next_poll = kAbortPollCycles;
   const uint32_t *abortp = sync_at(a, SY_ABORT);
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15) == 0) {
+    pump();
+    const long long el = clock64() - t0;
+    if (el > next_poll) {
+      next_poll = el + kAbortPollCycles;
       if (ld_relaxed(abortp)) return false;
-      if (globaltimer() - t0 > a.watchdog_ns) {
+      if (el > limit) {
         raise_error(a, code);
         return false;
       }
@@ -199,72 +244,157 @@ __device__ bool wait_mbar(const KernelArgs &a, uint64_t *bar, uint32_t parity, u
   }
 }
 
-// ------------------------------------------------------------------ producer
-struct Producer {
+// ------------------------------------------------------------------ weight pump
+// Thread 0 of each CTA issues the CTA's weight tiles, in the order they are
+// consumed, into free ring slots: one cp.async.bulk (1-D bulk copy, no tensor
+// map, no multicast, L2 evict-first) per tile, completing on the slot's full
+// mbarrier.  It never blocks: pump() returns when the next slot is still in
+// use, and thread 0 calls it from every wait loop it runs (dependency gates,
+// tile waits) and after every tile, so the weight stream keeps flowing while
+// the CTA waits for other SMs -- weights do not depend on activations.
+struct Pump {
   const KernelArgs &a;
   Smem s;
-  uint32_t T = 0;          // tiles issued
-  const uint8_t *cur = nullptr;
-  uint64_t policy;
-  bool ok = true;
+  __device__ Pump(const KernelArgs &a_, Smem s_) : a(a_), s(s_) {}
 
-  __device__ Producer(const KernelArgs &a_, Smem s_) : a(a_), s(s_) { policy = policy_evict_first(); }
+  __device__ bool lm_step(int step) const { return a.logits_every_step || step == a.n_steps - 1; }
 
-  __device__ void stage(int k) {
-    if (!ok) return;
-    const StageShape sh = a.shape[k];
-    const StageCta &c = s.misc->sc[k];
-    const int NS = a.ring_slots;
-    for (int bi = 0; bi < c.nblk; ++bi) {
-      const Block b = s.misc->blk[c.blk_begin + bi];
-      for (int r0 = 0; r0 < b.nrows; r0 += sh.R) {
-        const int rows = min(sh.R, b.nrows - r0);
-        const uint32_t bytes = uint32_t(rows) * uint32_t(sh.KT) * 2u;
-        for (int sg = 0; sg < sh.nseg; ++sg) {
-          const uint32_t slot = T % NS;
-          if (T >= (uint32_t)NS) {
-            if (!wait_mbar(a, &s.empty[slot], ((T / NS) - 1) & 1, DE_TIMEOUT_EMPTY | (k << 8))) {
-              ok = false;
-              return;
-            }
-          }
-          mbar_expect_tx(&s.full[slot], bytes);
-          bulk_g2s(s.ring + size_t(slot) * kSlotBytes, cur, bytes, &s.full[slot], policy);
-          cur += bytes;
-          ++T;
-        }
-      }
+  __device__ void load_seq(PumpState &p) const {
+    p.nseq = 0;
+    const bool lanes = a.n_lanes > 1;
+    if (p.l < a.n_layers) {
+      p.seq[p.nseq++] = ST_QKV;
+      if (lanes && p.l >= 1) p.seq[p.nseq++] = ST_MIX;
+      p.seq[p.nseq++] = ST_O;
+      p.seq[p.nseq++] = ST_GU;
+      p.seq[p.nseq++] = ST_D;
+    } else if (lm_step(p.step)) {
+      if (lanes) p.seq[p.nseq++] = ST_MIX;
+      p.seq[p.nseq++] = ST_LM;
     }
   }
 
-  __device__ void run(int cta) {
-    const uint8_t *base = a.wstream + a.cta_stream_off[cta];
-    const int L = a.n_layers;
-    const bool lanes = a.n_lanes > 1;
-    for (int step = 0; step < a.n_steps && ok; ++step) {
-      const bool lm = a.logits_every_step || step == a.n_steps - 1;
-      cur = base;
-      for (int l = 0; l < L && ok; ++l) {
-        stage(ST_QKV);
-        if (lanes && l >= 1) stage(ST_MIX);
-        stage(ST_O);
-        stage(ST_GU);
-        stage(ST_D);
+  // move (si, bi, r0) forward to the next tile that exists
+  __device__ void normalize(PumpState &p, const uint8_t *base) const {
+    while (!p.done) {
+      if (p.si < p.nseq) {
+        const StageCta &c = s.misc->sc[p.seq[p.si]];
+        if (p.bi < c.nblk) {
+          if (p.r0 < s.misc->blk[c.blk_begin + p.bi].nrows) return;
+          ++p.bi;
+          p.r0 = 0;
+          continue;
+        }
+        ++p.si;
+        p.bi = 0;
+        p.r0 = 0;
+        continue;
       }
-      if (lm) {
-        if (lanes) stage(ST_MIX);
-        stage(ST_LM);
+      p.si = p.bi = p.r0 = 0;
+      if (p.l < a.n_layers) {
+        ++p.l;
+      } else {
+        ++p.step;
+        p.l = 0;
+        p.cur = base;
+        if (p.step >= a.n_steps) {
+          p.done = 1;
+          return;
+        }
       }
+      load_seq(p);
     }
-    // Leave no copy in flight: each slot holds at most one outstanding copy,
-    // the most recent one issued into it.
+  }
+
+  __device__ void init_state(PumpState &p, int cta) const {
+    p.cur = a.wstream + a.cta_stream_off[cta];
+    p.T = 0;
+    p.step = p.l = p.si = p.bi = p.r0 = 0;
+    p.done = a.n_steps > 0 ? 0 : 1;
+    load_seq(p);
+    normalize(p, p.cur);
+  }
+
+  __device__ uint32_t tile_bytes(const PumpState &p) const {
+    const int k = p.seq[p.si];
+    const StageShape &sh = a.shape[k];
+    const Block &b = s.misc->blk[s.misc->sc[k].blk_begin + p.bi];
+    return uint32_t(min(sh.R, b.nrows - p.r0)) * uint32_t(sh.K) * 2u;
+  }
+
+  __device__ void advance(PumpState &p, uint32_t bytes, const uint8_t *base) const {
+    p.cur += bytes;
+    ++p.T;
+    p.r0 += a.shape[p.seq[p.si]].R;
+    normalize(p, base);
+  }
+
+  __device__ void init(int cta) {
+    init_state(s.misc->pump, cta);
+    init_state(s.misc->pf, cta);
+  }
+
+  // Copy tiles into every free ring slot; returns when the next slot is busy.
+  __device__ void pump(int cta) {
+    PumpState &p = s.misc->pump;
     const uint32_t NS = a.ring_slots;
+    const uint8_t *base = a.wstream + a.cta_stream_off[cta];
+    while (!p.done) {
+      const uint32_t slot = p.T % NS;
+      if (p.T >= NS && !mbar_try_wait(&s.empty[slot], ((p.T / NS) - 1) & 1)) return;
+      const uint32_t bytes = tile_bytes(p);
+      mbar_expect_tx(&s.full[slot], bytes);
+      bulk_g2s(s.ring + size_t(slot) * kSlotBytes, p.cur, bytes, &s.full[slot], policy_evict_first());
+      advance(p, bytes, base);
+    }
+  }
+
+  // While the ring is full, pull the next l2_prefetch_tiles tiles into L2 so
+  // that HBM keeps streaming and the ring refills from L2 once slots free up.
+  __device__ void prefetch(int cta) {
+    PumpState &q = s.misc->pf;
+    const uint32_t T = s.misc->pump.T;
+    const uint8_t *base = a.wstream + a.cta_stream_off[cta];
+    while (!q.done && q.T < T + uint32_t(a.l2_prefetch_tiles)) {
+      const uint32_t bytes = tile_bytes(q);
+      if (q.T >= T) prefetch_l2(q.cur, bytes);
+      advance(q, bytes, base);
+    }
+  }
+
+  // The producer warp's loop: fill free slots, prefetch ahead into L2, then
+  // sleep on the next slot's empty barrier until every consumer warp released
+  // it (bounded by the watchdog).
+  __device__ void run(int cta) {
+    init(cta);
+    PumpState &p = s.misc->pump;
+    const uint32_t NS = a.ring_slots;
+    while (!p.done) {
+      pump(cta);
+      if (p.done) break;
+      prefetch(cta);
+      const uint32_t slot = p.T % NS;
+#ifdef KIE_PROFILE
+      const long long tw = clock64();
+#endif
+      if (!wait_mbar(a, &s.empty[slot], ((p.T / NS) - 1) & 1, DE_TIMEOUT_EMPTY, [] {})) break;
+#ifdef KIE_PROFILE
+      s.misc->prof[PF_PROD_EMPTY] += clock64() - tw;
+#endif
+    }
+    drain();
+  }
+
+  // Before the CTA exits: each slot holds at most one outstanding copy, the
+  // last one issued into it; wait (bounded) until those have landed.
+  __device__ void drain() {
+    const uint32_t NS = a.ring_slots, T = s.misc->pump.T;
     const uint32_t first = T > NS ? T - NS : 0;
     for (uint32_t t = first; t < T; ++t) {
       if (!mbar_try_wait(&s.full[t % NS], (t / NS) & 1)) {
-        const uint64_t t0 = globaltimer();
+        const long long t0 = clock64();
         while (!mbar_try_wait(&s.full[t % NS], (t / NS) & 1)) {
-          if (globaltimer() - t0 > a.watchdog_ns) break;
+          if (clock64() - t0 > (long long)a.watchdog_ns * 2) break;
         }
       }
     }
@@ -278,6 +408,7 @@ struct Consumer {
   Smem s;
   const int tid, warp, lane, cta;
   uint32_t Tbase = 0;   // tiles consumed before the current stage
+  uint32_t slot = 0, phase = 0;   // ring position of the next tile (every warp sees every tile)
   int step = 0, l = 0, tok = 0, p = 0;
   uint32_t lm_count = 0;
 
@@ -289,19 +420,25 @@ struct Consumer {
   // thread 0 waits for a counter, everyone learns the outcome
   __device__ bool gate(int slot, uint32_t target, uint32_t where) {
     if (tid == 0) {
-      if (!wait_counter(a, sync_at(a, slot), target, where)) s.misc->abort = 1;
-      __threadfence();
+#ifdef KIE_PROFILE
+      const long long t0 = clock64();
+#endif
+      if (!wait_counter(a, sync_at(a, slot), target, where, [] {})) s.misc->abort = 1;
+#ifdef KIE_PROFILE
+      s.misc->prof[PF_GATE] += clock64() - t0;
+      s.misc->prof[PF_GATE_K + slot] += clock64() - t0;
+      s.misc->prof[PF_NGATE] += 1;
+#endif
     }
     cbar();
     return !aborted();
   }
 
   __device__ void signal(int slot) {
+    KP_BEGIN(t_sig);
     cbar();
-    if (tid == 0) {
-      __threadfence();
-      red_release_add(sync_at(a, slot), 1u);
-    }
+    if (tid == 0) red_release_add(sync_at(a, slot), 1u);
+    KP_END(t_sig, PF_SIGNAL);
   }
 
   // ---- stage inputs
@@ -313,109 +450,193 @@ struct Consumer {
     return v;
   }
 
-  // vbuf = RMSNorm of vbuf (already holding the raw input) with `gain`,
-  // per lane slice of width `seg`.
-  __device__ void norm_vbuf(const float *gain, int n, int seg) {
-    float *v = s.vbuf;
-    const int nseg = n / seg;
-    cbar();
-    if (nseg == 1) {
-      float acc = 0.f;
-      for (int i = tid; i < n; i += kNC) acc = fmaf(v[i], v[i], acc);
-      for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) s.misc->red_v[warp] = acc;
-      cbar();
-      if (tid == 0) {
-        float t = 0.f;
-        for (int w = 0; w < kConsumerWarps; ++w) t += s.misc->red_v[w];
-        s.misc->rinv[0] = rsqrtf(t / float(n) + a.rms_eps);
-      }
+  // elements 4j..4j+3 of the residual entering the current layer
+  __device__ float4 xin4(int j) const {
+    float4 v;
+    if (l == 0) {
+      const uint2 w = *reinterpret_cast<const uint2 *>(a.embed + size_t(tok) * a.d_model + 4 * j);
+      const float2 lo = Store<T>::pair(w.x), hi = Store<T>::pair(w.y);
+      v = make_float4(lo.x, lo.y, hi.x, hi.y);
     } else {
-      for (int sgi = warp; sgi < nseg; sgi += kConsumerWarps) {
-        float acc = 0.f;
-        for (int i = lane; i < seg; i += 32) acc = fmaf(v[sgi * seg + i], v[sgi * seg + i], acc);
-        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) s.misc->rinv[sgi] = rsqrtf(acc / float(seg) + a.rms_eps);
+      v = __ldcg(reinterpret_cast<const float4 *>(a.x) + j);
+    }
+    if (a.n_lanes > 1 && l >= a.lane_delay) {
+      const float4 q = __ldcg(reinterpret_cast<const float4 *>(
+                                  a.dsum + size_t((l - a.lane_delay) % a.lane_delay) * a.d_model) + j);
+      v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
+    }
+    return v;
+  }
+
+  // vbuf[0..n) = RMSNorm(src) * gain, per lane slice of width seg (a
+  // multiple of 128).  src(i4) returns elements 4*i4 .. 4*i4+3.  Each thread
+  // holds up to 4 float4 groups; warp partial sums of squares go through
+  // shared memory and every thread adds up the ones of its own slice.
+  template <typename Src>
+  __device__ void stage_norm(Src src, const float *gain, int n, int seg) {
+    KP_BEGIN(t_norm);
+    const int ng = n >> 2;
+    float4 *vb = reinterpret_cast<float4 *>(s.vbuf);
+    float4 *gb = vb + ng;   // the gains, staged beside the input
+    for (int q = 0; q * kNC < ng; ++q) {
+      const int j = tid + q * kNC;
+      float ss = 0.f;
+      if (j < ng) {
+        const float4 v = src(j);
+        gb[j] = *reinterpret_cast<const float4 *>(gain + 4 * j);
+        vb[j] = v;
+        ss = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      }
+      for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) s.misc->red_sq[q * kConsumerWarps + warp] = ss;
+    }
+    cbar();
+    for (int q = 0; q * kNC < ng; ++q) {
+      const int j = tid + q * kNC;
+      if (j < ng) {
+        // the slice holding element 4j covers warps' 128-element ranges
+        // e = e0, e0 + 128, ...; range e was summed into red_sq[e / 2048 * 16 + e % 2048 / 128]
+        const int e0 = (4 * j) / seg * seg;
+        float tot = 0.f;
+        for (int e = e0; e < e0 + seg; e += 128) tot += s.misc->red_sq[(e >> 11) * kConsumerWarps + ((e >> 7) & 15)];
+        const float r = rsqrtf(tot / float(seg) + a.rms_eps);
+        const float4 g = gb[j];
+        const float4 v = vb[j];
+        vb[j] = make_float4(v.x * r * g.x, v.y * r * g.y, v.z * r * g.z, v.w * r * g.w);
       }
     }
     cbar();
-    for (int i = tid; i < n; i += kNC) v[i] = v[i] * s.misc->rinv[i / seg] * gain[i];
-    cbar();
-  }
-
-  __device__ void load_vbuf(const float *src, int n) {
-    for (int i = tid; i < n; i += kNC) s.vbuf[i] = __ldcg(src + i);
-    cbar();
+    KP_END(t_norm, PF_STAGE);
   }
 
   // ---- GEMV over the stage's tiles: partial sums into s.part
-  template <int R>
-  __device__ void tile_dot(const uint8_t *tile, const float *vin, int KT, int rows, int nseg,
-                           int prow, int sg) {
-    const int nch = KT >> 3;
-    const uint4 *w4 = reinterpret_cast<const uint4 *>(tile);
-    const float4 *v4 = reinterpret_cast<const float4 *>(vin);
-    float acc[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) acc[r] = 0.f;
-    for (int c = lane; c < nch; c += 32) {
-      const float4 va = v4[2 * c], vb = v4[2 * c + 1];
-#pragma unroll
-      for (int r = 0; r < R; ++r)
-        if (r < rows) acc[r] = dot8<T>(w4[r * nch + c], va, vb, acc[r]);
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      float v = acc[r];
-      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      acc[r] = v;
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int r = 0; r < R; ++r)
-        if (r < rows) s.part[(prow + r) * nseg + sg] = acc[r];
-    }
+  // Every consumer warp waits on every tile in order and handles its row group
+  // and column split; its slice of the input vector stays in registers for
+  // the whole block.  `vin` is the stage input (shared or global memory).
+  __device__ void gemv(int k, const float *vin, bool vin_global) {
+    if (a.shape[k].rpw > 1) gemv_impl<true>(k, vin, vin_global);
+    else gemv_impl<false>(k, vin, vin_global);
   }
 
-  __device__ void gemv(int k) {
+  template <bool MULTI>
+  __device__ void gemv_impl(int k, const float *vin, bool vin_global) {
+    KP_BEGIN(t_gemv);
     const StageShape sh = a.shape[k];
     const StageCta &c = s.misc->sc[k];
-    const uint32_t NS = a.ring_slots;
+    const int rg = warp / sh.nseg, split = warp - rg * sh.nseg;
+    const int row0 = rg * sh.rpw;               // first row of this warp inside a tile
+    const bool active = row0 < sh.R;
+    const int nchunk = sh.rpw * sh.cps;         // chunks this warp covers per tile (<= 128)
+    // Per-lane chunk layout, the same for every tile of the stage: byte offset
+    // inside the tile, row inside the tile (INT_MAX if unused), input column.
+    uint32_t off[4];
+    int crow[4], ccol[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int ci = lane + 32 * i;
+      const int rr = ci / sh.cps, cc = ci - rr * sh.cps;
+      const bool valid = active && ci < nchunk;
+      crow[i] = valid ? row0 + rr : 0x7fffffff;
+      ccol[i] = (split * sh.cps + cc) * 8;
+      off[i] = uint32_t((row0 + rr) * sh.K + ccol[i]) * 2u;
+    }
     bool ok = !aborted();
     for (int bi = 0; bi < c.nblk && ok; ++bi) {
       const Block b = s.misc->blk[c.blk_begin + bi];
-      const int nrg = (b.nrows + sh.R - 1) / sh.R;
-      const int nt = nrg * sh.nseg;
-      int first = (warp - (b.tile0 % kConsumerWarps) + kConsumerWarps) % kConsumerWarps;
-      for (int tl = first; tl < nt; tl += kConsumerWarps) {
-        const int g = tl / sh.nseg, sg = tl - g * sh.nseg;
-        const int rows = min(sh.R, b.nrows - g * sh.R);
-        const uint32_t Tt = Tbase + b.tile0 + tl;
-        const uint32_t slot = Tt % NS;
-        bool got = true;
-        if (lane == 0) got = wait_mbar(a, &s.full[slot], (Tt / NS) & 1, DE_TIMEOUT_FULL | (k << 8));
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) {
-          s.misc->abort = 1;
-          ok = false;
-          break;
+      // this warp's slice of the input vector, kept in registers for the block
+      float vr[4][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (crow[i] != 0x7fffffff) {
+          const float *src = vin + b.in_off + ccol[i];
+          float4 x0, x1;
+          if (vin_global) { x0 = __ldcg(reinterpret_cast<const float4 *>(src)); x1 = __ldcg(reinterpret_cast<const float4 *>(src) + 1); }
+          else { x0 = reinterpret_cast<const float4 *>(src)[0]; x1 = reinterpret_cast<const float4 *>(src)[1]; }
+          vr[i][0] = x0.x; vr[i][1] = x0.y; vr[i][2] = x0.z; vr[i][3] = x0.w;
+          vr[i][4] = x1.x; vr[i][5] = x1.y; vr[i][6] = x1.z; vr[i][7] = x1.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) vr[i][e] = 0.f;
         }
-        const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes;
-        const float *vin = s.vbuf + b.in_off + sg * sh.KT;
-        const int prow = b.lrow0 + g * sh.R;
-        switch (sh.R) {
-          case 1: tile_dot<1>(tile, vin, sh.KT, rows, sh.nseg, prow, sg); break;
-          case 2: tile_dot<2>(tile, vin, sh.KT, rows, sh.nseg, prow, sg); break;
-          case 4: tile_dot<4>(tile, vin, sh.KT, rows, sh.nseg, prow, sg); break;
-          case 8: tile_dot<8>(tile, vin, sh.KT, rows, sh.nseg, prow, sg); break;
-          default: tile_dot<16>(tile, vin, sh.KT, rows, sh.nseg, prow, sg); break;
+      }
+      // Tiles go in batches of `batch` (4 / rpw) tiles: each tile's dot
+      // products are folded into one value per (tile, row) and its slot is
+      // released at once; the batch's 4 values are then reduced across the
+      // warp together (transposed butterfly: 6 shuffles for 4 values).
+      const int ntile = (b.nrows + sh.R - 1) / sh.R;
+      const int batch = MULTI ? 4 / sh.rpw : 4;
+      for (int t0 = 0; t0 < ntile && ok; t0 += batch) {
+        float val[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int bt = 0; bt < 4; ++bt) {
+          if (bt < batch && t0 + bt < ntile) {
+            bool got = true;
+#ifdef KIE_PROFILE
+            const long long tw = (tid == 0) ? clock64() : 0ll;
+#endif
+            if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [] {});
+#ifdef KIE_PROFILE
+            if (tid == 0) s.misc->prof[PF_FULLWAIT] += clock64() - tw;
+#endif
+            got = __shfl_sync(0xffffffffu, got, 0);
+            if (!got) {
+              s.misc->abort = 1;
+              ok = false;
+            } else {
+              const int rows = min(sh.R, b.nrows - (t0 + bt) * sh.R);
+              const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                if (crow[i] < rows) {
+                  const float4 va = make_float4(vr[i][0], vr[i][1], vr[i][2], vr[i][3]);
+                  const float4 vb = make_float4(vr[i][4], vr[i][5], vr[i][6], vr[i][7]);
+                  const float d = dot8<T>(*reinterpret_cast<const uint4 *>(tile + off[i]), va, vb, 0.f);
+                  // value index: tile bt of the batch, row crow[i] - row0 of the
+                  // warp's rows (uniform across lanes); < 4 because batch * rpw == 4
+                  if (!MULTI) {
+                    val[bt] += d;
+                  } else {
+                    const int vidx = bt * sh.rpw + (crow[i] - row0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                      if (j == vidx) val[j] += d;
+                  }
+                }
+              }
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&s.empty[slot]);
+              if (++slot == uint32_t(a.ring_slots)) { slot = 0; phase ^= 1u; }
+            }
+          }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.empty[slot]);
+        if (!ok) break;
+        // transposed butterfly: after it, lane l holds the warp sum of value (l >> 3) & 3
+        const bool b4 = lane & 16, b3 = lane & 8;
+        const float r0 = __shfl_xor_sync(0xffffffffu, b4 ? val[0] : val[2], 16);
+        const float r1 = __shfl_xor_sync(0xffffffffu, b4 ? val[1] : val[3], 16);
+        const float k0 = (b4 ? val[2] : val[0]) + r0;
+        const float k1 = (b4 ? val[3] : val[1]) + r1;
+        const float r2 = __shfl_xor_sync(0xffffffffu, b3 ? k0 : k1, 8);
+        float v = (b3 ? k1 : k0) + r2;
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        if (active && (lane & 7) == 0) {
+          const int vi = lane >> 3;                        // value index 0..3
+          const int bt = MULTI ? vi / sh.rpw : vi;          // tile within the batch
+          const int r = MULTI ? vi - bt * sh.rpw : 0;       // row within the warp's rows
+          const int t = t0 + bt;
+          if (t < ntile && r < sh.rpw) {
+            const int rows = min(sh.R, b.nrows - t * sh.R);
+            if (row0 + r < rows) s.part[(b.lrow0 + t * sh.R + row0 + r) * sh.nseg + split] = v;
+          }
+        }
       }
     }
     Tbase += c.ntiles;
     cbar();
+    KP_END(t_gemv, k == ST_LM ? PF_LM : PF_GEMV);
+    KP_END(t_gemv, PF_GEMV_K + k);
   }
 
   __device__ float rowsum(int i, int nseg) const {
@@ -426,6 +647,12 @@ struct Consumer {
 
   // ---- attention over the cache for one KV head group (split-KV)
   __device__ void attention() {
+    KP_BEGIN(t_attn);
+    attention_body();
+    KP_END(t_attn, PF_ATTN);
+  }
+
+  __device__ void attention_body() {
     const int dh = a.head_dim, half = dh >> 1;
     const int Hkv = a.n_kv_heads, G = a.n_heads / a.n_kv_heads;
     const int g = cta % Hkv;
@@ -551,10 +778,8 @@ struct Consumer {
     cbar();
     const uint32_t epoch = uint32_t(step) * a.n_layers + l + 1;
     if (tid == 0) {
-      __threadfence();
       const uint32_t old = atom_acq_rel_add(sync_at(a, SY_ATTN0 + g), 1u);
       s.misc->flag = (old + 1 == epoch * uint32_t(nsplit)) ? 1 : 0;
-      __threadfence();
     }
     cbar();
     if (s.misc->flag) {
@@ -611,6 +836,12 @@ struct Consumer {
   }
 
   __device__ void run() {
+    KP_BEGIN(t_total);
+    run_body();
+    KP_END(t_total, PF_TOTAL);
+  }
+
+  __device__ void run_body() {
     const int L = a.n_layers, d = a.d_model;
     const bool lanes = a.n_lanes > 1;
     const int delta = a.lane_delay;
@@ -623,9 +854,8 @@ struct Consumer {
         const uint32_t e = uint32_t(step) * L + l + 1;  // epoch of this (step, layer)
         // ---------------- RMSNorm + QKV
         if (l > 0 && !gate(SY_X2, (e - 1) * nc, 0x10 + ST_QKV)) goto done;
-        for (int i = tid; i < d; i += kNC) s.vbuf[i] = xin(i);
-        norm_vbuf(a.gain_attn + size_t(l) * d, d, a.lane_width);
-        gemv(ST_QKV);
+        stage_norm([=](int j) { return xin4(j); }, a.gain_attn + size_t(l) * d, d, a.lane_width);
+        gemv(ST_QKV, s.vbuf, false);
         if (aborted()) goto done;
         {
           const StageCta &c = s.misc->sc[ST_QKV];
@@ -635,8 +865,7 @@ struct Consumer {
         if (!(a.skip_signal_cta == cta && step == 0 && l == 0)) signal(SY_QKV);
         // ---------------- delayed cross-lane sum of the previous layer
         if (lanes && l >= 1) {
-          load_vbuf(a.ubuf + size_t((l - 1) & 1) * d, d);
-          gemv(ST_MIX);
+          gemv(ST_MIX, a.ubuf + size_t((l - 1) & 1) * d, true);
           if (aborted()) goto done;
           const StageCta &c = s.misc->sc[ST_MIX];
           const int nseg = a.shape[ST_MIX].nseg;
@@ -648,13 +877,20 @@ struct Consumer {
         attention();
         // ---------------- O + residual
         if (!gate(SY_OREADY, e * uint32_t(a.n_kv_heads), 0x30)) goto done;
-        load_vbuf(a.attn_o, a.n_heads * a.head_dim);
-        gemv(ST_O);
-        if (aborted()) goto done;
         {
+          // residual rows this CTA updates, fetched while the GEMV runs
           const StageCta &c = s.misc->sc[ST_O];
+          const float xr = tid < c.nout ? xin(c.row0 + tid) : 0.f;
+          gemv(ST_O, a.attn_o, true);
+          if (aborted()) goto done;
           const int nseg = a.shape[ST_O].nseg;
-          for (int i = tid; i < c.nout; i += kNC) {
+          if (tid < c.nout) {
+            const int r = c.row0 + tid;
+            const float v = rowsum(tid, nseg);
+            a.x[r] = xr + v;
+            if (lanes) a.ubuf[size_t(l & 1) * d + r] = v;
+          }
+          for (int i = tid + kNC; i < c.nout; i += kNC) {
             const int r = c.row0 + i;
             const float v = rowsum(i, nseg);
             a.x[r] = xin(r) + v;
@@ -664,9 +900,9 @@ struct Consumer {
         signal(SY_X1);
         // ---------------- RMSNorm + gate/up + SwiGLU
         if (!gate(SY_X1, e * nc, 0x40)) goto done;
-        for (int i = tid; i < d; i += kNC) s.vbuf[i] = __ldcg(a.x + i);
-        norm_vbuf(a.gain_ffn + size_t(l) * d, d, a.lane_width);
-        gemv(ST_GU);
+        stage_norm([=](int j) { return __ldcg(reinterpret_cast<const float4 *>(a.x) + j); },
+                   a.gain_ffn + size_t(l) * d, d, a.lane_width);
+        gemv(ST_GU, s.vbuf, false);
         if (aborted()) goto done;
         {
           const StageCta &c = s.misc->sc[ST_GU];
@@ -679,13 +915,14 @@ struct Consumer {
         signal(SY_H);
         // ---------------- down + residual
         if (!gate(SY_H, e * nc, 0x50)) goto done;
-        load_vbuf(a.hbuf, a.ffn_dim);
-        gemv(ST_D);
-        if (aborted()) goto done;
         {
           const StageCta &c = s.misc->sc[ST_D];
+          const float xr = tid < c.nout ? __ldcg(a.x + c.row0 + tid) : 0.f;
+          gemv(ST_D, a.hbuf, true);
+          if (aborted()) goto done;
           const int nseg = a.shape[ST_D].nseg;
-          for (int i = tid; i < c.nout; i += kNC) {
+          if (tid < c.nout && !lanes) a.x[c.row0 + tid] = xr + rowsum(tid, nseg);
+          for (int i = (lanes ? tid : tid + kNC); i < c.nout; i += kNC) {
             const int r = c.row0 + i;
             const float v = rowsum(i, nseg);
             a.x[r] = __ldcg(a.x + r) + v;
@@ -702,8 +939,7 @@ struct Consumer {
         if (!gate(SY_X2, (uint32_t(step) * L + L) * nc, 0x60)) goto done;
         if (lanes) {
           // the last layer's delayed sum, flushed before the final norm
-          load_vbuf(a.ubuf + size_t((L - 1) & 1) * d, d);
-          gemv(ST_MIX);
+          gemv(ST_MIX, a.ubuf + size_t((L - 1) & 1) * d, true);
           if (aborted()) goto done;
           const StageCta &c = s.misc->sc[ST_MIX];
           const int nseg = a.shape[ST_MIX].nseg;
@@ -712,15 +948,18 @@ struct Consumer {
           signal(SY_MIXF);
           if (!gate(SY_MIXF, lm_count * nc, 0x70)) goto done;
         }
-        for (int i = tid; i < d; i += kNC) {
-          float v = __ldcg(a.x + i);
-          if (lanes)
-            for (int li = (L > delta ? L - delta : 0); li < L; ++li)
-              v += __ldcg(a.dsum + size_t(li % delta) * d + i);
-          s.vbuf[i] = v;
-        }
-        norm_vbuf(a.gain_final, d, d);
-        gemv(ST_LM);
+        stage_norm(
+            [=](int j) {
+              float4 v = __ldcg(reinterpret_cast<const float4 *>(a.x) + j);
+              if (lanes)
+                for (int li = (L > delta ? L - delta : 0); li < L; ++li) {
+                  const float4 q = __ldcg(reinterpret_cast<const float4 *>(a.dsum + size_t(li % delta) * d) + j);
+                  v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
+                }
+              return v;
+            },
+            a.gain_final, d, d);
+        gemv(ST_LM, s.vbuf, false);
         if (aborted()) goto done;
         lm_epilogue();
         signal(SY_TOK);
@@ -757,27 +996,38 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
       mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], 1);
+      mbar_init(&s.empty[i], kConsumerWarps);
     }
     s.misc->abort = 0;
     s.misc->flag = 0;
+    for (int i = 0; i < kProfSlots; ++i) s.misc->prof[i] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
   if (tid >= kNC) {
     if (tid == kNC) {
-      Producer pr(a, s);
-      pr.run(cta);
+#ifdef KIE_PROFILE
+      const long long t0 = clock64();
+#endif
+      Pump pm(a, s);
+      pm.run(cta);
+#ifdef KIE_PROFILE
+      s.misc->prof[PF_PROD_TOTAL] += clock64() - t0;
+      s.misc->prof[PF_TILES] = s.misc->pump.T;
+#endif
     }
     __syncwarp();
   } else {
     Consumer<T> c(a, s, tid, cta);
     c.run();
-    // a consumer that gave up makes sure the producer stops too
+    // a CTA that gave up makes every other CTA (and its own producer) leave
     if (tid == 0 && c.aborted()) atomicExch(sync_at(a, SY_ABORT), 1u);
   }
   __syncthreads();
+#ifdef KIE_PROFILE
+  if (a.prof && tid < kProfSlots) a.prof[size_t(cta) * kProfSlots + tid] = s.misc->prof[tid];
+#endif
 }
 
 // ------------------------------------------------------------------ weight repack
@@ -810,6 +1060,14 @@ size_t monokernel_smem_bytes(int ring_slots, int vbuf_floats, int part_floats) {
 }
 
 int monokernel_threads() { return kThreads; }
+
+bool monokernel_profiled() {
+#ifdef KIE_PROFILE
+  return true;
+#else
+  return false;
+#endif
+}
 
 const void *monokernel_fn(int dtype) {
   return dtype == 0 ? reinterpret_cast<const void *>(&monokernel<__half>)

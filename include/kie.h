@@ -152,6 +152,17 @@ int kie_get_stats(const kie_ctx *ctx, kie_stats *out);
 int kie_copy_kv(const kie_ctx *ctx, int32_t layer, int32_t kv_head, int32_t pos0, int32_t n,
                 uint16_t *k_out, uint16_t *v_out);
 
+/* Per-SM activity counters of the most recent launch, in SM clock cycles:
+ * out[cta * 32 + slot] for slots 0 total, 1 waiting on other SMs, 2 GEMV
+ * stages, 3 waiting for weight tiles, 4 attention, 5 input staging and norm,
+ * 6 end-of-stage barrier, 7 LM head, 8 producer blocked on a full ring,
+ * 9 producer total, 10 tiles issued, 11 dependency waits, 12..17 GEMV time
+ * per stage (QKV, O, gate/up, down, mix, LM head), 18..24 waiting time per
+ * counter.  Only the profiling build (libkie_prof.so, compiled with
+ * KIE_PROFILE) records them; the normal build returns KIE_ERR_INVALID.
+ * n_words must be >= 32 * n_ctas. */
+int kie_get_profile(const kie_ctx *ctx, uint64_t *out, int32_t n_words);
+
 /* Test hooks for the device watchdog (no effect unless called).
  *   watchdog_ms: limit of every in-kernel wait (default 2000, env KIE_WATCHDOG_MS).
  *   skip_signal_cta: if >= 0, that CTA never signals the first stage of the

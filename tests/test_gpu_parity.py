@@ -116,7 +116,9 @@ _VARIANTS = {
     "gqa4": _TINY.replace(n_heads=4, n_kv_heads=1, n_layers=2),
     "bf16": _TINY.replace(dtype="bf16", rope_theta=500000.0),
     "lanes2_d2": _TINY.replace(n_lanes=2, lane_delay=2, n_layers=4, mix_std=0.02, gain_std=0.1),
-    "lanes4_d3": _TINY.replace(n_lanes=4, lane_delay=3, n_layers=5, mix_std=0.02),
+    "lanes4_d3": ModelShape(n_layers=5, d_model=1024, n_heads=8, n_kv_heads=8, head_dim=128,
+                            ffn_dim=2048, vocab=5000, dtype="f16", n_lanes=4, lane_delay=3,
+                            mix_std=0.02),
     "dh128": ModelShape(n_layers=2, d_model=512, n_heads=4, n_kv_heads=2, head_dim=128,
                         ffn_dim=1376, vocab=5000, dtype="f16"),
 }
