@@ -24,6 +24,9 @@ KIE_ERR_CAPACITY = -4
 KIE_ERR_NOT_RESIDENT = -5
 KIE_ERR_DEVICE_TIMEOUT = -6
 KIE_ERR_POISONED = -7
+KIE_ERR_NONFINITE = -8
+KIE_SYNC_DEPENDENCY = 0
+KIE_SYNC_GRID = 1
 KIE_F16 = 0
 KIE_BF16 = 1
 
@@ -79,6 +82,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kie_get_stats": ([_P, ctypes.POINTER(kie_stats)], _I),
         "kie_copy_kv": ([_P, _I, _I, _I, _I, _P, _P], _I),
         "kie_debug_set": ([_P, _I, _I], _I),
+        "kie_set_sync_mode": ([_P, _I], _I),
         "kie_get_profile": ([_P, _P, _I], _I),
     }
     for name, (args, res) in sig.items():
@@ -185,6 +189,9 @@ class Decoder:
 
     def kie_debug_set(self, watchdog_ms: int, skip_signal_cta: int = -1) -> None:
         _check(load().kie_debug_set(self._h, watchdog_ms, skip_signal_cta))
+
+    def kie_set_sync_mode(self, mode: int) -> None:
+        _check(load().kie_set_sync_mode(self._h, mode))
 
     def kie_destroy(self) -> None:
         if self._h:

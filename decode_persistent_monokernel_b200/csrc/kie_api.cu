@@ -43,10 +43,13 @@ static void set_error(const char *what, cudaError_t e) {
 // ---------------------------------------------------------------- canonical layout
 namespace {
 
-struct Piece {          // rows of one canonical matrix inside a stage's row space
-  int64_t src;          // element offset of the piece's first row in layer 0
-  int64_t src2;         // second source (up rows of a gate/up piece), or -1
-  int32_t rows, K, in_off;
+// Rows of one stage's per-CTA row space that come from one canonical matrix.
+struct Piece {
+  int64_t src;      // canonical element offset (layer 0) of the first row, or of
+                    // the first column's top element for transposed pieces
+  int64_t src2;     // second source (up rows of a gate/up piece), or -1
+  int32_t rows, K, in_off, out_off;
+  int32_t trans, ld;  // transposed pieces: rows are columns of a [K, ld] matrix
 };
 
 struct Layout {
@@ -100,9 +103,7 @@ struct Plan {
   int64_t weight_bytes_per_step = 0;
 };
 
-// Tile shape of a stage whose rows have K elements (see StageShape).  Rows
-// longer than one slot, or splits that would give a lane more than 4 chunks,
-// are rejected.
+// Tile shape of a row stage whose rows have K elements (see StageShape).
 const char *make_shape(int K, int in_len, int out_len, StageShape &s) {
   s = StageShape{};
   s.K = K;
@@ -129,43 +130,39 @@ const char *make_shape(int K, int in_len, int out_len, StageShape &s) {
   return nullptr;
 }
 
-// Row pieces of each stage in the stage's output order.
-void stage_pieces(const kie_model_desc &m, const Layout &Ly, int k, std::vector<Piece> &out) {
-  out.clear();
-  const int nl = m.n_lanes, d = m.d_model, dh = m.head_dim;
-  const int dl = d / nl, hq = m.n_heads / nl, hkv = m.n_kv_heads / nl, fl = m.ffn_dim / nl;
-  auto lane = [&](int ln) { return Ly.layer0 + int64_t(ln) * Ly.lane_stride; };
-  switch (k) {
-    case ST_QKV:
-      for (int ln = 0; ln < nl; ++ln) out.push_back({lane(ln) + Ly.wq, -1, hq * dh, dl, ln * dl});
-      for (int ln = 0; ln < nl; ++ln) out.push_back({lane(ln) + Ly.wk, -1, hkv * dh, dl, ln * dl});
-      for (int ln = 0; ln < nl; ++ln) out.push_back({lane(ln) + Ly.wv, -1, hkv * dh, dl, ln * dl});
-      break;
-    case ST_O:
-      for (int ln = 0; ln < nl; ++ln)
-        out.push_back({lane(ln) + Ly.wo, -1, dl, hq * dh, ln * hq * dh});
-      break;
-    case ST_GU:
-      for (int ln = 0; ln < nl; ++ln)
-        out.push_back({lane(ln) + Ly.wg, lane(ln) + Ly.wu, fl, dl, ln * dl});
-      break;
-    case ST_D:
-      for (int ln = 0; ln < nl; ++ln) out.push_back({lane(ln) + Ly.wd, -1, dl, fl, ln * fl});
-      break;
-    case ST_MIX:
-      out.push_back({Ly.layer0 + Ly.mix, -1, d, d, 0});
-      break;
-    case ST_LM:
-      out.push_back({Ly.lm_head, -1, m.vocab, d, 0});
-      break;
+// Tile shape of a column stage whose rows (canonical columns) have n_out
+// elements: the output vector length.
+const char *make_cshape(int n_out, int in_len, StageShape &s) {
+  s = StageShape{};
+  s.cols = 1;
+  s.K = n_out;
+  s.in_len = in_len;
+  s.out_len = n_out;
+  const int nthreads = kConsumerWarps * 32;
+  const int ngrp = n_out / 4;
+  if (n_out % 4 || 2 * n_out > kSlotBytes) return "output slice of a split projection must fit one slot";
+  if (ngrp >= nthreads) {
+    if (ngrp % nthreads) return "split projection output must be a multiple of 2048 or divide it";
+    s.cps = ngrp / nthreads;
+    s.nseg = 1;
+  } else {
+    if (nthreads % ngrp) return "split projection output must be a multiple of 2048 or divide it";
+    s.cps = 1;
+    s.nseg = nthreads / ngrp;
   }
+  if (s.cps > 4) return "split projection output too long";
+  int R = 1;
+  while (R * 2 * 2 * n_out <= kSlotBytes && R < 64) R *= 2;
+  s.R = R;
+  s.rpw = 1;
+  return nullptr;
 }
 
 // Blocks of one CTA's row range [r0, r1) of a stage; `up` selects the second
-// source of gate/up pieces.  Returns (src offsets of layer 0) per block.
+// source of gate/up pieces.  Returns the layer-0 source of each block.
 void cut_blocks(const std::vector<Piece> &pieces, int r0, int r1, bool up, int lrow_base,
                 const StageShape &sh, int &tile, std::vector<Block> &blk,
-                std::vector<int64_t> &src) {
+                std::vector<Piece> &src) {
   int base = 0;
   for (const Piece &pc : pieces) {
     const int a = std::max(r0, base), b = std::min(r1, base + pc.rows);
@@ -175,9 +172,14 @@ void cut_blocks(const std::vector<Piece> &pieces, int r0, int r1, bool up, int l
       B.nrows = b - a;
       B.in_off = pc.in_off;
       B.tile0 = tile;
+      B.out_off = pc.trans ? pc.out_off : pc.out_off + (a - base);
       tile += (B.nrows + sh.R - 1) / sh.R;
       blk.push_back(B);
-      src.push_back((up ? pc.src2 : pc.src) + int64_t(a - base) * pc.K);
+      Piece one = pc;
+      one.rows = b - a;
+      const int64_t s0 = up ? pc.src2 : pc.src;
+      one.src = pc.trans ? s0 + (a - base) : s0 + int64_t(a - base) * pc.K;
+      src.push_back(one);
     }
     base += pc.rows;
   }
@@ -186,39 +188,86 @@ void cut_blocks(const std::vector<Piece> &pieces, int r0, int r1, bool up, int l
 const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Plan &P) {
   const Layout Ly = make_layout(m);
   const int nl = m.n_lanes, d = m.d_model, dh = m.head_dim;
+  const int dl = d / nl, hq = m.n_heads / nl, hkv = m.n_kv_heads / nl, fl = m.ffn_dim / nl;
+  const int Hkv = m.n_kv_heads, G = m.n_heads / m.n_kv_heads;
   const bool lanes = nl > 1;
   P.n_ctas = n_ctas;
   const char *err = nullptr;
-  if ((err = make_shape(d / nl, d, (m.n_heads + 2 * m.n_kv_heads) * dh, P.shape[ST_QKV])) ||
-      (err = make_shape(m.n_heads / nl * dh, m.n_heads * dh, d, P.shape[ST_O])) ||
-      (err = make_shape(d / nl, d, m.ffn_dim, P.shape[ST_GU])) ||
-      (err = make_shape(m.ffn_dim / nl, m.ffn_dim, d, P.shape[ST_D])) ||
+  if ((err = make_shape(dl, d, (m.n_heads + 2 * Hkv) * dh, P.shape[ST_QKV])) ||
+      (err = make_cshape(dl, m.n_heads * dh, P.shape[ST_O])) ||
+      (err = make_shape(dl, d, m.ffn_dim, P.shape[ST_GU])) ||
+      (err = make_cshape(dl, m.ffn_dim, P.shape[ST_D])) ||
       (err = make_shape(d, d, d, P.shape[ST_MIX])) ||
       (err = make_shape(d, d, m.vocab, P.shape[ST_LM])))
     return err;
+  auto lane0 = [&](int ln) { return Ly.layer0 + int64_t(ln) * Ly.lane_stride; };
 
-  // per-CTA blocks of every stage kind (same for every layer)
   P.stage_cta.assign(size_t(ST_COUNT) * n_ctas, StageCta{});
-  std::vector<std::vector<int64_t>> src_of_cta(n_ctas);   // per CTA, per block: layer-0 source
+  std::vector<std::vector<Piece>> src_of_cta(n_ctas);
   P.cta_blk_begin.assign(n_ctas + 1, 0);
-  std::vector<Piece> pieces;
   int part_max = 4;
   for (int c = 0; c < n_ctas; ++c) {
     P.cta_blk_begin[c] = int(P.blocks.size());
     int local_blk = 0;
+    const int g = c % Hkv, sidx = c / Hkv, ng = (n_ctas - 1 - g) / Hkv + 1;
+    const int ln_g = g / hkv;   // lane of KV head g (0 for dense models)
     for (int k = 0; k < ST_COUNT; ++k) {
       StageCta &sc = P.stage_cta[size_t(k) * n_ctas + c];
       if (k == ST_MIX && !lanes) continue;
-      stage_pieces(m, Ly, k, pieces);
       const StageShape &sh = P.shape[k];
-      const int N = sh.out_len;
-      const int r0 = int(int64_t(N) * c / n_ctas), r1 = int(int64_t(N) * (c + 1) / n_ctas);
+      std::vector<Piece> pieces;
+      int r0 = 0, r1 = 0;
+      switch (k) {
+        case ST_QKV: {   // q rows of the group's query heads, then its k and v rows
+          for (int h = G * g; h < G * (g + 1); ++h)
+            pieces.push_back({lane0(ln_g) + Ly.wq + int64_t(h - ln_g * hq) * dh * dl, -1, dh, dl,
+                              ln_g * dl, h * dh, 0, 0});
+          pieces.push_back({lane0(ln_g) + Ly.wk + int64_t(g - ln_g * hkv) * dh * dl, -1, dh, dl,
+                            ln_g * dl, m.n_heads * dh + g * dh, 0, 0});
+          pieces.push_back({lane0(ln_g) + Ly.wv + int64_t(g - ln_g * hkv) * dh * dl, -1, dh, dl,
+                            ln_g * dl, (m.n_heads + Hkv) * dh + g * dh, 0, 0});
+          const int N = (G + 2) * dh;
+          r0 = int(int64_t(N) * sidx / ng);
+          r1 = int(int64_t(N) * (sidx + 1) / ng);
+          break;
+        }
+        case ST_O: {     // columns of Wo for the group's attention outputs
+          pieces.push_back({lane0(ln_g) + Ly.wo + int64_t(G * g * dh - ln_g * hq * dh), -1, G * dh,
+                            dl, 0, ln_g * dl, 1, hq * dh});
+          const int N = G * dh;
+          r0 = int(int64_t(N) * sidx / ng);
+          r1 = int(int64_t(N) * (sidx + 1) / ng);
+          break;
+        }
+        case ST_GU:
+        case ST_D: {     // this CTA's slice of the hidden units, per lane
+          for (int ln = 0; ln < nl; ++ln) {
+            if (k == ST_GU)
+              pieces.push_back({lane0(ln) + Ly.wg, lane0(ln) + Ly.wu, fl, dl, ln * dl, ln * fl, 0, 0});
+            else
+              pieces.push_back({lane0(ln) + Ly.wd, -1, fl, dl, 0, ln * dl, 1, fl});
+          }
+          r0 = int(int64_t(m.ffn_dim) * c / n_ctas);
+          r1 = int(int64_t(m.ffn_dim) * (c + 1) / n_ctas);
+          break;
+        }
+        case ST_MIX:
+          pieces.push_back({Ly.layer0 + Ly.mix, -1, d, d, 0, 0, 0, 0});
+          r0 = int(int64_t(d) * c / n_ctas);
+          r1 = int(int64_t(d) * (c + 1) / n_ctas);
+          break;
+        case ST_LM:
+          pieces.push_back({Ly.lm_head, -1, m.vocab, d, 0, 0, 0, 0});
+          r0 = int(int64_t(m.vocab) * c / n_ctas);
+          r1 = int(int64_t(m.vocab) * (c + 1) / n_ctas);
+          break;
+      }
       sc.row0 = r0;
       sc.nout = r1 - r0;
       sc.blk_begin = local_blk;
       int tile = 0;
       std::vector<Block> blk;
-      std::vector<int64_t> src;
+      std::vector<Piece> src;
       cut_blocks(pieces, r0, r1, false, 0, sh, tile, blk, src);
       if (k == ST_GU) cut_blocks(pieces, r0, r1, true, sc.nout, sh, tile, blk, src);
       sc.nlocal = (k == ST_GU) ? 2 * sc.nout : sc.nout;
@@ -227,7 +276,9 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
       int64_t bytes = 0;
       for (const Block &B : blk) bytes += int64_t(B.nrows) * sh.K * 2;
       sc.bytes = bytes;
-      part_max = std::max(part_max, sc.nlocal * sh.nseg);
+      if (!sh.cols) part_max = std::max(part_max, sc.nlocal * sh.nseg);
+      if (sh.cols && sc.nlocal > kMaxLocal) return "too many split-projection rows per CTA";
+      if (k == ST_GU && sc.nout > kMaxLocal) return "hidden slice per CTA too large";
       for (size_t i = 0; i < blk.size(); ++i) {
         P.blocks.push_back(blk[i]);
         src_of_cta[c].push_back(src[i]);
@@ -247,13 +298,14 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
       const StageShape &sh = P.shape[k];
       for (int b = 0; b < sc.nblk; ++b) {
         const Block &B = P.blocks[P.cta_blk_begin[c] + sc.blk_begin + b];
+        const Piece &pc = src_of_cta[c][sc.blk_begin + b];
         RepackJob j{};
-        j.src_elem = src_of_cta[c][sc.blk_begin + b] + layer_off;
+        j.src_elem = pc.src + layer_off;
         j.dst_byte = off;
         j.nrows = B.nrows;
         j.K = sh.K;
-        j.KT = sh.K;   // tiles are whole rows: the block is copied as is
-        j.R = sh.R;
+        j.trans = pc.trans;
+        j.src_ld = pc.ld;
         P.jobs.push_back(j);
         off += int64_t(B.nrows) * sh.K * 2;
       }
@@ -272,10 +324,12 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
   }
   P.stream_bytes = off;
 
-  // shared memory: input vector / attention scratch, partial sums, ring
-  const int G = m.n_heads / m.n_kv_heads;
-  int vb = 2 * d;   // normalised inputs (and their gains) are staged in shared memory
-  vb = std::max(vb, (G + 2) * dh + kConsumerWarps * G * (dh + 2));
+  // shared memory: staging / attention scratch, partial sums, ring
+  int vb = 2 * d;   // normalised input and its gains
+  vb = std::max(vb, (G + 2) * dh + kConsumerWarps * G * (dh + 2));   // attention scratch
+  vb = std::max(vb, G * std::min((n_ctas + Hkv - 1) / Hkv, kMaxSplit) * (dh + 2));  // group partials
+  for (int k : {int(ST_O), int(ST_D)})                               // column-stage phases
+    vb = std::max(vb, P.shape[k].nseg * P.shape[k].K);
   P.vbuf_floats = (vb + 3) / 4 * 4;
   P.part_floats = (part_max + 3) / 4 * 4;
   const size_t fixed = monokernel_smem_bytes(0, P.vbuf_floats, P.part_floats);
@@ -284,11 +338,10 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
   slots = std::min(slots, 16);
   P.ring_slots = slots;
   P.smem = monokernel_smem_bytes(slots, P.vbuf_floats, P.part_floats);
-  P.max_split = (n_ctas + m.n_kv_heads - 1) / m.n_kv_heads;
+  P.max_split = std::min((n_ctas + Hkv - 1) / Hkv, kMaxSplit);
 
   // weights streamed by one decode step: all matrices, norms, one embedding row
-  const int64_t esz = 2;
-  P.weight_bytes_per_step = (Ly.total - int64_t(m.vocab) * d + d) * esz;
+  P.weight_bytes_per_step = (Ly.total - int64_t(m.vocab) * d + d) * 2;
   return nullptr;
 }
 
@@ -304,8 +357,8 @@ struct kie_ctx {
   int pending = -1;
   int poisoned = 0;   // sticky error code
   uint64_t watchdog_ns = 2000000000ull;
-  int l2_prefetch_tiles = 0;
   int skip_signal_cta = -1;
+  int grid_sync = 0;
   float last_ms = 0.f;
   int last_steps = 0;
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
@@ -324,7 +377,10 @@ struct kie_ctx {
   int32_t *d_blk_begin = nullptr;
   int64_t *d_stream_off = nullptr;
   unsigned long long *prof = nullptr;  // [n_ctas][kProfSlots] (profiling build)
-  size_t off_x, off_qkv, off_o, off_h, off_u, off_dsum, off_part, act_floats;
+  // activation buffer layout (floats): residual bases, the two layer
+  // accumulators (both parities, contiguous so one memset clears them), q/k/v,
+  // delayed sums, attention partials
+  size_t off_xres, off_acc, off_qkv, off_dsum, off_part, act_floats;
   size_t kv_elems = 0;
   std::vector<int32_t> host_tokens;
 };
@@ -412,10 +468,6 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
     long v = atol(env);
     if (v > 0) ctx->watchdog_ns = uint64_t(v) * 1000000ull;
   }
-  if (const char *env = getenv("KIE_L2_PREFETCH_TILES")) {
-    long v = atol(env);
-    if (v >= 0 && v <= 64) ctx->l2_prefetch_tiles = int(v);
-  }
   cudaError_t e = cudaGetDevice(&ctx->device);
   if (e != cudaSuccess) return fail(cuda_fail(nullptr, "cudaGetDevice", e));
   cudaPointerAttributes pa{};
@@ -465,16 +517,14 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
   if ((rc = alloc(ctx, (void **)&ctx->vcache, ctx->kv_elems * 2, "V cache"))) return fail(rc);
   size_t o = 0;
   auto take = [&](size_t n) { size_t r = o; o += (n + 63) / 64 * 64; return r; };
-  ctx->off_x = take(d);
+  ctx->off_xres = take(size_t(2) * d);
+  ctx->off_acc = take(size_t(4) * d);   // acc_o[2][d] then acc_d[2][d]
   ctx->off_qkv = take(size_t(m.n_heads + 2 * m.n_kv_heads) * dh);
-  ctx->off_o = take(size_t(m.n_heads) * dh);
-  ctx->off_h = take(m.ffn_dim);
-  ctx->off_u = take(size_t(2) * d);
   ctx->off_dsum = take(size_t(std::max(1, m.lane_delay)) * d);
   ctx->off_part = take(size_t(m.n_heads) * P.max_split * (dh + 2));
   ctx->act_floats = o;
   if ((rc = alloc(ctx, (void **)&ctx->act, o * 4, "activations"))) return fail(rc);
-  const size_t sync_words = size_t(SY_ATTN0 + m.n_kv_heads) * kSyncStride;
+  const size_t sync_words = size_t(SY_QG0 + 2 * m.n_kv_heads) * kSyncStride;
   if ((rc = alloc(ctx, (void **)&ctx->sync, sync_words * 4, "sync"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->keys, size_t(m.max_seq) * 8, "keys"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->tokens_in, size_t(m.max_seq) * 4, "tokens"))) return fail(rc);
@@ -550,6 +600,24 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
 }
 
 // Run the persistent kernel for n steps from position pos0.
+// Turns the kernel's status word into a kie_status and poisons the context:
+// the launch left mid-step, so the KV cache and position are not consistent.
+// Low byte: 1..3 a bounded wait ran out (which counter or barrier in the next
+// byte), 4 a NaN logit or an out-of-range token id (step in bits 8..23).
+static int device_error(kie_ctx *ctx, uint32_t status) {
+  char buf[160];
+  const uint32_t kind = status & 0xffu;
+  const int rc = kind == 4u ? KIE_ERR_NONFINITE : KIE_ERR_DEVICE_TIMEOUT;
+  if (kind == 4u)
+    snprintf(buf, sizeof buf, "non-finite logits or token id out of range at step %u (code 0x%x)",
+             status >> 8, status);
+  else
+    snprintf(buf, sizeof buf, "device watchdog: a bounded wait ran out (code 0x%x)", status);
+  g_last_error = buf;
+  ctx->poisoned = rc;
+  return rc;
+}
+
 static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int first_token,
                bool logits_every_step, float *logits_out, int32_t *out_host) {
   const kie_model_desc &m = ctx->m;
@@ -573,8 +641,9 @@ static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int fi
   a.gain_attn = ctx->gains; a.gain_ffn = ctx->gains + size_t(m.n_layers) * m.d_model;
   a.gain_final = ctx->gains + size_t(2 * m.n_layers) * m.d_model;
   a.rope_cs = ctx->rope; a.kcache = ctx->kcache; a.vcache = ctx->vcache;
-  a.x = ctx->act + ctx->off_x; a.qkv = ctx->act + ctx->off_qkv; a.attn_o = ctx->act + ctx->off_o;
-  a.hbuf = ctx->act + ctx->off_h; a.ubuf = ctx->act + ctx->off_u; a.dsum = ctx->act + ctx->off_dsum;
+  a.xres = ctx->act + ctx->off_xres;
+  a.acc_o = ctx->act + ctx->off_acc; a.acc_d = a.acc_o + 2 * size_t(m.d_model);
+  a.qkv = ctx->act + ctx->off_qkv; a.dsum = ctx->act + ctx->off_dsum;
   a.attn_part = ctx->act + ctx->off_part; a.max_split = P.max_split;
   a.sync = ctx->sync; a.keys = ctx->keys;
   a.pos0 = pos0; a.n_steps = n; a.first_token = first_token;
@@ -584,13 +653,14 @@ static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int fi
   a.watchdog_ns = ctx->watchdog_ns;
   a.skip_signal_cta = ctx->skip_signal_cta;
   ctx->skip_signal_cta = -1;
-  a.l2_prefetch_tiles = ctx->l2_prefetch_tiles;
+  a.grid_sync = ctx->grid_sync;
   a.prof = ctx->prof;
 
-  const size_t sync_words = size_t(SY_ATTN0 + m.n_kv_heads) * kSyncStride;
+  const size_t sync_words = size_t(SY_QG0 + 2 * m.n_kv_heads) * kSyncStride;
   if (forced_host)
     CK(cudaMemcpyAsync(ctx->tokens_in, forced_host, size_t(n) * 4, cudaMemcpyHostToDevice, st));
   CK(cudaMemsetAsync(ctx->sync, 0, sync_words * 4, st));
+  CK(cudaMemsetAsync(a.acc_o, 0, size_t(4) * m.d_model * 4, st));   // both accumulators, both parities
   CK(cudaMemsetAsync(ctx->keys, 0, size_t(n) * 8, st));
   void *args[] = {&a};
   CK(cudaEventRecord(ctx->ev0, st));
@@ -604,13 +674,7 @@ static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int fi
   CK(cudaStreamSynchronize(st));
   CK(cudaEventElapsedTime(&ctx->last_ms, ctx->ev0, ctx->ev1));
   ctx->last_steps = n;
-  if (status != 0) {
-    char buf[160];
-    snprintf(buf, sizeof buf, "device watchdog: a bounded wait ran out (code 0x%x)", status);
-    g_last_error = buf;
-    ctx->poisoned = KIE_ERR_DEVICE_TIMEOUT;
-    return KIE_ERR_DEVICE_TIMEOUT;
-  }
+  if (status != 0) return device_error(ctx, status);
   if (out_host) memcpy(out_host, ctx->host_tokens.data(), size_t(n) * 4);
   return KIE_OK;
 }
@@ -673,6 +737,7 @@ extern "C" const char *kie_strerror(int status) {
     case KIE_ERR_NOT_RESIDENT: base = "persistent grid cannot be co-resident"; break;
     case KIE_ERR_DEVICE_TIMEOUT: base = "device watchdog timeout"; break;
     case KIE_ERR_POISONED: base = "context poisoned by an earlier device error"; break;
+    case KIE_ERR_NONFINITE: base = "non-finite logits on the device"; break;
   }
   msg = base;
   if (!g_last_error.empty() && status != KIE_OK) msg += ": " + g_last_error;
@@ -735,6 +800,12 @@ extern "C" int kie_debug_set(kie_ctx *ctx, int32_t watchdog_ms, int32_t skip_sig
   return KIE_OK;
 }
 
+extern "C" int kie_set_sync_mode(kie_ctx *ctx, int32_t mode) {
+  if (!ctx || (mode != KIE_SYNC_DEPENDENCY && mode != KIE_SYNC_GRID)) return KIE_ERR_INVALID;
+  ctx->grid_sync = mode == KIE_SYNC_GRID ? 1 : 0;
+  return KIE_OK;
+}
+
 // ---------------------------------------------------------------- decode without allocation
 // kie_decode_ex_static: the same decode as kie_decode_ex, but the persistent
 // kernel's per-launch scratch (activation vectors, attention partials, the
@@ -786,7 +857,7 @@ extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t
   const Plan &P = ctx->plan;
   // carve the scratch: counters | keys | forced tokens | out tokens | activations
   auto up = [](size_t b) { return (b + 255) / 256 * 256; };
-  const size_t sync_bytes = size_t(SY_ATTN0 + m.n_kv_heads) * kSyncStride * 4;
+  const size_t sync_bytes = size_t(SY_QG0 + 2 * m.n_kv_heads) * kSyncStride * 4;
   const size_t o_keys = up(sync_bytes);
   const size_t o_tin = o_keys + up(size_t(n_steps) * 8);
   const size_t o_tout = o_tin + up(size_t(n_steps) * 4);
@@ -831,8 +902,9 @@ extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t
   a.gain_attn = ctx->gains; a.gain_ffn = ctx->gains + size_t(m.n_layers) * m.d_model;
   a.gain_final = ctx->gains + size_t(2 * m.n_layers) * m.d_model;
   a.rope_cs = ctx->rope; a.kcache = ctx->kcache; a.vcache = ctx->vcache;
-  a.x = act + ctx->off_x; a.qkv = act + ctx->off_qkv; a.attn_o = act + ctx->off_o;
-  a.hbuf = act + ctx->off_h; a.ubuf = act + ctx->off_u; a.dsum = act + ctx->off_dsum;
+  a.xres = act + ctx->off_xres;
+  a.acc_o = act + ctx->off_acc; a.acc_d = a.acc_o + 2 * size_t(m.d_model);
+  a.qkv = act + ctx->off_qkv; a.dsum = act + ctx->off_dsum;
   a.attn_part = act + ctx->off_part; a.max_split = P.max_split;
   a.sync = reinterpret_cast<uint32_t *>(s);
   a.keys = reinterpret_cast<unsigned long long *>(s + o_keys);
@@ -843,13 +915,14 @@ extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t
   a.logits_out = logits_out;
   a.watchdog_ns = ctx->watchdog_ns;
   a.skip_signal_cta = -1;
-  a.l2_prefetch_tiles = ctx->l2_prefetch_tiles;
+  a.grid_sync = ctx->grid_sync;
 
   cudaStream_t st = ctx->stream;
   // the counters and the argmax keys must start at zero on every call
   if (forced_tokens)
     CK(cudaMemcpyAsync(s + o_tin, forced_tokens, size_t(n_steps) * 4, cudaMemcpyHostToDevice, st));
   CK(cudaMemsetAsync(s, 0, o_tin, st));
+  CK(cudaMemsetAsync(a.acc_o, 0, size_t(4) * m.d_model * 4, st));   // both accumulators
   void *args[] = {&a};
   CK(cudaEventRecord(ctx->ev0, st));
   CK(cudaLaunchCooperativeKernel(monokernel_fn(m.dtype), dim3(P.n_ctas), dim3(monokernel_threads()),
@@ -861,13 +934,7 @@ extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t
   CK(cudaStreamSynchronize(st));
   CK(cudaEventElapsedTime(&ctx->last_ms, ctx->ev0, ctx->ev1));
   ctx->last_steps = n_steps;
-  if (status != 0) {
-    char buf[160];
-    snprintf(buf, sizeof buf, "device watchdog: a bounded wait ran out (code 0x%x)", status);
-    g_last_error = buf;
-    ctx->poisoned = KIE_ERR_DEVICE_TIMEOUT;
-    return KIE_ERR_DEVICE_TIMEOUT;
-  }
+  if (status != 0) return device_error(ctx, status);
   ctx->pos += n_steps;
   ctx->pending = out_tokens[n_steps - 1];
   return KIE_OK;

@@ -6,93 +6,107 @@
 
 namespace kie {
 
-// Stage kinds of one decode step, in the order a layer runs them.
+// Stage kinds of one decode step, in the order a layer streams them.
 enum StageKind : int {
-  ST_QKV = 0,  // RMSNorm(attn) + fused q/k/v GEMV            -> qkv
-  ST_O = 1,    // O GEMV + residual add                        -> x (and u)
-  ST_GU = 2,   // RMSNorm(ffn) + gate/up GEMV + SwiGLU         -> h
-  ST_D = 3,    // down GEMV + residual add                     -> x (and u)
-  ST_MIX = 4,  // lane models: delayed cross-lane sum M_i u_i  -> dsum[i % delta]
-  ST_LM = 5,   // final RMSNorm + LM head GEMV + argmax        -> logits / token
+  ST_QKV = 0,  // RMSNorm(attn) + q/k/v rows of this CTA's KV-head group   -> qkv
+  ST_O = 1,    // O projection split along its input: the Wo columns of the
+               // attention outputs this CTA holds                          -> acc_o (atomics)
+  ST_GU = 2,   // RMSNorm(ffn) + gate/up rows of this CTA's hidden slice + SwiGLU -> h (smem)
+  ST_D = 3,    // down projection split along its input: Wd columns of that slice -> acc_d
+  ST_MIX = 4,  // lane models: delayed cross-lane sum M_i u_i (rows)        -> dsum[i % delta]
+  ST_LM = 5,   // final RMSNorm + LM head rows + argmax                     -> logits / token
   ST_COUNT = 6
 };
 
 // Global counters used as epoch barriers (one 128-byte line each).
 enum SyncSlot : int {
-  SY_QKV = 0,    // CTAs that finished the QKV stage
-  SY_OREADY = 1, // KV-head groups whose attention output is merged
-  SY_X1 = 2,     // CTAs that finished the O stage
-  SY_H = 3,      // CTAs that finished the gate/up stage
-  SY_X2 = 4,     // CTAs that finished the down stage
-  SY_MIXF = 5,   // CTAs that finished the final delayed-sum flush
-  SY_TOK = 6,    // CTAs that folded their LM-head rows into the argmax
-  SY_ABORT = 7,  // nonzero: a CTA gave up; everyone leaves
-  SY_STATUS = 8, // first device error code (0 = none)
-  SY_ATTN0 = 16, // per KV-head attention split counters start here
+  SY_S1 = 0,     // CTAs whose O contribution is in acc_o
+  SY_S2 = 1,     // CTAs whose down contribution is in acc_d
+  SY_MIXF = 2,   // CTAs that finished the final delayed-sum flush
+  SY_TOK = 3,    // CTAs that folded their LM-head rows into the argmax
+  SY_ABORT = 4,  // nonzero: a CTA gave up; everyone leaves
+  SY_STATUS = 5, // first device error code (0 = none)
+  SY_GRID = 6,   // grid-barrier mode: signals made by all CTAs together
+  SY_QG0 = 8,    // SY_QG0 + g: CTAs of KV group g whose q/k/v rows are written;
+                 // SY_QG0 + n_kv_heads + g: ... whose attention partials are written
 };
 constexpr int kSyncStride = 32;  // uint32 words per counter (128 bytes)
 
+// Per-SM activity counters of the profiling build (SM clock cycles).
+enum ProfSlot : int {
+  PF_TOTAL = 0,       // consumer thread 0: whole launch
+  PF_GATE = 1,        // waiting for other SMs (epoch counters)
+  PF_GEMV = 2,        // weight stages except the LM head (incl. ring waits)
+  PF_FULLWAIT = 3,    // warp 0: waiting for weight tiles to land (ring empty)
+  PF_ATTN = 4,        // attention and the merge of the group's partials
+  PF_STAGE = 5,       // input staging and RMSNorm
+  PF_SIGNAL = 6,      // end-of-stage barrier + release
+  PF_LM = 7,          // LM-head GEMV
+  PF_PROD_EMPTY = 8,  // producer: waiting for a free slot (ring full)
+  PF_PROD_TOTAL = 9,  // producer: whole launch
+  PF_TILES = 10,      // weight tiles issued
+  PF_NGATE = 11,      // number of dependency waits
+  PF_GEMV_K = 12,     // 12..17: time per stage kind
+  PF_GATE_K = 18,     // 18..23: waiting time on S1, S2, MIXF, TOK, q/k/v group, attention group
+};
+constexpr int kProfSlots = 32;
+
 // Per-stage constants shared by every CTA.  A tile is R whole rows (at most
-// kSlotBytes).  All consumer warps share every tile: warp w takes row group
-// w / nseg (rpw consecutive rows) and column split w % nseg (cps 8-element
-// chunks of each of those rows), so each lane holds at most 4 chunks.
+// kSlotBytes).
+//  Row stages (QKV, GU, MIX, LM): out[row] = sum_k W[row][k] in[k].  All
+//    consumer warps share every tile: warp w takes row group w / nseg (rpw
+//    rows) and column split w % nseg (cps 8-element chunks of each row).
+//  Column stages (O, D): out[:] += sum_row s[row] W[row][:], where a row is
+//    a column of the canonical matrix.  Thread t takes row phase t / ngrp
+//    and 4-element output groups t % ngrp + ngrp * j (j < cps); nseg phases.
 struct StageShape {
-  int32_t K;       // reduction length of every row
+  int32_t K;       // row length (row stages: reduction length; column stages: output length)
   int32_t R;       // rows per tile (power of two)
-  int32_t nseg;    // column splits per row = partial sums per row
-  int32_t rpw;     // rows per warp (1 unless R > 16)
-  int32_t cps;     // 8-element chunks per (row, split) = K / 8 / nseg
+  int32_t nseg;    // row stages: column splits per row; column stages: row phases
+  int32_t rpw;     // row stages: rows per warp (1 unless R > 16)
+  int32_t cps;     // row stages: 8-element chunks per (row, split);
+                   // column stages: 4-element output groups per thread
   int32_t in_len;  // length of the stage input vector
   int32_t out_len; // length of the stage output vector
+  int32_t cols;    // 1 for column stages
 };
 
-// One CTA's share of a stage: output rows [row0, row0 + nout).
+// One CTA's share of a stage.
 struct StageCta {
-  int32_t row0, nout;
-  int32_t nlocal;     // local rows held in partial sums (2*nout for gate/up)
+  int32_t row0, nout; // GU: hidden slice [row0, row0 + nout); MIX, LM: output rows
+  int32_t nlocal;     // local rows (partial sums of row stages, scalars of column stages)
   int32_t ntiles;
   int32_t blk_begin;  // first block, counted from the CTA's own first block
   int32_t nblk;
   int64_t bytes;      // stream bytes of one instance of this stage
 };
 
-// A run of rows of one CTA's stage that read the same input slice.
+// A run of rows of one CTA's stage with one input slice and one output place.
 struct Block {
   int32_t lrow0;   // first local row
   int32_t nrows;
-  int32_t in_off;  // offset of the rows' input within the stage input vector
+  int32_t in_off;  // row stages: offset of the rows' input in the stage input vector
   int32_t tile0;   // index of the block's first tile within the stage
+  int32_t out_off; // row stages: output index of the first row; column stages:
+                   // offset of the block's output slice in the d-vector
+  int32_t pad;
 };
 
 // Copy job of the weight repack: one block of one stage instance.
+//  trans == 0: nrows canonical rows of K elements, copied as they are;
+//  trans == 1: nrows columns of a row-major matrix with K rows and row stride
+//              src_ld, each written as one row of K elements.
 struct RepackJob {
-  int64_t src_elem;  // canonical element offset of the block's first row
+  int64_t src_elem;  // canonical element offset of the first row (or first column's top)
   int64_t dst_byte;  // byte offset in the streaming buffer
-  int32_t nrows, K, KT, R;
+  int32_t nrows, K, trans, src_ld;
 };
-
-// Per-SM activity counters of the profiling build (SM clock cycles).
-enum ProfSlot : int {
-  PF_TOTAL = 0,       // consumer thread 0: whole launch
-  PF_GATE = 1,        // waiting for other SMs (epoch counters)
-  PF_GEMV = 2,        // GEMV stages except the LM head (incl. ring waits)
-  PF_FULLWAIT = 3,    // warp 0: waiting for weight tiles to land (ring empty)
-  PF_ATTN = 4,        // attention (incl. the merge)
-  PF_STAGE = 5,       // input staging and RMSNorm
-  PF_SIGNAL = 6,      // end-of-stage barrier + release
-  PF_LM = 7,          // LM-head GEMV
-  PF_PROD_EMPTY = 8,  // (unused: the copy pump never blocks)
-  PF_PROD_TOTAL = 9,  // (unused)
-  PF_TILES = 10,      // weight tiles issued
-  PF_NGATE = 11,      // number of dependency waits
-  PF_GEMV_K = 12,     // 12..17: GEMV time per stage kind
-  PF_GATE_K = 18,     // 18..24: dependency-wait time per counter (SyncSlot order)
-};
-constexpr int kProfSlots = 32;
 
 constexpr int kMaxBlocksPerCta = 64;
 constexpr int kSlotBytes = 32768;  // one bulk copy per tile: >= 16 KB keeps HBM saturated
 constexpr int kConsumerWarps = 16;
+constexpr int kMaxLocal = 256;     // scalars a column stage holds per CTA
+constexpr int kMaxSplit = 32;      // CTAs that share one KV head's positions (others only merge)
 
 struct KernelArgs {
   // model
@@ -117,11 +131,10 @@ struct KernelArgs {
   const float2 *rope_cs;     // [max_seq, dh/2] (cos, sin)
   // state
   uint16_t *kcache, *vcache; // [L, Hkv, max_seq, dh]
-  float *x;      // [d] residual
+  float *xres;   // [2, d] residual entering global layer G, in xres[G % 2] (row owners write it)
+  float *acc_o;  // [2, d] attention sublayer output of layer G (atomic sums; zero when reused)
+  float *acc_d;  // [2, d] MLP sublayer output of layer G
   float *qkv;    // [(Hq + 2 Hkv) dh]
-  float *attn_o; // [Hq dh]
-  float *hbuf;   // [F]
-  float *ubuf;   // [2, d] lane outputs of the last two layers
   float *dsum;   // [delta, d] delayed cross-lane sums
   float *attn_part;  // [Hq, max_split, dh + 2] per-split attention partials
   int32_t max_split; // most CTAs sharing one KV head
@@ -136,7 +149,7 @@ struct KernelArgs {
   float *logits_out;            // device [n_steps, V] or nullptr
   uint64_t watchdog_ns;
   int32_t skip_signal_cta;      // test hook, -1 = off
-  int32_t l2_prefetch_tiles;    // tiles the producer pulls into L2 beyond the ring
+  int32_t grid_sync;            // 1: every dependency wait is a grid-wide barrier
   unsigned long long *prof;     // [n_ctas][kProfSlots] (profiling build), or nullptr
 };
 

@@ -39,6 +39,7 @@ enum DevErr : uint32_t {
   DE_TIMEOUT_COUNTER = 1,
   DE_TIMEOUT_FULL = 2,
   DE_TIMEOUT_EMPTY = 3,
+  DE_NONFINITE = 4,  // a NaN logit, or a token id outside [0, vocab)
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -69,6 +70,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// try_wait with a suspend-time hint: the thread sleeps in hardware until the
+// phase completes or about hint_ns pass, instead of spinning on issue slots
+// that the consumer warps of its sub-partition need.
+__device__ __forceinline__ bool mbar_wait_hint(uint64_t *b, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -105,6 +120,11 @@ __device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t *p, uint32_t v) {
   uint32_t old;
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
+}
+__device__ __forceinline__ void red_add_v4(float *p, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
+               : "memory");
 }
 // Named barrier over the consumer warps only (the producer never joins).
 __device__ __forceinline__ void cbar() {
@@ -154,15 +174,6 @@ __device__ __forceinline__ float dot8(uint4 w, float4 a, float4 b, float acc) {
 #endif
 
 // ------------------------------------------------------------------ shared state
-// Position of the next weight tile to issue (thread 0's copy pump).
-struct PumpState {
-  const uint8_t *cur;        // next byte of this CTA's weight stream
-  uint32_t T;                // tiles issued
-  int32_t step, l, si, bi, r0, nseq;
-  int32_t seq[6];            // stage kinds of the current layer (or tail)
-  int32_t done;
-};
-
 struct Misc {
   StageCta sc[ST_COUNT];
   Block blk[kMaxBlocksPerCta];
@@ -172,14 +183,18 @@ struct Misc {
   volatile int32_t abort;  // a consumer saw a failed wait
   int32_t flag;            // broadcast slot
   long long prof[kProfSlots];
-  PumpState pump;   // next tile to copy into the ring
-  PumpState pf;     // next tile to prefetch into L2 (runs ahead of `pump`)
 };
+
+// Scalars of the column stages: the merged attention output of the CTA's KV
+// group (at most 4 heads x 128) and the CTA's slice of the SwiGLU hidden units.
+constexpr int kSvecO = 512;
+constexpr int kSvecFloats = kSvecO + kMaxLocal;
 
 struct Smem {
   uint8_t *ring;
   uint64_t *full, *empty;
   float *vbuf, *part;
+  float *svec;   // [0, kSvecO): merged attention output; [kSvecO, ...): hidden slice
   Misc *misc;
 };
 
@@ -222,15 +237,17 @@ __device__ bool wait_counter(const KernelArgs &a, const uint32_t *ctr, uint32_t 
 }
 
 // Bounded wait on an mbarrier phase.
+constexpr uint32_t kSuspendHintNs = 20000;
+
 template <typename PumpT>
 __device__ bool wait_mbar(const KernelArgs &a, uint64_t *bar, uint32_t parity, uint32_t code,
                           PumpT &&pump) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_wait_hint(bar, parity, kSuspendHintNs)) return true;
   const long long t0 = clock64(), limit = (long long)a.watchdog_ns * 2;
   long long next_poll = kAbortPollCycles;
   const uint32_t *abortp = sync_at(a, SY_ABORT);
   for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_wait_hint(bar, parity, kSuspendHintNs)) return true;
     pump();
     const long long el = clock64() - t0;
     if (el > next_poll) {
@@ -244,159 +261,103 @@ __device__ bool wait_mbar(const KernelArgs &a, uint64_t *bar, uint32_t parity, u
   }
 }
 
-// ------------------------------------------------------------------ weight pump
-// Thread 0 of each CTA issues the CTA's weight tiles, in the order they are
-// consumed, into free ring slots: one cp.async.bulk (1-D bulk copy, no tensor
-// map, no multicast, L2 evict-first) per tile, completing on the slot's full
-// mbarrier.  It never blocks: pump() returns when the next slot is still in
-// use, and thread 0 calls it from every wait loop it runs (dependency gates,
-// tile waits) and after every tile, so the weight stream keeps flowing while
-// the CTA waits for other SMs -- weights do not depend on activations.
-struct Pump {
+// ------------------------------------------------------------------ weight producer
+// One lane of the producer warp issues the CTA's weight tiles, in the order
+// the consumers take them, into the ring: one cp.async.bulk (1-D bulk copy, no
+// tensor map, no multicast, L2 evict-first) per tile, completing on the slot's
+// full mbarrier, after the slot's empty mbarrier says all 16 consumer warps
+// released its previous tile.  Weights do not depend on activations, so the
+// stream runs ahead across stage, layer and step boundaries while the
+// consumers wait for other SMs.  Its state lives in registers; its waits
+// sleep in hardware (bounded).
+struct Producer {
   const KernelArgs &a;
   Smem s;
-  __device__ Pump(const KernelArgs &a_, Smem s_) : a(a_), s(s_) {}
+  const int cta;
+  uint32_t T = 0;        // tiles issued
+  __device__ Producer(const KernelArgs &a_, Smem s_, int cta_) : a(a_), s(s_), cta(cta_) {}
 
-  __device__ bool lm_step(int step) const { return a.logits_every_step || step == a.n_steps - 1; }
+  // The cached K/V rows this CTA's attention split reads in layer l of step
+  // `step` (positions before the step's own), pulled into L2 when the layer's
+  // first weight tile is issued, well before the attention needs them.
+  __device__ void prefetch_kv(int step, int l) const {
+    const int Hkv = a.n_kv_heads, g = cta % Hkv, split = cta / Hkv;
+    const int nsplit = min((a.n_ctas - 1 - g) / Hkv + 1, kMaxSplit);
+    if (split >= nsplit) return;
+    const int pos = a.pos0 + step, Lctx = pos + 1;
+    const int j0 = int((int64_t)split * Lctx / nsplit);
+    const int j1 = min(int((int64_t)(split + 1) * Lctx / nsplit), pos);
+    if (j1 <= j0) return;
+    const size_t row = ((size_t(l) * Hkv + g) * a.max_seq + j0) * a.head_dim;
+    const uint32_t bytes = uint32_t(j1 - j0) * uint32_t(a.head_dim) * 2u;
+    prefetch_l2(a.kcache + row, bytes);
+    prefetch_l2(a.vcache + row, bytes);
+  }
 
-  __device__ void load_seq(PumpState &p) const {
-    p.nseq = 0;
+  // Issues every tile of stage k (its blocks in order); false once a wait
+  // for a free slot gave up.
+  __device__ bool stage(int k, const uint8_t *&cur, uint32_t &slot, uint32_t &phase) {
+    const StageCta &c = s.misc->sc[k];
+    const int nblk = c.nblk, b0 = c.blk_begin;
+    const int R = a.shape[k].R;
+    const uint32_t rowb = uint32_t(a.shape[k].K) * 2u;
+    const uint32_t NS = a.ring_slots;
+    for (int bi = 0; bi < nblk; ++bi) {
+      const int nrows = s.misc->blk[b0 + bi].nrows;
+      for (int r0 = 0; r0 < nrows; r0 += R) {
+        if (T >= NS) {
+#ifdef KIE_PROFILE
+          const long long tw = clock64();
+#endif
+          // the slot's previous tile (T - NS) was released by every consumer warp
+          if (!wait_mbar(a, &s.empty[slot], phase ^ 1u, DE_TIMEOUT_EMPTY, [] {})) return false;
+#ifdef KIE_PROFILE
+          s.misc->prof[PF_PROD_EMPTY] += clock64() - tw;
+#endif
+        }
+        const uint32_t bytes = uint32_t(min(R, nrows - r0)) * rowb;
+        mbar_expect_tx(&s.full[slot], bytes);
+        bulk_g2s(s.ring + size_t(slot) * kSlotBytes, cur, bytes, &s.full[slot], policy_evict_first());
+        cur += bytes;
+        ++T;
+        if (++slot == NS) { slot = 0; phase ^= 1u; }
+      }
+    }
+    return true;
+  }
+
+  __device__ void run() {
+    const uint8_t *base = a.wstream + a.cta_stream_off[cta];
     const bool lanes = a.n_lanes > 1;
-    if (p.l < a.n_layers) {
-      p.seq[p.nseq++] = ST_QKV;
-      if (lanes && p.l >= 1) p.seq[p.nseq++] = ST_MIX;
-      p.seq[p.nseq++] = ST_O;
-      p.seq[p.nseq++] = ST_GU;
-      p.seq[p.nseq++] = ST_D;
-    } else if (lm_step(p.step)) {
-      if (lanes) p.seq[p.nseq++] = ST_MIX;
-      p.seq[p.nseq++] = ST_LM;
-    }
-  }
-
-  // move (si, bi, r0) forward to the next tile that exists
-  __device__ void normalize(PumpState &p, const uint8_t *base) const {
-    while (!p.done) {
-      if (p.si < p.nseq) {
-        const StageCta &c = s.misc->sc[p.seq[p.si]];
-        if (p.bi < c.nblk) {
-          if (p.r0 < s.misc->blk[c.blk_begin + p.bi].nrows) return;
-          ++p.bi;
-          p.r0 = 0;
-          continue;
-        }
-        ++p.si;
-        p.bi = 0;
-        p.r0 = 0;
-        continue;
+    uint32_t slot = 0, phase = 0;   // phase: parity of the slot's current use
+    bool ok = true;
+    for (int step = 0; step < a.n_steps && ok; ++step) {
+      const uint8_t *cur = base;
+      for (int l = 0; l < a.n_layers && ok; ++l) {
+        prefetch_kv(step, l);
+        ok = stage(ST_QKV, cur, slot, phase);
+        if (ok && lanes && l >= 1) ok = stage(ST_MIX, cur, slot, phase);
+        ok = ok && stage(ST_O, cur, slot, phase);
+        ok = ok && stage(ST_GU, cur, slot, phase);
+        ok = ok && stage(ST_D, cur, slot, phase);
       }
-      p.si = p.bi = p.r0 = 0;
-      if (p.l < a.n_layers) {
-        ++p.l;
-      } else {
-        ++p.step;
-        p.l = 0;
-        p.cur = base;
-        if (p.step >= a.n_steps) {
-          p.done = 1;
-          return;
-        }
+      if (ok && (a.logits_every_step || step == a.n_steps - 1)) {
+        if (lanes) ok = stage(ST_MIX, cur, slot, phase);
+        ok = ok && stage(ST_LM, cur, slot, phase);
       }
-      load_seq(p);
-    }
-  }
-
-  __device__ void init_state(PumpState &p, int cta) const {
-    p.cur = a.wstream + a.cta_stream_off[cta];
-    p.T = 0;
-    p.step = p.l = p.si = p.bi = p.r0 = 0;
-    p.done = a.n_steps > 0 ? 0 : 1;
-    load_seq(p);
-    normalize(p, p.cur);
-  }
-
-  __device__ uint32_t tile_bytes(const PumpState &p) const {
-    const int k = p.seq[p.si];
-    const StageShape &sh = a.shape[k];
-    const Block &b = s.misc->blk[s.misc->sc[k].blk_begin + p.bi];
-    return uint32_t(min(sh.R, b.nrows - p.r0)) * uint32_t(sh.K) * 2u;
-  }
-
-  __device__ void advance(PumpState &p, uint32_t bytes, const uint8_t *base) const {
-    p.cur += bytes;
-    ++p.T;
-    p.r0 += a.shape[p.seq[p.si]].R;
-    normalize(p, base);
-  }
-
-  __device__ void init(int cta) {
-    init_state(s.misc->pump, cta);
-    init_state(s.misc->pf, cta);
-  }
-
-  // Copy tiles into every free ring slot; returns when the next slot is busy.
-  __device__ void pump(int cta) {
-    PumpState &p = s.misc->pump;
-    const uint32_t NS = a.ring_slots;
-    const uint8_t *base = a.wstream + a.cta_stream_off[cta];
-    while (!p.done) {
-      const uint32_t slot = p.T % NS;
-      if (p.T >= NS && !mbar_try_wait(&s.empty[slot], ((p.T / NS) - 1) & 1)) return;
-      const uint32_t bytes = tile_bytes(p);
-      mbar_expect_tx(&s.full[slot], bytes);
-      bulk_g2s(s.ring + size_t(slot) * kSlotBytes, p.cur, bytes, &s.full[slot], policy_evict_first());
-      advance(p, bytes, base);
-    }
-  }
-
-  // While the ring is full, pull the next l2_prefetch_tiles tiles into L2 so
-  // that HBM keeps streaming and the ring refills from L2 once slots free up.
-  __device__ void prefetch(int cta) {
-    PumpState &q = s.misc->pf;
-    const uint32_t T = s.misc->pump.T;
-    const uint8_t *base = a.wstream + a.cta_stream_off[cta];
-    while (!q.done && q.T < T + uint32_t(a.l2_prefetch_tiles)) {
-      const uint32_t bytes = tile_bytes(q);
-      if (q.T >= T) prefetch_l2(q.cur, bytes);
-      advance(q, bytes, base);
-    }
-  }
-
-  // The producer warp's loop: fill free slots, prefetch ahead into L2, then
-  // sleep on the next slot's empty barrier until every consumer warp released
-  // it (bounded by the watchdog).
-  __device__ void run(int cta) {
-    init(cta);
-    PumpState &p = s.misc->pump;
-    const uint32_t NS = a.ring_slots;
-    while (!p.done) {
-      pump(cta);
-      if (p.done) break;
-      prefetch(cta);
-      const uint32_t slot = p.T % NS;
-#ifdef KIE_PROFILE
-      const long long tw = clock64();
-#endif
-      if (!wait_mbar(a, &s.empty[slot], ((p.T / NS) - 1) & 1, DE_TIMEOUT_EMPTY, [] {})) break;
-#ifdef KIE_PROFILE
-      s.misc->prof[PF_PROD_EMPTY] += clock64() - tw;
-#endif
     }
     drain();
   }
 
   // Before the CTA exits: each slot holds at most one outstanding copy, the
   // last one issued into it; wait (bounded) until those have landed.
-  __device__ void drain() {
-    const uint32_t NS = a.ring_slots, T = s.misc->pump.T;
+  __device__ void drain() const {
+    const uint32_t NS = a.ring_slots;
     const uint32_t first = T > NS ? T - NS : 0;
     for (uint32_t t = first; t < T; ++t) {
-      if (!mbar_try_wait(&s.full[t % NS], (t / NS) & 1)) {
-        const long long t0 = clock64();
-        while (!mbar_try_wait(&s.full[t % NS], (t / NS) & 1)) {
-          if (clock64() - t0 > (long long)a.watchdog_ns * 2) break;
-        }
-      }
+      const long long t0 = clock64();
+      while (!mbar_wait_hint(&s.full[t % NS], (t / NS) & 1, kSuspendHintNs))
+        if (clock64() - t0 > (long long)a.watchdog_ns * 2) break;
     }
   }
 };
@@ -410,23 +371,32 @@ struct Consumer {
   uint32_t Tbase = 0;   // tiles consumed before the current stage
   uint32_t slot = 0, phase = 0;   // ring position of the next tile (every warp sees every tile)
   int step = 0, l = 0, tok = 0, p = 0;
+  uint32_t gl = 0;        // global layer index step * n_layers + l (parity of the buffers)
   uint32_t lm_count = 0;
+  uint32_t nsig = 0;      // signals this CTA has made (grid-barrier mode)
 
   __device__ Consumer(const KernelArgs &a_, Smem s_, int tid_, int cta_)
       : a(a_), s(s_), tid(tid_), warp(tid_ >> 5), lane(tid_ & 31), cta(cta_) {}
 
   __device__ bool aborted() const { return s.misc->abort != 0; }
 
-  // thread 0 waits for a counter, everyone learns the outcome
-  __device__ bool gate(int slot, uint32_t target, uint32_t where) {
+  // thread 0 waits for a counter, everyone learns the outcome.  In grid-barrier
+  // mode (an ablation of the per-dependency counters) every wait is instead
+  // for all CTAs to have made as many signals as this one: every CTA makes the
+  // same sequence of signals, and each gate follows the signal it waits for.
+  __device__ bool gate(int slot, uint32_t target, uint32_t where, int pkind) {
     if (tid == 0) {
 #ifdef KIE_PROFILE
       const long long t0 = clock64();
 #endif
+      if (a.grid_sync) {
+        slot = SY_GRID;
+        target = nsig * a.n_ctas;
+      }
       if (!wait_counter(a, sync_at(a, slot), target, where, [] {})) s.misc->abort = 1;
 #ifdef KIE_PROFILE
       s.misc->prof[PF_GATE] += clock64() - t0;
-      s.misc->prof[PF_GATE_K + slot] += clock64() - t0;
+      s.misc->prof[PF_GATE_K + pkind] += clock64() - t0;
       s.misc->prof[PF_NGATE] += 1;
 #endif
     }
@@ -437,20 +407,21 @@ struct Consumer {
   __device__ void signal(int slot) {
     KP_BEGIN(t_sig);
     cbar();
-    if (tid == 0) red_release_add(sync_at(a, slot), 1u);
+    ++nsig;
+    if (tid == 0) red_release_add(sync_at(a, a.grid_sync ? int(SY_GRID) : slot), 1u);
     KP_END(t_sig, PF_SIGNAL);
   }
 
   // ---- stage inputs
-  __device__ float xin(int i) const {
-    // residual entering the current layer, plus the delayed sum landing here
-    float v = (l == 0) ? Store<T>::to_f(a.embed[size_t(tok) * a.d_model + i]) : __ldcg(a.x + i);
-    if (a.n_lanes > 1 && l >= a.lane_delay)
-      v += __ldcg(a.dsum + size_t((l - a.lane_delay) % a.lane_delay) * a.d_model + i);
-    return v;
+  __device__ static float4 add4(float4 u, float4 v) {
+    return make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
+  }
+  __device__ const float4 *vec4(const float *base, uint32_t parity) const {
+    return reinterpret_cast<const float4 *>(base + size_t(parity & 1u) * a.d_model);
   }
 
-  // elements 4j..4j+3 of the residual entering the current layer
+  // elements 4j..4j+3 of the residual entering the current layer (the
+  // embedding row at layer 0), plus the delayed cross-lane sum landing here
   __device__ float4 xin4(int j) const {
     float4 v;
     if (l == 0) {
@@ -458,13 +429,13 @@ struct Consumer {
       const float2 lo = Store<T>::pair(w.x), hi = Store<T>::pair(w.y);
       v = make_float4(lo.x, lo.y, hi.x, hi.y);
     } else {
-      v = __ldcg(reinterpret_cast<const float4 *>(a.x) + j);
+      const uint32_t q = gl - 1;
+      v = add4(add4(__ldcg(vec4(a.xres, q) + j), __ldcg(vec4(a.acc_o, q) + j)),
+               __ldcg(vec4(a.acc_d, q) + j));
     }
-    if (a.n_lanes > 1 && l >= a.lane_delay) {
-      const float4 q = __ldcg(reinterpret_cast<const float4 *>(
-                                  a.dsum + size_t((l - a.lane_delay) % a.lane_delay) * a.d_model) + j);
-      v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
-    }
+    if (a.n_lanes > 1 && l >= a.lane_delay)
+      v = add4(v, __ldcg(reinterpret_cast<const float4 *>(
+                             a.dsum + size_t((l - a.lane_delay) % a.lane_delay) * a.d_model) + j));
     return v;
   }
 
@@ -472,8 +443,11 @@ struct Consumer {
   // multiple of 128).  src(i4) returns elements 4*i4 .. 4*i4+3.  Each thread
   // holds up to 4 float4 groups; warp partial sums of squares go through
   // shared memory and every thread adds up the ones of its own slice.
+  // If own is not null, this CTA's rows [own_lo, own_hi) of the raw input are
+  // also written to own (the residual of the layer, kept by its row owners).
   template <typename Src>
-  __device__ void stage_norm(Src src, const float *gain, int n, int seg) {
+  __device__ void stage_norm(Src src, const float *gain, int n, int seg, float *own = nullptr,
+                             int own_lo = 0, int own_hi = 0) {
     KP_BEGIN(t_norm);
     const int ng = n >> 2;
     float4 *vb = reinterpret_cast<float4 *>(s.vbuf);
@@ -483,6 +457,12 @@ struct Consumer {
       float ss = 0.f;
       if (j < ng) {
         const float4 v = src(j);
+        if (own && 4 * j + 3 >= own_lo && 4 * j < own_hi) {
+          const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (4 * j + u >= own_lo && 4 * j + u < own_hi) own[4 * j + u] = e[u];
+        }
         gb[j] = *reinterpret_cast<const float4 *>(gain + 4 * j);
         vb[j] = v;
         ss = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
@@ -646,21 +626,64 @@ struct Consumer {
   }
 
   // ---- attention over the cache for one KV head group (split-KV)
-  __device__ void attention() {
+  // Positions of this CTA's split: [j0, j1) of 0..p.  Each warp folds
+  // positions j0 + warp + W*i, two per iteration.
+  static constexpr int kU = 2;
+  struct KvWords {
+    uint2 k[kU], v[kU];   // raw storage words of this lane (dh 64 uses .x only)
+  };
+  __device__ void kv_range(int &j0, int &j1, int &split, int &nsplit) const {
+    const int Hkv = a.n_kv_heads, g = cta % Hkv;
+    split = cta / Hkv;
+    const int ngroup = (a.n_ctas - 1 - g) / Hkv + 1;      // CTAs of this KV group
+    nsplit = min(ngroup, kMaxSplit);                      // those that take positions
+    const int Lctx = p + 1;
+    j0 = split < nsplit ? int((int64_t)split * Lctx / nsplit) : 0;
+    j1 = split < nsplit ? int((int64_t)(split + 1) * Lctx / nsplit) : 0;
+  }
+  // Loads the cached K/V rows of positions jb + u*W (u < kU) that lie in
+  // [jb, j1) and before p (row p is written in this step and comes from
+  // shared memory instead).
+  __device__ void kv_load(KvWords &w, int jb, int j1) const {
+    const int dh = a.head_dim, Hkv = a.n_kv_heads, g = cta % Hkv;
+    const size_t base = ((size_t(l) * Hkv + g) * a.max_seq) * dh;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int j = jb + u * kConsumerWarps;
+      w.k[u] = make_uint2(0u, 0u);
+      w.v[u] = make_uint2(0u, 0u);
+      if (j < j1 && j != p) {
+        if (dh == 128) {
+          w.k[u] = __ldcg(reinterpret_cast<const uint2 *>(a.kcache + base + size_t(j) * dh) + lane);
+          w.v[u] = __ldcg(reinterpret_cast<const uint2 *>(a.vcache + base + size_t(j) * dh) + lane);
+        } else {
+          w.k[u].x = __ldcg(reinterpret_cast<const unsigned int *>(a.kcache + base + size_t(j) * dh) + lane);
+          w.v[u].x = __ldcg(reinterpret_cast<const unsigned int *>(a.vcache + base + size_t(j) * dh) + lane);
+        }
+      }
+    }
+  }
+  // Issued before the q/k/v gate: the cache rows do not depend on this step.
+  __device__ void attention_prefetch(KvWords &w) const {
+    int j0, j1, split, nsplit;
+    kv_range(j0, j1, split, nsplit);
+    kv_load(w, j0 + warp, j1);
+  }
+
+  __device__ void attention(KvWords &pre) {
     KP_BEGIN(t_attn);
-    attention_body();
+    attention_body(pre);
     KP_END(t_attn, PF_ATTN);
   }
 
-  __device__ void attention_body() {
+  __device__ void attention_body(KvWords &kw) {
     const int dh = a.head_dim, half = dh >> 1;
     const int Hkv = a.n_kv_heads, G = a.n_heads / a.n_kv_heads;
     const int g = cta % Hkv;
-    const int split = cta / Hkv;
-    const int nsplit = (a.n_ctas - 1 - g) / Hkv + 1;
-    const int Lctx = p + 1;
-    const int j0 = int((int64_t)split * Lctx / nsplit);
-    const int j1 = int((int64_t)(split + 1) * Lctx / nsplit);
+    const int ngroup = (a.n_ctas - 1 - g) / Hkv + 1;      // CTAs of this KV group
+    int j0, j1, split, nsplit;
+    kv_range(j0, j1, split, nsplit);
+    const bool active = split < nsplit;
     const bool writer = (split == nsplit - 1);  // its range holds position p
     float *qs = s.vbuf;              // [G][dh] roped, scaled queries
     float *kcur = qs + G * dh;       // [dh] roped, rounded key of position p
@@ -693,7 +716,10 @@ struct Consumer {
       }
     }
     cbar();
-    // each warp folds positions j0 + warp, j0 + warp + W, ... with an online softmax
+    // Online softmax, kU positions per iteration: their score reductions are
+    // independent and one rescale covers them.  The next iteration's rows are
+    // requested before this one's arithmetic (the first ones were requested
+    // before the q/k/v gate).
     const int dpl = dh >> 5;  // dims per lane: 4 (dh 128) or 2 (dh 64)
     float m[4], lsum[4], o[4][4];
 #pragma unroll
@@ -703,45 +729,63 @@ struct Consumer {
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
     }
-    const uint16_t *kbase = a.kcache + ((size_t(l) * Hkv + g) * a.max_seq) * dh;
-    const uint16_t *vbase = a.vcache + ((size_t(l) * Hkv + g) * a.max_seq) * dh;
-    for (int j = j0 + warp; j < j1; j += kConsumerWarps) {
-      float kv[4], vv[4];
-      if (j == p) {
+    constexpr int U = kU;
+    for (int jb = j0 + warp; jb < j1; jb += U * kConsumerWarps) {
+      float kv[U][4], vv[U][4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (e < dpl) { kv[e] = kcur[lane * dpl + e]; vv[e] = vcur[lane * dpl + e]; }
-      } else if (dpl == 4) {
-        const uint2 kw = __ldcg(reinterpret_cast<const uint2 *>(kbase + size_t(j) * dh) + lane);
-        const uint2 vw = __ldcg(reinterpret_cast<const uint2 *>(vbase + size_t(j) * dh) + lane);
-        float2 f;
-        f = Store<T>::pair(kw.x); kv[0] = f.x; kv[1] = f.y;
-        f = Store<T>::pair(kw.y); kv[2] = f.x; kv[3] = f.y;
-        f = Store<T>::pair(vw.x); vv[0] = f.x; vv[1] = f.y;
-        f = Store<T>::pair(vw.y); vv[2] = f.x; vv[3] = f.y;
-      } else {
-        const uint32_t kw = __ldcg(reinterpret_cast<const unsigned int *>(kbase + size_t(j) * dh) + lane);
-        const uint32_t vw = __ldcg(reinterpret_cast<const unsigned int *>(vbase + size_t(j) * dh) + lane);
-        float2 f;
-        f = Store<T>::pair(kw); kv[0] = f.x; kv[1] = f.y;
-        f = Store<T>::pair(vw); vv[0] = f.x; vv[1] = f.y;
-        kv[2] = kv[3] = vv[2] = vv[3] = 0.f;
+      for (int u = 0; u < U; ++u) {
+        const int j = jb + u * kConsumerWarps;
+        if (j == p) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            kv[u][e] = e < dpl ? kcur[lane * dpl + e] : 0.f;
+            vv[u][e] = e < dpl ? vcur[lane * dpl + e] : 0.f;
+          }
+        } else {
+          float2 f;
+          f = Store<T>::pair(kw.k[u].x); kv[u][0] = f.x; kv[u][1] = f.y;
+          f = Store<T>::pair(kw.k[u].y); kv[u][2] = f.x; kv[u][3] = f.y;
+          f = Store<T>::pair(kw.v[u].x); vv[u][0] = f.x; vv[u][1] = f.y;
+          f = Store<T>::pair(kw.v[u].y); vv[u][2] = f.x; vv[u][3] = f.y;
+        }
       }
+      kv_load(kw, jb + U * kConsumerWarps, j1);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         if (i < G) {
-          float sc = 0.f;
+          float sc[U];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (e < dpl) sc = fmaf(qs[i * dh + lane * dpl + e], kv[e], sc);
-          for (int of = 16; of; of >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, of);
-          const float mn = fmaxf(m[i], sc);
-          const float corr = expf(m[i] - mn);
-          const float pj = expf(sc - mn);
-          lsum[i] = lsum[i] * corr + pj;
+          for (int u = 0; u < U; ++u) {
+            float t = 0.f;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) o[i][e] = o[i][e] * corr + pj * vv[e];
-          m[i] = mn;
+            for (int e = 0; e < 4; ++e)
+              if (e < dpl) t = fmaf(qs[i * dh + lane * dpl + e], kv[u][e], t);
+            sc[u] = t;
+          }
+#pragma unroll
+          for (int of = 16; of; of >>= 1)
+#pragma unroll
+            for (int u = 0; u < U; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], of);
+          float mx = m[i];
+#pragma unroll
+          for (int u = 0; u < U; ++u)
+            if (jb + u * kConsumerWarps < j1) mx = fmaxf(mx, sc[u]);
+          const float corr = expf(m[i] - mx);
+          float pu[U], ps = 0.f;
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            pu[u] = (jb + u * kConsumerWarps < j1) ? expf(sc[u] - mx) : 0.f;
+            ps += pu[u];
+          }
+          lsum[i] = lsum[i] * corr + ps;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float acc = o[i][e] * corr;
+#pragma unroll
+            for (int u = 0; u < U; ++u) acc = fmaf(pu[u], vv[u][e], acc);
+            o[i][e] = acc;
+          }
+          m[i] = mx;
         }
       }
     }
@@ -758,7 +802,7 @@ struct Consumer {
     }
     cbar();
     // combine the warps into this CTA's partial for each query head
-    for (int idx = tid; idx < G * dh; idx += kNC) {
+    for (int idx = tid; idx < (active ? G * dh : 0); idx += kNC) {
       const int i = idx / dh, d = idx - i * dh;
       float M = -INFINITY;
       for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, wst[(size_t(w) * G + i) * st + dh]);
@@ -775,43 +819,136 @@ struct Consumer {
       dst[d] = O;
       if (d == 0) { dst[dh] = M; dst[dh + 1] = Ls; }
     }
-    cbar();
-    const uint32_t epoch = uint32_t(step) * a.n_layers + l + 1;
-    if (tid == 0) {
-      const uint32_t old = atom_acq_rel_add(sync_at(a, SY_ATTN0 + g), 1u);
-      s.misc->flag = (old + 1 == epoch * uint32_t(nsplit)) ? 1 : 0;
+    // every split of the group publishes its partial, then each CTA of the
+    // group loads all of them into shared memory (one coalesced pass) and
+    // merges them (log-sum-exp) into the group's attention output
+    signal(SY_QG0 + Hkv + g);
+    if (!gate(SY_QG0 + Hkv + g, (gl + 1) * uint32_t(ngroup), 0x28, 5)) return;
+    float *pb = s.vbuf;   // [G][nsplit][st]
+    for (int i = 0; i < G; ++i) {
+      const float *src = a.attn_part + size_t(g * G + i) * a.max_split * st;
+      for (int q = tid; q < nsplit * st; q += kNC) pb[(size_t(i) * nsplit) * st + q] = __ldcg(src + q);
     }
     cbar();
-    if (s.misc->flag) {
-      // last split of this group: merge all splits into attn_o
-      for (int idx = tid; idx < G * dh; idx += kNC) {
-        const int i = idx / dh, d = idx - i * dh;
-        const float *src = a.attn_part + size_t(g * G + i) * a.max_split * st;
-        float M = -INFINITY;
-        for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, __ldcg(src + size_t(sp) * st + dh));
-        float Ls = 0.f, O = 0.f;
-        for (int sp = 0; sp < nsplit; ++sp) {
-          const float *ps = src + size_t(sp) * st;
-          const float f = expf(__ldcg(ps + dh) - M);
-          Ls += __ldcg(ps + dh + 1) * f;
-          O += __ldcg(ps + d) * f;
-        }
-        a.attn_o[size_t(g * G + i) * dh + d] = O / Ls;
+    float *og = s.svec;   // [G * dh] merged attention output of the group
+    for (int idx = tid; idx < G * dh; idx += kNC) {
+      const int i = idx / dh, d = idx - i * dh;
+      const float *src = pb + size_t(i) * nsplit * st;
+      float M = -INFINITY;
+      for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, src[size_t(sp) * st + dh]);
+      float Ls = 0.f, O = 0.f;
+      for (int sp = 0; sp < nsplit; ++sp) {
+        const float *ps = src + size_t(sp) * st;
+        const float f = expf(ps[dh] - M);
+        Ls += ps[dh + 1] * f;
+        O += ps[d] * f;
       }
-      signal(SY_OREADY);
+      og[idx] = O / Ls;
     }
+    cbar();
+  }
+
+  // ---- column stages (O, down): out[:] += sum_i svals[i] * W_i[:]
+  // W_i are the stage's streamed rows (columns of the canonical matrix), svals
+  // the matching scalars in shared memory (index = local row).  Each thread
+  // accumulates 4-element output groups over its row phase; phases are summed
+  // in shared memory, then every group is added to acc with one vector atomic.
+  __device__ void gemv_cols(int k, const float *svals, float *acc) {
+    KP_BEGIN(t_gemv);
+    const StageShape sh = a.shape[k];
+    const StageCta &c = s.misc->sc[k];
+    const int ngrp = sh.K >> 2;                  // 4-element groups of the output
+    const int tpr = sh.nseg > 1 ? ngrp : kNC;    // threads per row phase
+    const int ph = tid / tpr, gi = tid - ph * tpr;
+    // A failed wait stops this warp's tile work, but every warp still goes
+    // through the same barriers so that none is left waiting.
+    bool ok = !aborted();
+    for (int bi = 0; bi < c.nblk; ++bi) {
+      const Block b = s.misc->blk[c.blk_begin + bi];
+      float acc4[4][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc4[j][e] = 0.f;
+      const int ntile = (b.nrows + sh.R - 1) / sh.R;
+      for (int t = 0; t < ntile && ok; ++t) {
+        bool got = true;
+#ifdef KIE_PROFILE
+        const long long tw = (tid == 0) ? clock64() : 0ll;
+#endif
+        if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [] {});
+#ifdef KIE_PROFILE
+        if (tid == 0) s.misc->prof[PF_FULLWAIT] += clock64() - tw;
+#endif
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          s.misc->abort = 1;
+          ok = false;
+          break;
+        }
+        const int rows = min(sh.R, b.nrows - t * sh.R);
+        const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes;
+        const float *sv = svals + b.lrow0 + t * sh.R;
+        for (int r = ph; r < rows; r += sh.nseg) {
+          const float x = sv[r];
+          const uint8_t *row = tile + size_t(r) * sh.K * 2;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < sh.cps) {
+              const uint2 w = *reinterpret_cast<const uint2 *>(row + size_t(gi + tpr * j) * 8);
+              const float2 lo = Store<T>::pair(w.x), hi = Store<T>::pair(w.y);
+              acc4[j][0] = fmaf(x, lo.x, acc4[j][0]);
+              acc4[j][1] = fmaf(x, lo.y, acc4[j][1]);
+              acc4[j][2] = fmaf(x, hi.x, acc4[j][2]);
+              acc4[j][3] = fmaf(x, hi.y, acc4[j][3]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.empty[slot]);
+        if (++slot == uint32_t(a.ring_slots)) { slot = 0; phase ^= 1u; }
+      }
+      float *dst = acc + b.out_off;
+      if (sh.nseg == 1) {
+        if (ok) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (j < sh.cps)
+              red_add_v4(dst + 4 * (gi + tpr * j),
+                         make_float4(acc4[j][0], acc4[j][1], acc4[j][2], acc4[j][3]));
+        }
+      } else {
+        // several row phases: add them up in shared memory first (cps == 1)
+        float4 *scr = reinterpret_cast<float4 *>(s.vbuf);
+        scr[ph * ngrp + gi] = make_float4(acc4[0][0], acc4[0][1], acc4[0][2], acc4[0][3]);
+        cbar();
+        if (tid < ngrp && !aborted()) {
+          float4 v = scr[tid];
+          for (int q = 1; q < sh.nseg; ++q) v = add4(v, scr[q * ngrp + tid]);
+          red_add_v4(dst + 4 * tid, v);
+        }
+        cbar();
+      }
+    }
+    Tbase += c.ntiles;
+    cbar();
+    KP_END(t_gemv, PF_GEMV);
+    KP_END(t_gemv, PF_GEMV_K + k);
   }
 
   // ---- LM head epilogue: logits and the CTA's share of the argmax
   __device__ void lm_epilogue() {
     const StageCta &c = s.misc->sc[ST_LM];
     const int nseg = a.shape[ST_LM].nseg;
+    // bidx starts at a row of this CTA so that the key always names a valid
+    // token; a NaN logit never wins a comparison and raises DE_NONFINITE.
     float best = -INFINITY;
-    int bidx = 0x7fffffff;
+    int bidx = c.row0;
     for (int i = tid; i < c.nout; i += kNC) {
       const float v = rowsum(i, nseg);
       const int row = c.row0 + i;
       if (a.logits_out) a.logits_out[size_t(step) * a.vocab + row] = v;
+      if (v != v) raise_error(a, DE_NONFINITE | (uint32_t(step & 0xffff) << 8));
       if (v > best || (v == best && row < bidx)) { best = v; bidx = row; }
     }
     for (int o = 16; o; o >>= 1) {
@@ -846,124 +983,132 @@ struct Consumer {
     const bool lanes = a.n_lanes > 1;
     const int delta = a.lane_delay;
     const uint32_t nc = a.n_ctas;
+    const int Hkv = a.n_kv_heads;
+    const int g = cta % Hkv;                              // this CTA's KV-head group
+    const uint32_t ng = uint32_t((a.n_ctas - 1 - g) / Hkv + 1);
+    const int own_lo = int(int64_t(d) * cta / a.n_ctas);  // residual rows this CTA owns
+    const int own_hi = int(int64_t(d) * (cta + 1) / a.n_ctas);
     tok = a.forced ? a.forced[0] : a.first_token;
     for (step = 0; step < a.n_steps; ++step) {
       p = a.pos0 + step;
+      // Every CTA sees the same token, so all of them leave together here
+      // before an embedding row outside the table could be read.
+      if (unsigned(tok) >= unsigned(a.vocab)) {
+        raise_error(a, DE_NONFINITE | (uint32_t(step & 0xffff) << 8));
+        goto done;
+      }
       const bool lm = a.logits_every_step || step == a.n_steps - 1;
       for (l = 0; l < L; ++l) {
-        const uint32_t e = uint32_t(step) * L + l + 1;  // epoch of this (step, layer)
-        // ---------------- RMSNorm + QKV
-        if (l > 0 && !gate(SY_X2, (e - 1) * nc, 0x10 + ST_QKV)) goto done;
-        stage_norm([=](int j) { return xin4(j); }, a.gain_attn + size_t(l) * d, d, a.lane_width);
+        gl = uint32_t(step) * L + l;
+        const uint32_t cur = gl & 1u, prev = (gl - 1) & 1u;
+        // ---------------- RMSNorm + q/k/v rows of the group
+        // (every CTA's down contribution to the previous layer is in)
+        if (gl > 0 && !gate(SY_S2, gl * nc, 0x10, 1)) goto done;
+        stage_norm([=](int j) { return xin4(j); }, a.gain_attn + size_t(l) * d, d, a.lane_width,
+                   a.xres + size_t(cur) * d, own_lo, own_hi);
         gemv(ST_QKV, s.vbuf, false);
         if (aborted()) goto done;
         {
           const StageCta &c = s.misc->sc[ST_QKV];
           const int nseg = a.shape[ST_QKV].nseg;
-          for (int i = tid; i < c.nout; i += kNC) a.qkv[c.row0 + i] = rowsum(i, nseg);
+          for (int bi = 0; bi < c.nblk; ++bi) {
+            const Block b = s.misc->blk[c.blk_begin + bi];
+            for (int i = tid; i < b.nrows; i += kNC) a.qkv[b.out_off + i] = rowsum(b.lrow0 + i, nseg);
+          }
         }
-        if (!(a.skip_signal_cta == cta && step == 0 && l == 0)) signal(SY_QKV);
+        if (!(a.skip_signal_cta == cta && step == 0 && l == 0)) signal(SY_QG0 + g);
         // ---------------- delayed cross-lane sum of the previous layer
         if (lanes && l >= 1) {
-          gemv(ST_MIX, a.ubuf + size_t((l - 1) & 1) * d, true);
+          const float4 *uo = vec4(a.acc_o, prev), *ud = vec4(a.acc_d, prev);
+          for (int j = tid; j < (d >> 2); j += kNC)
+            reinterpret_cast<float4 *>(s.vbuf)[j] = add4(__ldcg(uo + j), __ldcg(ud + j));
+          cbar();
+          gemv(ST_MIX, s.vbuf, false);
           if (aborted()) goto done;
           const StageCta &c = s.misc->sc[ST_MIX];
           const int nseg = a.shape[ST_MIX].nseg;
           float *dst = a.dsum + size_t((l - 1) % delta) * d;
           for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(i, nseg);
         }
-        // ---------------- attention
-        if (!gate(SY_QKV, e * nc, 0x20)) goto done;
-        attention();
-        // ---------------- O + residual
-        if (!gate(SY_OREADY, e * uint32_t(a.n_kv_heads), 0x30)) goto done;
+        // ---------------- attention of the group, merged in every group CTA
         {
-          // residual rows this CTA updates, fetched while the GEMV runs
-          const StageCta &c = s.misc->sc[ST_O];
-          const float xr = tid < c.nout ? xin(c.row0 + tid) : 0.f;
-          gemv(ST_O, a.attn_o, true);
-          if (aborted()) goto done;
-          const int nseg = a.shape[ST_O].nseg;
-          if (tid < c.nout) {
-            const int r = c.row0 + tid;
-            const float v = rowsum(tid, nseg);
-            a.x[r] = xr + v;
-            if (lanes) a.ubuf[size_t(l & 1) * d + r] = v;
-          }
-          for (int i = tid + kNC; i < c.nout; i += kNC) {
-            const int r = c.row0 + i;
-            const float v = rowsum(i, nseg);
-            a.x[r] = xin(r) + v;
-            if (lanes) a.ubuf[size_t(l & 1) * d + r] = v;
-          }
+          KvWords kw;
+          attention_prefetch(kw);
+          if (!gate(SY_QG0 + g, (gl + 1) * ng, 0x20, 4)) goto done;
+          attention(kw);
         }
-        signal(SY_X1);
-        // ---------------- RMSNorm + gate/up + SwiGLU
-        if (!gate(SY_X1, e * nc, 0x40)) goto done;
-        stage_norm([=](int j) { return __ldcg(reinterpret_cast<const float4 *>(a.x) + j); },
-                   a.gain_ffn + size_t(l) * d, d, a.lane_width);
+        if (aborted()) goto done;
+        // ---------------- O projection over the group's attention outputs
+        gemv_cols(ST_O, s.svec + s.misc->sc[ST_O].row0, a.acc_o + size_t(cur) * d);
+        if (aborted()) goto done;
+        signal(SY_S1);
+        // ---------------- RMSNorm + gate/up + SwiGLU of this CTA's hidden slice
+        if (!gate(SY_S1, (gl + 1) * nc, 0x40, 0)) goto done;
+        // the previous layer's accumulators were read by every CTA before S1;
+        // clear this CTA's rows of them for the layer after next
+        if (gl > 0)
+          for (int r = own_lo + tid; r < own_hi; r += kNC) {
+            a.acc_o[size_t(prev) * d + r] = 0.f;
+            a.acc_d[size_t(prev) * d + r] = 0.f;
+          }
+        {
+          const float4 *xr = vec4(a.xres, cur), *ao = vec4(a.acc_o, cur);
+          stage_norm([=](int j) { return add4(__ldcg(xr + j), __ldcg(ao + j)); },
+                     a.gain_ffn + size_t(l) * d, d, a.lane_width);
+        }
         gemv(ST_GU, s.vbuf, false);
         if (aborted()) goto done;
         {
           const StageCta &c = s.misc->sc[ST_GU];
           const int nseg = a.shape[ST_GU].nseg;
+          float *h = s.svec + kSvecO;
           for (int i = tid; i < c.nout; i += kNC) {
             const float gt = rowsum(i, nseg), up = rowsum(c.nout + i, nseg);
-            a.hbuf[c.row0 + i] = gt / (1.f + expf(-gt)) * up;
+            h[i] = gt / (1.f + expf(-gt)) * up;
           }
+          cbar();
         }
-        signal(SY_H);
-        // ---------------- down + residual
-        if (!gate(SY_H, e * nc, 0x50)) goto done;
-        {
-          const StageCta &c = s.misc->sc[ST_D];
-          const float xr = tid < c.nout ? __ldcg(a.x + c.row0 + tid) : 0.f;
-          gemv(ST_D, a.hbuf, true);
-          if (aborted()) goto done;
-          const int nseg = a.shape[ST_D].nseg;
-          if (tid < c.nout && !lanes) a.x[c.row0 + tid] = xr + rowsum(tid, nseg);
-          for (int i = (lanes ? tid : tid + kNC); i < c.nout; i += kNC) {
-            const int r = c.row0 + i;
-            const float v = rowsum(i, nseg);
-            a.x[r] = __ldcg(a.x + r) + v;
-            if (lanes) {
-              float *u = a.ubuf + size_t(l & 1) * d + r;
-              *u = __ldcg(u) + v;
-            }
-          }
-        }
-        signal(SY_X2);
+        // ---------------- down projection over that slice
+        gemv_cols(ST_D, s.svec + kSvecO, a.acc_d + size_t(cur) * d);
+        if (aborted()) goto done;
+        signal(SY_S2);
       }
       if (lm) {
         ++lm_count;
-        if (!gate(SY_X2, (uint32_t(step) * L + L) * nc, 0x60)) goto done;
+        const uint32_t last = gl & 1u;   // parity of the last layer
+        if (!gate(SY_S2, (gl + 1) * nc, 0x60, 1)) goto done;
         if (lanes) {
           // the last layer's delayed sum, flushed before the final norm
-          gemv(ST_MIX, a.ubuf + size_t((L - 1) & 1) * d, true);
+          const float4 *uo = vec4(a.acc_o, last), *ud = vec4(a.acc_d, last);
+          for (int j = tid; j < (d >> 2); j += kNC)
+            reinterpret_cast<float4 *>(s.vbuf)[j] = add4(__ldcg(uo + j), __ldcg(ud + j));
+          cbar();
+          gemv(ST_MIX, s.vbuf, false);
           if (aborted()) goto done;
           const StageCta &c = s.misc->sc[ST_MIX];
           const int nseg = a.shape[ST_MIX].nseg;
           float *dst = a.dsum + size_t((L - 1) % delta) * d;
           for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(i, nseg);
           signal(SY_MIXF);
-          if (!gate(SY_MIXF, lm_count * nc, 0x70)) goto done;
+          if (!gate(SY_MIXF, lm_count * nc, 0x70, 2)) goto done;
         }
-        stage_norm(
-            [=](int j) {
-              float4 v = __ldcg(reinterpret_cast<const float4 *>(a.x) + j);
-              if (lanes)
-                for (int li = (L > delta ? L - delta : 0); li < L; ++li) {
-                  const float4 q = __ldcg(reinterpret_cast<const float4 *>(a.dsum + size_t(li % delta) * d) + j);
-                  v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
-                }
-              return v;
-            },
-            a.gain_final, d, d);
+        {
+          const float4 *xr = vec4(a.xres, last), *ao = vec4(a.acc_o, last), *ad = vec4(a.acc_d, last);
+          stage_norm(
+              [=](int j) {
+                float4 v = add4(add4(__ldcg(xr + j), __ldcg(ao + j)), __ldcg(ad + j));
+                if (lanes)
+                  for (int li = (L > delta ? L - delta : 0); li < L; ++li)
+                    v = add4(v, __ldcg(reinterpret_cast<const float4 *>(a.dsum + size_t(li % delta) * d) + j));
+                return v;
+              },
+              a.gain_final, d, d);
+        }
         gemv(ST_LM, s.vbuf, false);
         if (aborted()) goto done;
         lm_epilogue();
         signal(SY_TOK);
-        if (!gate(SY_TOK, lm_count * nc, 0x80)) goto done;
+        if (!gate(SY_TOK, lm_count * nc, 0x80, 3)) goto done;
         const unsigned long long key = __ldcg(a.keys + step);
         const int next = int(0xffffffffu - uint32_t(key & 0xffffffffull));
         if (cta == 0 && tid == 0) a.out_tokens[step] = next;
@@ -988,7 +1133,8 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
   s.empty = s.full + NS;
   s.vbuf = reinterpret_cast<float *>(s.empty + NS);
   s.part = s.vbuf + a.vbuf_floats;
-  s.misc = reinterpret_cast<Misc *>(s.part + a.part_floats);
+  s.svec = s.part + a.part_floats;
+  s.misc = reinterpret_cast<Misc *>(s.svec + kSvecFloats);
 
   const int b0 = a.cta_blk_begin[cta], b1 = a.cta_blk_begin[cta + 1];
   for (int i = tid; i < b1 - b0; i += kThreads) s.misc->blk[i] = a.blocks[b0 + i];
@@ -1010,11 +1156,11 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
 #ifdef KIE_PROFILE
       const long long t0 = clock64();
 #endif
-      Pump pm(a, s);
-      pm.run(cta);
+      Producer pr(a, s, cta);
+      pr.run();
 #ifdef KIE_PROFILE
       s.misc->prof[PF_PROD_TOTAL] += clock64() - t0;
-      s.misc->prof[PF_TILES] = s.misc->pump.T;
+      s.misc->prof[PF_TILES] = pr.T;
 #endif
     }
     __syncwarp();
@@ -1031,32 +1177,46 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
 }
 
 // ------------------------------------------------------------------ weight repack
-// Copies each block of canonical row-major rows into tile order: row groups of
-// R rows, each split into K/KT column segments stored as R x KT row-major.
-__global__ void repack_kernel(const uint16_t *__restrict__ src, uint8_t *__restrict__ dst,
-                              const RepackJob *__restrict__ jobs, int njobs) {
-  for (int j = blockIdx.x; j < njobs; j += gridDim.x) {
-    const RepackJob job = jobs[j];
-    const int64_t K = job.K, KT = job.KT, R = job.R;
-    const int64_t nvec = int64_t(job.nrows) * K / 8;
+// Builds the per-SM weight streams from the canonical weights.  A plain job
+// copies nrows canonical rows as they are; a transposed job writes nrows
+// columns of a row-major [K, src_ld] matrix as rows of K elements (through a
+// 32 x 32 shared-memory tile so that both sides stay coalesced).
+__global__ void __launch_bounds__(256) repack_kernel(const uint16_t *__restrict__ src,
+                                                     uint8_t *__restrict__ dst,
+                                                     const RepackJob *__restrict__ jobs, int njobs) {
+  __shared__ uint16_t tile[32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int jb = blockIdx.x; jb < njobs; jb += gridDim.x) {
+    const RepackJob job = jobs[jb];
     uint16_t *out = reinterpret_cast<uint16_t *>(dst + job.dst_byte);
-    for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
-      const int64_t e = v * 8;             // element index in row-major source order
-      const int64_t i = e / K, k = e - i * K;
-      const int64_t g = i / R, ii = i - g * R;
-      const int64_t rg = min(R, int64_t(job.nrows) - g * R);
-      const int64_t sg = k / KT, kk = k - sg * KT;
-      const int64_t o = g * R * K + sg * rg * KT + ii * KT + kk;
-      *reinterpret_cast<uint4 *>(out + o) =
-          *reinterpret_cast<const uint4 *>(src + job.src_elem + e);
+    const uint16_t *in = src + job.src_elem;
+    if (!job.trans) {
+      const int64_t nvec = int64_t(job.nrows) * job.K / 8;
+      for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x)
+        reinterpret_cast<uint4 *>(out)[v] = *reinterpret_cast<const uint4 *>(in + v * 8);
+      continue;
     }
+    const int ncol = job.nrows, K = job.K;
+    for (int r0 = 0; r0 < K; r0 += 32)
+      for (int c0 = 0; c0 < ncol; c0 += 32) {
+        for (int rr = ty; rr < 32; rr += 8) {
+          const int r = r0 + rr, cc = c0 + tx;
+          tile[rr][tx] = (r < K && cc < ncol) ? in[int64_t(r) * job.src_ld + cc] : uint16_t(0);
+        }
+        __syncthreads();
+        for (int ii = ty; ii < 32; ii += 8) {
+          const int cc = c0 + ii, r = r0 + tx;
+          if (cc < ncol && r < K) out[int64_t(cc) * K + r] = tile[tx][ii];
+        }
+        __syncthreads();
+      }
   }
 }
 
 // ------------------------------------------------------------------ host entry points
 size_t monokernel_smem_bytes(int ring_slots, int vbuf_floats, int part_floats) {
   return size_t(ring_slots) * kSlotBytes + size_t(ring_slots) * 16 +
-         size_t(vbuf_floats + part_floats) * 4 + sizeof(Misc);
+         size_t(vbuf_floats + part_floats + kSvecFloats) * 4 + sizeof(Misc);
 }
 
 int monokernel_threads() { return kThreads; }

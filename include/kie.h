@@ -24,8 +24,9 @@
  *   - returns KIE_OK (0) or a negative kie_status; kie_strerror() names it;
  *   - calls are synchronous: they return after the work queued on the
  *     context's stream has finished;
- *   - after KIE_ERR_DEVICE_TIMEOUT or KIE_ERR_CUDA the context is poisoned:
- *     every later call except kie_destroy returns the same error.
+ *   - after KIE_ERR_DEVICE_TIMEOUT, KIE_ERR_NONFINITE or KIE_ERR_CUDA the
+ *     context is poisoned:
+ *     every later call except kie_destroy returns KIE_ERR_POISONED.
  *   - a context is not thread-safe; use one per host thread.
  */
 #ifndef KIE_H
@@ -45,7 +46,9 @@ typedef enum {
   KIE_ERR_CAPACITY = -4,       /* pos + n would exceed max_seq */
   KIE_ERR_NOT_RESIDENT = -5,   /* the persistent grid cannot be co-resident */
   KIE_ERR_DEVICE_TIMEOUT = -6, /* a bounded in-kernel wait ran out (watchdog) */
-  KIE_ERR_POISONED = -7        /* an earlier device error poisoned this context */
+  KIE_ERR_POISONED = -7,       /* an earlier device error poisoned this context */
+  KIE_ERR_NONFINITE = -8       /* a NaN logit, or a token id outside [0, vocab), met
+                                  on the device; the kernel stops before using it */
 } kie_status;
 
 typedef enum { KIE_F16 = 0, KIE_BF16 = 1 } kie_dtype;
@@ -169,6 +172,18 @@ int kie_get_profile(const kie_ctx *ctx, uint64_t *out, int32_t n_words);
  *     next launch, so the other CTAs' waits must run out and the call must
  *     return KIE_ERR_DEVICE_TIMEOUT.  Reset to -1 after one launch. */
 int kie_debug_set(kie_ctx *ctx, int32_t watchdog_ms, int32_t skip_signal_cta);
+
+/* How the persistent kernel's SMs wait for one another (applies to later
+ * launches of this context; results are the same in both modes).
+ *   KIE_SYNC_DEPENDENCY (default): each wait is for exactly the SMs whose
+ *     output it reads -- the KV-head group for q/k/v and attention partials,
+ *     every SM only for the two residual updates of a layer.
+ *   KIE_SYNC_GRID: every wait is a grid-wide barrier across all SMs, the
+ *     scheme the monokernel page reports as a third of per-token time on
+ *     conventional stacks; kept as a measured ablation.
+ * Returns KIE_ERR_INVALID for any other mode. */
+enum { KIE_SYNC_DEPENDENCY = 0, KIE_SYNC_GRID = 1 };
+int kie_set_sync_mode(kie_ctx *ctx, int32_t mode);
 
 #ifdef __cplusplus
 }

@@ -2,6 +2,7 @@
 rejects bad descriptors on the host (no GPU needed: validation runs before any
 CUDA call)."""
 import ctypes
+import os
 import subprocess
 
 import pytest
@@ -26,6 +27,25 @@ def test_exports_every_declared_function(lib):
     assert not missing, missing
     for n in names:
         getattr(lib, n)
+
+
+def test_ubench_library_exports_its_header(lib):
+    from decode_persistent_monokernel_b200 import ceilings
+    hdr = os.path.join(os.path.dirname(kie.HEADER), "kie_ubench.h")
+    names = kie.header_functions(hdr)
+    assert set(names) == {"kie_ubench_launch_overhead", "kie_ubench_stream",
+                          "kie_ubench_barrier"}
+    out = subprocess.check_output(["nm", "-D", "--defined-only", ceilings.LIB_PATH], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    assert set(names) <= exported
+    ub = ceilings.load()
+    f = ctypes.c_float()
+    # argument checks happen before any device work
+    assert ub.kie_ubench_launch_overhead(0, ctypes.byref(f)) == -1
+    assert ub.kie_ubench_stream(None, 32768, 1, 1, 6, 1, ctypes.byref(f)) == -1
+    assert ub.kie_ubench_stream(ctypes.c_void_p(256), 1000, 1, 1, 6, 1, ctypes.byref(f)) == -1
+    assert ub.kie_ubench_stream(ctypes.c_void_p(256), 32768, 1, 1, 7, 1, ctypes.byref(f)) == -1
+    assert ub.kie_ubench_barrier(0, 10, ctypes.byref(f)) == -1
 
 
 def test_build_targets_sm100a_only():
@@ -75,3 +95,5 @@ def test_null_context_calls_rejected(lib):
     assert lib.kie_get_stats(None, None) == kie.KIE_ERR_INVALID
     assert "invalid" in kie.strerror(kie.KIE_ERR_INVALID)
     assert "watchdog" in kie.strerror(kie.KIE_ERR_DEVICE_TIMEOUT)
+    assert "non-finite" in kie.strerror(kie.KIE_ERR_NONFINITE)
+    assert lib.kie_set_sync_mode(None, kie.KIE_SYNC_GRID) == kie.KIE_ERR_INVALID

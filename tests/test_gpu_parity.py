@@ -95,7 +95,9 @@ def test_tiny_free_run_teacher_forced_and_cache():
     dec.kie_destroy()
 
 
-def test_tiny_is_deterministic():
+def test_tiny_is_repeatable():
+    """Two launches agree to float rounding.  The split projections are summed
+    with atomics, so the summation order (and the last bits) may differ."""
     w = synth.WORKLOADS[0]
     m = w.model
     bits = synth.generate_weights(m, w.weight_seed)
@@ -107,7 +109,28 @@ def test_tiny_is_deterministic():
         dec.kie_prefill(prompt)
         runs.append(_gpu_logits(dec, 24, m.vocab, forced)[1])
         dec.kie_destroy()
-    np.testing.assert_array_equal(runs[0].view(np.uint32), runs[1].view(np.uint32))
+    a, b = runs[0].astype(np.float64), runs[1].astype(np.float64)
+    rel = np.linalg.norm(a - b, axis=1) / np.linalg.norm(a, axis=1)
+    assert rel.max() < 1e-5, rel.max()
+
+
+@pytest.mark.parametrize("shape", ["tiny", "lanes2_d2"])
+def test_grid_barrier_mode_matches_oracle(shape):
+    """The grid-barrier ablation (every dependency wait across all SMs) gives
+    the same results as the per-dependency counters."""
+    import decode_persistent_monokernel_b200 as kie
+    m = synth.WORKLOADS[0].model if shape == "tiny" else _VARIANTS[shape]
+    bits = synth.generate_weights(m, 77)
+    prompt = synth.prompt(synth.WORKLOADS[0])
+    forced = synth.forced_tokens(synth.WORKLOADS[0], 12) % m.vocab
+    dec = make_decoder(m, bits, 40)
+    dec.kie_set_sync_mode(kie.KIE_SYNC_GRID)
+    dec.kie_prefill(prompt)
+    toks, z = _gpu_logits(dec, 12, m.vocab, forced.astype(np.int32))
+    dec.kie_destroy()
+    z_ora = Oracle(m, bits, 40).teacher_forced_logits(prompt, forced)
+    check_logits(z, z_ora, f"{shape} grid barriers")
+    check_argmax(toks, z_ora, f"{shape} grid barriers")
 
 
 _TINY = synth.WORKLOADS[0].model
@@ -271,4 +294,25 @@ def test_errors_and_capacity():
     assert e.value.code == kie.KIE_ERR_CAPACITY
     # the context is still usable after host-side rejections
     assert dec.kie_prefill(np.arange(3, dtype=np.int32)) >= 0
+    dec.kie_destroy()
+
+
+def test_nonfinite_logits_stop_the_kernel():
+    """A NaN in one LM-head row makes that logit NaN: the kernel reports
+    KIE_ERR_NONFINITE (it never turns a NaN argmax into a token id) and the
+    context is poisoned afterwards."""
+    import decode_persistent_monokernel_b200 as kie
+    w = synth.WORKLOADS[0]
+    m = w.model
+    bits = synth.generate_weights(m, w.weight_seed).copy()
+    head = [t for t in synth.tensor_table(m) if t.name == "lm_head"][0]
+    row = m.vocab // 3
+    bits[head.offset + row * m.d_model] = 0x7E00           # fp16 quiet NaN
+    dec = make_decoder(m, bits, 16)
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_prefill(np.arange(4, dtype=np.int32))
+    assert e.value.code == kie.KIE_ERR_NONFINITE
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_decode(1)
+    assert e.value.code == kie.KIE_ERR_POISONED
     dec.kie_destroy()

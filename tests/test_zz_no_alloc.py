@@ -11,7 +11,8 @@ import numpy as np
 import pytest
 
 import synth
-from tests.gpu_util import check_logits, make_decoder
+from oracle import top2_margin
+from tests.gpu_util import NEAR_TIE, check_argmax, check_logits, make_decoder
 
 pytestmark = pytest.mark.gpu
 
@@ -44,8 +45,18 @@ def test_static_scratch_decode_matches_decode_ex(teacher_forced):
     chunks = (10, 14)                       # two calls in a row
     t_ref, z_ref = _run(dec, dec.kie_decode_ex, prompt, forced, chunks, m.vocab)
     t_new, z_new = _run(dec, dec.kie_decode_ex_static, prompt, forced, chunks, m.vocab)
-    np.testing.assert_array_equal(t_new, t_ref)
-    check_logits(z_new, z_ref, "static scratch")
+    # the split projections are summed with atomics, so two launches may differ
+    # in the last bits: compare logits within the tests' tolerance and tokens by
+    # the near-tie rule; a free run may part ways only at a near tie
+    n = len(t_ref)
+    if not teacher_forced:
+        for k in range(n):
+            if t_new[k] != t_ref[k]:
+                assert top2_margin(z_ref[k]) < NEAR_TIE, (k, t_new[k], t_ref[k])
+                n = k + 1
+                break
+    check_logits(z_new[:n], z_ref[:n], "static scratch")
+    check_argmax(t_new[:n], z_ref[:n], "static scratch")
     assert dec.kie_get_stats().pos == len(prompt) + sum(chunks)
     dec.kie_destroy()
 
