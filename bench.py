@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="bounded CPU work for the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sync", choices=["dependency", "grid"], default="dependency",
+                    help="how SMs wait for one another: per-dependency counters (default) or "
+                         "a grid-wide barrier at every dependency point (ablation)")
     ap.add_argument("--profile", action="store_true",
                     help="run the profiling build (libkie_prof.so) and report where each "
                          "SM's time goes; its timings are not the benchmark value")
@@ -69,7 +72,9 @@ def profile_summary(prof, steps, mhz):
     out["dependency_waits_per_step"] = round(float(prof[:, 11].mean() / steps), 1)
     stages = ["qkv", "o", "gate_up", "down", "mix", "lm_head"]
     out["gemv_by_stage_us"] = {n: round(float(us[:, 12 + i].mean()), 1) for i, n in enumerate(stages)}
-    gates = ["qkv_done", "attn_merged", "o_done", "gate_up_done", "down_done", "mix_flush", "token"]
+    # dependency counters in the kernel's order: after O (grid), after down
+    # (grid), lane-mix flush, token, q/k/v of the KV group, attention partials
+    gates = ["o_done_grid", "down_done_grid", "mix_flush", "token", "qkv_group", "attn_group"]
     out["wait_by_counter_us"] = {n: round(float(us[:, 18 + i].mean()), 1) for i, n in enumerate(gates)}
     out["wait_by_counter_min_us"] = {n: round(float(us[:, 18 + i].min()), 1) for i, n in enumerate(gates)}
     out["tiles_per_step"] = round(float(prof[:, 10].mean() / steps), 1)
@@ -221,6 +226,8 @@ def main():
     wdev = torch.from_numpy(bits.view(np.int16)).cuda()
     stream = torch.cuda.current_stream()
     dec = kie.Decoder(kie.make_desc(m, max_seq), wdev, stream=stream)
+    if args.sync == "grid":
+        dec.kie_set_sync_mode(kie.KIE_SYNC_GRID)
     del wdev
     torch.cuda.empty_cache()
     st = dec.kie_get_stats()
@@ -267,6 +274,7 @@ def main():
         else "f32 (bf16 weights/KV)", "data": "synthetic (seeded weights and prompt)",
         "config": {"workload": w.name, "prompt": P, "decode_steps": K, "batch": 1,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "sync": args.sync,
                    "l2": "inputs larger than L2: %.2f GB of weights streamed per step"
                          % (st.weight_bytes_per_step / 1e9)},
         "us_per_token": 1e3 * ms / K,

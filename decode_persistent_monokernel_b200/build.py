@@ -1,4 +1,5 @@
-"""Builds libkie.so (the C-ABI decode library) in-tree with nvcc for sm_100a."""
+"""Builds libkie.so (the C-ABI decode library), its profiling twin and the
+micro-benchmark library libkie_ubench.so in-tree with nvcc for sm_100a."""
 from __future__ import annotations
 
 import os
@@ -12,6 +13,9 @@ SOURCES = ["kie_api.cu", "monokernel.cu"]
 HEADERS = ["kie_internal.h", os.path.join("..", "..", "include", "kie.h")]
 LIB = os.path.join(HERE, "libkie.so")
 PROF_LIB = os.path.join(HERE, "libkie_prof.so")  # activity counters compiled in
+UBENCH_LIB = os.path.join(HERE, "libkie_ubench.so")  # micro-benchmarks (kie_ubench.h)
+UBENCH_SOURCES = ["ubench.cu"]
+UBENCH_HEADERS = [os.path.join("..", "..", "include", "kie_ubench.h")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -28,20 +32,22 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def _stale(lib: str) -> bool:
+def _stale(lib: str, sources, headers) -> bool:
     if not os.path.exists(lib):
         return True
     t = os.path.getmtime(lib)
-    deps = [os.path.join(CSRC, s) for s in SOURCES + HEADERS]
+    deps = [os.path.join(CSRC, s) for s in sources + headers]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def _build_one(lib: str, extra, force: bool, verbose: bool) -> str:
-    if not force and not _stale(lib):
+def _build_one(lib: str, extra, force: bool, verbose: bool, sources=None, headers=None) -> str:
+    sources = SOURCES if sources is None else sources
+    headers = HEADERS if headers is None else headers
+    if not force and not _stale(lib, sources, headers):
         return lib
     tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"),
-           *[os.path.join(CSRC, s) for s in SOURCES], "-o", tmp]
+           *[os.path.join(CSRC, s) for s in sources], "-o", tmp]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
@@ -59,6 +65,7 @@ def build(force: bool = False, verbose: bool = False, profile: bool = True) -> s
     _build_one(LIB, [], force, verbose)
     if profile:
         _build_one(PROF_LIB, ["-DKIE_PROFILE"], force, False)
+    _build_one(UBENCH_LIB, [], force, False, UBENCH_SOURCES, UBENCH_HEADERS)
     return LIB
 
 
