@@ -77,9 +77,40 @@ def profile_summary(prof, steps, mhz):
     gates = ["o_done_grid", "down_done_grid", "mix_flush", "token", "qkv_group", "attn_group"]
     out["wait_by_counter_us"] = {n: round(float(us[:, 18 + i].mean()), 1) for i, n in enumerate(gates)}
     out["wait_by_counter_min_us"] = {n: round(float(us[:, 18 + i].min()), 1) for i, n in enumerate(gates)}
+    out["tile_wait_per_warp_us"] = {n: round(float(us[:, 24 + i].mean()), 1)
+                                     for i, n in enumerate(["mean", "max", "min"])}
     out["tiles_per_step"] = round(float(prof[:, 10].mean() / steps), 1)
     out["clock_mhz_used"] = mhz
     return out
+
+
+TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                            "monokernel_traffic.json")
+
+
+def kernel_sources_digest(files):
+    import hashlib
+    h = hashlib.sha256()
+    root = os.path.dirname(os.path.abspath(__file__))
+    for f in files:
+        with open(os.path.join(root, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def dram_traffic(algorithmic_bytes):
+    """DRAM bytes of the timed launch, from the last hardware-counter capture of
+    the decode kernel: that capture's DRAM bytes / algorithmic bytes, times this
+    launch's algorithmic bytes (the traffic scales with the bytes streamed).
+    None when there is no capture or the kernel sources changed since."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+        if kernel_sources_digest(rec["files"]) != rec["kernel_sources_sha256"]:
+            return None, "kernel changed since the last counter capture"
+        return rec["ratio"] * algorithmic_bytes, rec["capture"]
+    except (OSError, KeyError, ValueError):
+        return None, "no counter capture recorded"
 
 
 def peak_hbm():
@@ -265,6 +296,7 @@ def main():
 
     total_bytes = workload_bytes(m, P, K, st.weight_bytes_per_step, st.kv_bytes_per_position)
     peak, peak_kind = peak_hbm()
+    traffic, traffic_src = dram_traffic(total_bytes)
     achieved = total_bytes / (kernel_ms * 1e-3) / 1e9
     value = world * K / (ms * 1e-3)
     line = {
@@ -281,8 +313,8 @@ def main():
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_8TBps_nominal": achieved / 8000.0,
-                     "bytes_per_step": total_bytes / K, "traffic": None,
-                     "kernel_ms": kernel_ms},
+                     "bytes_per_step": total_bytes / K, "traffic": traffic,
+                     "traffic_source": traffic_src, "kernel_ms": kernel_ms},
         "clocks": clk.summary(),
         "gpu_launches": 1,
         "e2e": {"value": world * K / e2e_s,

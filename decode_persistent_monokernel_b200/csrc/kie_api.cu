@@ -336,6 +336,11 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
   if (fixed + 3 * (kSlotBytes + 16) > smem_cap) return "shape needs more shared memory than the SM has";
   int slots = int((smem_cap - fixed) / (kSlotBytes + 16));
   slots = std::min(slots, 16);
+  // tuning override (never above what shared memory holds)
+  if (const char *env = getenv("KIE_RING_SLOTS")) {
+    const long v = atol(env);
+    if (v >= 2 && v < slots) slots = int(v);
+  }
   P.ring_slots = slots;
   P.smem = monokernel_smem_bytes(slots, P.vbuf_floats, P.part_floats);
   P.max_split = std::min((n_ctas + Hkv - 1) / Hkv, kMaxSplit);

@@ -48,6 +48,7 @@ enum ProfSlot : int {
   PF_NGATE = 11,      // number of dependency waits
   PF_GEMV_K = 12,     // 12..17: time per stage kind
   PF_GATE_K = 18,     // 18..23: waiting time on S1, S2, MIXF, TOK, q/k/v group, attention group
+  PF_WAIT_ALL = 24,   // 24..26: tile waits per consumer warp: mean, max, min over warps
 };
 constexpr int kProfSlots = 32;
 

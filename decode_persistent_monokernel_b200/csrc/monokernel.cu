@@ -151,13 +151,14 @@ template <> struct Store<__nv_bfloat16> {
   }
 };
 
+// Eight weights times eight inputs, as two interleaved fp32 partial sums
+// (packed fp32x2 FMAs: one instruction per weight pair).
 template <typename T>
-__device__ __forceinline__ float dot8(uint4 w, float4 a, float4 b, float acc) {
-  float2 f;
-  f = Store<T>::pair(w.x); acc = fmaf(f.x, a.x, acc); acc = fmaf(f.y, a.y, acc);
-  f = Store<T>::pair(w.y); acc = fmaf(f.x, a.z, acc); acc = fmaf(f.y, a.w, acc);
-  f = Store<T>::pair(w.z); acc = fmaf(f.x, b.x, acc); acc = fmaf(f.y, b.y, acc);
-  f = Store<T>::pair(w.w); acc = fmaf(f.x, b.z, acc); acc = fmaf(f.y, b.w, acc);
+__device__ __forceinline__ float2 dot8x2(uint4 w, const float2 (&x)[4], float2 acc) {
+  acc = __ffma2_rn(Store<T>::pair(w.x), x[0], acc);
+  acc = __ffma2_rn(Store<T>::pair(w.y), x[1], acc);
+  acc = __ffma2_rn(Store<T>::pair(w.z), x[2], acc);
+  acc = __ffma2_rn(Store<T>::pair(w.w), x[3], acc);
   return acc;
 }
 
@@ -183,6 +184,7 @@ struct Misc {
   volatile int32_t abort;  // a consumer saw a failed wait
   int32_t flag;            // broadcast slot
   long long prof[kProfSlots];
+  long long wwait[kConsumerWarps];   // profiling build: tile waits per consumer warp
 };
 
 // Scalars of the column stages: the merged attention output of the CTA's KV
@@ -524,7 +526,7 @@ struct Consumer {
     for (int bi = 0; bi < c.nblk && ok; ++bi) {
       const Block b = s.misc->blk[c.blk_begin + bi];
       // this warp's slice of the input vector, kept in registers for the block
-      float vr[4][8];
+      float2 vr[4][4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         if (crow[i] != 0x7fffffff) {
@@ -532,11 +534,11 @@ struct Consumer {
           float4 x0, x1;
           if (vin_global) { x0 = __ldcg(reinterpret_cast<const float4 *>(src)); x1 = __ldcg(reinterpret_cast<const float4 *>(src) + 1); }
           else { x0 = reinterpret_cast<const float4 *>(src)[0]; x1 = reinterpret_cast<const float4 *>(src)[1]; }
-          vr[i][0] = x0.x; vr[i][1] = x0.y; vr[i][2] = x0.z; vr[i][3] = x0.w;
-          vr[i][4] = x1.x; vr[i][5] = x1.y; vr[i][6] = x1.z; vr[i][7] = x1.w;
+          vr[i][0] = make_float2(x0.x, x0.y); vr[i][1] = make_float2(x0.z, x0.w);
+          vr[i][2] = make_float2(x1.x, x1.y); vr[i][3] = make_float2(x1.z, x1.w);
         } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) vr[i][e] = 0.f;
+          for (int e = 0; e < 4; ++e) vr[i][e] = make_float2(0.f, 0.f);
         }
       }
       // Tiles go in batches of `batch` (4 / rpw) tiles: each tile's dot
@@ -552,11 +554,15 @@ struct Consumer {
           if (bt < batch && t0 + bt < ntile) {
             bool got = true;
 #ifdef KIE_PROFILE
-            const long long tw = (tid == 0) ? clock64() : 0ll;
+            const long long tw = (lane == 0) ? clock64() : 0ll;
 #endif
             if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [] {});
 #ifdef KIE_PROFILE
-            if (tid == 0) s.misc->prof[PF_FULLWAIT] += clock64() - tw;
+            if (lane == 0) {
+              const long long dt = clock64() - tw;
+              if (tid == 0) s.misc->prof[PF_FULLWAIT] += dt;
+              s.misc->wwait[warp] += dt;
+            }
 #endif
             got = __shfl_sync(0xffffffffu, got, 0);
             if (!got) {
@@ -565,22 +571,26 @@ struct Consumer {
             } else {
               const int rows = min(sh.R, b.nrows - (t0 + bt) * sh.R);
               const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes;
+              float2 d2[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                if (crow[i] < rows) {
-                  const float4 va = make_float4(vr[i][0], vr[i][1], vr[i][2], vr[i][3]);
-                  const float4 vb = make_float4(vr[i][4], vr[i][5], vr[i][6], vr[i][7]);
-                  const float d = dot8<T>(*reinterpret_cast<const uint4 *>(tile + off[i]), va, vb, 0.f);
-                  // value index: tile bt of the batch, row crow[i] - row0 of the
-                  // warp's rows (uniform across lanes); < 4 because batch * rpw == 4
-                  if (!MULTI) {
-                    val[bt] += d;
-                  } else {
-                    const int vidx = bt * sh.rpw + (crow[i] - row0);
+                d2[i] = make_float2(0.f, 0.f);
+                if (crow[i] < rows)
+                  d2[i] = dot8x2<T>(*reinterpret_cast<const uint4 *>(tile + off[i]), vr[i], d2[i]);
+              }
+              if (!MULTI) {
+                const float2 q = __fadd2_rn(__fadd2_rn(d2[0], d2[1]), __fadd2_rn(d2[2], d2[3]));
+                val[bt] += q.x + q.y;
+              } else {
+                // value index: tile bt of the batch, row crow[i] - row0 of the
+                // warp's rows (uniform across lanes); < 4 because batch * rpw == 4
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                      if (j == vidx) val[j] += d;
-                  }
+                for (int i = 0; i < 4; ++i) {
+                  const int vidx = bt * sh.rpw + (crow[i] - row0);
+                  const float d = d2[i].x + d2[i].y;
+#pragma unroll
+                  for (int j = 0; j < 4; ++j)
+                    if (crow[i] < rows && j == vidx) val[j] += d;
                 }
               }
               __syncwarp();
@@ -865,20 +875,22 @@ struct Consumer {
     bool ok = !aborted();
     for (int bi = 0; bi < c.nblk; ++bi) {
       const Block b = s.misc->blk[c.blk_begin + bi];
-      float acc4[4][4];
+      float2 acc4[4][2];   // output group j: elements (0,1) and (2,3)
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc4[j][e] = 0.f;
+      for (int j = 0; j < 4; ++j) acc4[j][0] = acc4[j][1] = make_float2(0.f, 0.f);
       const int ntile = (b.nrows + sh.R - 1) / sh.R;
       for (int t = 0; t < ntile && ok; ++t) {
         bool got = true;
 #ifdef KIE_PROFILE
-        const long long tw = (tid == 0) ? clock64() : 0ll;
+        const long long tw = (lane == 0) ? clock64() : 0ll;
 #endif
         if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [] {});
 #ifdef KIE_PROFILE
-        if (tid == 0) s.misc->prof[PF_FULLWAIT] += clock64() - tw;
+        if (lane == 0) {
+          const long long dt = clock64() - tw;
+          if (tid == 0) s.misc->prof[PF_FULLWAIT] += dt;
+          s.misc->wwait[warp] += dt;
+        }
 #endif
         got = __shfl_sync(0xffffffffu, got, 0);
         if (!got) {
@@ -891,16 +903,14 @@ struct Consumer {
         const float *sv = svals + b.lrow0 + t * sh.R;
         for (int r = ph; r < rows; r += sh.nseg) {
           const float x = sv[r];
+          const float2 xx = make_float2(x, x);
           const uint8_t *row = tile + size_t(r) * sh.K * 2;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             if (j < sh.cps) {
               const uint2 w = *reinterpret_cast<const uint2 *>(row + size_t(gi + tpr * j) * 8);
-              const float2 lo = Store<T>::pair(w.x), hi = Store<T>::pair(w.y);
-              acc4[j][0] = fmaf(x, lo.x, acc4[j][0]);
-              acc4[j][1] = fmaf(x, lo.y, acc4[j][1]);
-              acc4[j][2] = fmaf(x, hi.x, acc4[j][2]);
-              acc4[j][3] = fmaf(x, hi.y, acc4[j][3]);
+              acc4[j][0] = __ffma2_rn(Store<T>::pair(w.x), xx, acc4[j][0]);
+              acc4[j][1] = __ffma2_rn(Store<T>::pair(w.y), xx, acc4[j][1]);
             }
           }
         }
@@ -915,12 +925,12 @@ struct Consumer {
           for (int j = 0; j < 4; ++j)
             if (j < sh.cps)
               red_add_v4(dst + 4 * (gi + tpr * j),
-                         make_float4(acc4[j][0], acc4[j][1], acc4[j][2], acc4[j][3]));
+                         make_float4(acc4[j][0].x, acc4[j][0].y, acc4[j][1].x, acc4[j][1].y));
         }
       } else {
         // several row phases: add them up in shared memory first (cps == 1)
         float4 *scr = reinterpret_cast<float4 *>(s.vbuf);
-        scr[ph * ngrp + gi] = make_float4(acc4[0][0], acc4[0][1], acc4[0][2], acc4[0][3]);
+        scr[ph * ngrp + gi] = make_float4(acc4[0][0].x, acc4[0][0].y, acc4[0][1].x, acc4[0][1].y);
         cbar();
         if (tid < ngrp && !aborted()) {
           float4 v = scr[tid];
@@ -1147,6 +1157,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
     s.misc->abort = 0;
     s.misc->flag = 0;
     for (int i = 0; i < kProfSlots; ++i) s.misc->prof[i] = 0;
+    for (int i = 0; i < kConsumerWarps; ++i) s.misc->wwait[i] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -1172,6 +1183,18 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
   }
   __syncthreads();
 #ifdef KIE_PROFILE
+  if (tid == 0) {
+    long long sum = 0, mx = 0, mn = s.misc->wwait[0];
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      sum += s.misc->wwait[w];
+      mx = max(mx, s.misc->wwait[w]);
+      mn = min(mn, s.misc->wwait[w]);
+    }
+    s.misc->prof[PF_WAIT_ALL] = sum / kConsumerWarps;
+    s.misc->prof[PF_WAIT_ALL + 1] = mx;
+    s.misc->prof[PF_WAIT_ALL + 2] = mn;
+  }
+  __syncthreads();
   if (a.prof && tid < kProfSlots) a.prof[size_t(cta) * kProfSlots + tid] = s.misc->prof[tid];
 #endif
 }

@@ -160,8 +160,11 @@ int kie_copy_kv(const kie_ctx *ctx, int32_t layer, int32_t kv_head, int32_t pos0
  * stages, 3 waiting for weight tiles, 4 attention, 5 input staging and norm,
  * 6 end-of-stage barrier, 7 LM head, 8 producer blocked on a full ring,
  * 9 producer total, 10 tiles issued, 11 dependency waits, 12..17 GEMV time
- * per stage (QKV, O, gate/up, down, mix, LM head), 18..24 waiting time per
- * counter.  Only the profiling build (libkie_prof.so, compiled with
+ * per stage (QKV, O, gate/up, down, mix, LM head), 18..23 waiting time per
+ * dependency counter (after O, after down, lane-mix flush, token, q/k/v of
+ * the KV group, attention partials of the group), 24..26 waiting for weight
+ * tiles per consumer warp (mean, max, min over the 16 warps).  Only the
+ * profiling build (libkie_prof.so, compiled with
  * KIE_PROFILE) records them; the normal build returns KIE_ERR_INVALID.
  * n_words must be >= 32 * n_ctas. */
 int kie_get_profile(const kie_ctx *ctx, uint64_t *out, int32_t n_words);
