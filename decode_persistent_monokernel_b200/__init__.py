@@ -83,6 +83,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "kie_copy_kv": ([_P, _I, _I, _I, _I, _P, _P], _I),
         "kie_debug_set": ([_P, _I, _I], _I),
         "kie_set_sync_mode": ([_P, _I], _I),
+        "kie_trace_request": ([_P, _I, _I], _I),
+        "kie_get_trace": ([_P, _P, _I], _I),
         "kie_get_profile": ([_P, _P, _I], _I),
     }
     for name, (args, res) in sig.items():
@@ -189,6 +191,18 @@ class Decoder:
 
     def kie_debug_set(self, watchdog_ms: int, skip_signal_cta: int = -1) -> None:
         _check(load().kie_debug_set(self._h, watchdog_ms, skip_signal_cta))
+
+    def kie_trace_request(self, cta: int, step: int) -> None:
+        _check(load().kie_trace_request(self._h, cta, step))
+
+    def kie_get_trace(self):
+        """(clock, type, argument) triples of the last traced launch."""
+        import numpy as np
+        out = np.zeros(65537, dtype=np.uint64)
+        _check(load().kie_get_trace(self._h, out.ctypes.data, out.size))
+        n = int(min(out[0], out.size - 1))
+        ev = out[1:1 + n]
+        return ev >> np.uint64(8), (ev >> np.uint64(4)) & np.uint64(15), ev & np.uint64(15)
 
     def kie_set_sync_mode(self, mode: int) -> None:
         _check(load().kie_set_sync_mode(self._h, mode))

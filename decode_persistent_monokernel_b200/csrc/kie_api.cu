@@ -154,6 +154,7 @@ const char *make_cshape(int n_out, int in_len, StageShape &s) {
   int R = 1;
   while (R * 2 * 2 * n_out <= kSlotBytes && R < 64) R *= 2;
   s.R = R;
+  if ((R + s.nseg - 1) / s.nseg > 8) return "split projection tile has more than 8 rows per thread";
   s.rpw = 1;
   return nullptr;
 }
@@ -382,6 +383,8 @@ struct kie_ctx {
   int32_t *d_blk_begin = nullptr;
   int64_t *d_stream_off = nullptr;
   unsigned long long *prof = nullptr;  // [n_ctas][kProfSlots] (profiling build)
+  unsigned long long *trace = nullptr; // [1 + kTraceCap] (profiling build)
+  int trace_cta = 0, trace_step = -1;
   // activation buffer layout (floats): residual bases, the two layer
   // accumulators (both parities, contiguous so one memset clears them), q/k/v,
   // delayed sums, attention partials
@@ -429,7 +432,7 @@ static void free_ctx(kie_ctx *c) {
   if (!c) return;
   void *ptrs[] = {c->wstream, c->embed, c->gains, c->rope, c->kcache, c->vcache, c->act,
                   c->sync, c->keys, c->tokens_in, c->tokens_out, c->d_stage_cta, c->d_blocks,
-                  c->d_blk_begin, c->d_stream_off, c->prof};
+                  c->d_blk_begin, c->d_stream_off, c->prof, c->trace};
   for (void *p : ptrs)
     if (p) cudaFree(p);
   if (c->ev0) cudaEventDestroy(c->ev0);
@@ -539,6 +542,8 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
   if ((rc = alloc(ctx, (void **)&ctx->d_blk_begin, P.cta_blk_begin.size() * 4, "plan"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->d_stream_off, P.cta_stream_off.size() * 8, "plan"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->prof, size_t(P.n_ctas) * kProfSlots * 8, "profile"))) return fail(rc);
+  if (monokernel_profiled() &&
+      (rc = alloc(ctx, (void **)&ctx->trace, size_t(kTraceCap + 1) * 8, "trace"))) return fail(rc);
   RepackJob *d_jobs = nullptr;
   if ((rc = alloc(ctx, (void **)&d_jobs, P.jobs.size() * sizeof(RepackJob), "repack jobs"))) return fail(rc);
 
@@ -660,6 +665,13 @@ static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int fi
   ctx->skip_signal_cta = -1;
   a.grid_sync = ctx->grid_sync;
   a.prof = ctx->prof;
+  if (ctx->trace && ctx->trace_step >= 0 && ctx->trace_step < n) {
+    a.trace = ctx->trace;
+    a.trace_cap = kTraceCap;
+    a.trace_cta = ctx->trace_cta;
+    a.trace_step = ctx->trace_step;
+    CK(cudaMemsetAsync(ctx->trace, 0, 8, st));
+  }
 
   const size_t sync_words = size_t(SY_QG0 + 2 * m.n_kv_heads) * kSyncStride;
   if (forced_host)
@@ -795,6 +807,29 @@ extern "C" int kie_get_profile(const kie_ctx *ctx, uint64_t *out, int32_t n_word
   if (n_words < need) return KIE_ERR_INVALID;
   cudaError_t e = cudaMemcpy(out, ctx->prof, size_t(need) * 8, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(const_cast<kie_ctx *>(ctx), "profile copy", e);
+  return KIE_OK;
+}
+
+extern "C" int kie_trace_request(kie_ctx *ctx, int32_t cta, int32_t step) {
+  if (!ctx || cta < 0 || cta >= ctx->plan.n_ctas) return KIE_ERR_INVALID;
+  if (!monokernel_profiled()) {
+    g_last_error = "not a profiling build";
+    return KIE_ERR_INVALID;
+  }
+  ctx->trace_cta = cta;
+  ctx->trace_step = step;
+  return KIE_OK;
+}
+
+extern "C" int kie_get_trace(const kie_ctx *ctx, uint64_t *out, int32_t n_words) {
+  if (!ctx || !out || n_words < 1) return KIE_ERR_INVALID;
+  if (!ctx->trace) {
+    g_last_error = "not a profiling build";
+    return KIE_ERR_INVALID;
+  }
+  const int32_t n = std::min<int32_t>(n_words, kTraceCap + 1);
+  cudaError_t e = cudaMemcpy(out, ctx->trace, size_t(n) * 8, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(const_cast<kie_ctx *>(ctx), "trace copy", e);
   return KIE_OK;
 }
 

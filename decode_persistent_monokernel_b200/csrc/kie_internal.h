@@ -52,6 +52,27 @@ enum ProfSlot : int {
 };
 constexpr int kProfSlots = 32;
 
+// Event types of the profiling build's trace (4 bits) -- the argument (4 bits)
+// is a stage kind, a wait kind or a sub-step.
+enum TraceEvent : int {
+  TE_LAYER = 0,        // a layer begins (argument: layer & 15; 15 = LM head)
+  TE_GATE_BEGIN = 1,   // waiting for other SMs (argument: counter kind)
+  TE_GATE_END = 2,
+  TE_SIGNAL_BEGIN = 3, // end-of-stage barrier, then the release
+  TE_SIGNAL_END = 4,
+  TE_NORM_BEGIN = 5,
+  TE_NORM_END = 6,
+  TE_STAGE_BEGIN = 7,  // a weight stage (argument: stage kind)
+  TE_STAGE_END = 8,
+  TE_TILE_WAIT = 9,    // warp 0 starts waiting for a tile
+  TE_TILE_READY = 10,
+  TE_TILE_DONE = 11,   // warp 0 released the tile
+  TE_ATTN = 12,        // attention: 0 begin, 1 positions folded, 2 partials written, 3 merged
+  TE_TILE_LOADED = 13, // warp 0 has the tile's words in registers (row stages)
+  TE_TILE_MATH = 14,   // warp 0 finished the tile's arithmetic
+};
+constexpr int kTraceCap = 1 << 16;
+
 // Per-stage constants shared by every CTA.  A tile is R whole rows (at most
 // kSlotBytes).
 //  Row stages (QKV, GU, MIX, LM): out[row] = sum_k W[row][k] in[k].  All
@@ -152,6 +173,8 @@ struct KernelArgs {
   int32_t skip_signal_cta;      // test hook, -1 = off
   int32_t grid_sync;            // 1: every dependency wait is a grid-wide barrier
   unsigned long long *prof;     // [n_ctas][kProfSlots] (profiling build), or nullptr
+  unsigned long long *trace;    // [1 + trace_cap] event trace (profiling build), or nullptr
+  int32_t trace_cap, trace_cta, trace_step;
 };
 
 }  // namespace kie

@@ -73,20 +73,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// try_wait with a suspend-time hint: the thread sleeps in hardware until the
-// phase completes or about hint_ns pass, instead of spinning on issue slots
-// that the consumer warps of its sub-partition need.
-__device__ __forceinline__ bool mbar_wait_hint(uint64_t *b, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
                                          uint64_t *bar, uint64_t policy) {
   asm volatile(
@@ -169,9 +155,14 @@ __device__ __forceinline__ float2 dot8x2(uint4 w, const float2 (&x)[4], float2 a
 #define KP_BEGIN(var) long long var = (tid == 0) ? clock64() : 0ll
 #define KP_END(var, slot) \
   do { if (tid == 0) s.misc->prof[slot] += clock64() - var; } while (0)
+// Event trace of one SM over one decode step (thread 0's view): 64-bit words
+// (SM clock << 8) | (event type << 4) | argument, into KernelArgs::trace.
+#define KT(type, arg) \
+  do { if (tracing && tid == 0) trace_put((type), (arg)); } while (0)
 #else
 #define KP_BEGIN(var) do {} while (0)
 #define KP_END(var, slot) do {} while (0)
+#define KT(type, arg) do {} while (0)
 #endif
 
 // ------------------------------------------------------------------ shared state
@@ -185,6 +176,7 @@ struct Misc {
   int32_t flag;            // broadcast slot
   long long prof[kProfSlots];
   long long wwait[kConsumerWarps];   // profiling build: tile waits per consumer warp
+  int32_t tn;                        // profiling build: trace events recorded
 };
 
 // Scalars of the column stages: the merged attention output of the CTA's KV
@@ -239,17 +231,15 @@ __device__ bool wait_counter(const KernelArgs &a, const uint32_t *ctr, uint32_t 
 }
 
 // Bounded wait on an mbarrier phase.
-constexpr uint32_t kSuspendHintNs = 20000;
-
 template <typename PumpT>
 __device__ bool wait_mbar(const KernelArgs &a, uint64_t *bar, uint32_t parity, uint32_t code,
                           PumpT &&pump) {
-  if (mbar_wait_hint(bar, parity, kSuspendHintNs)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64(), limit = (long long)a.watchdog_ns * 2;
   long long next_poll = kAbortPollCycles;
   const uint32_t *abortp = sync_at(a, SY_ABORT);
   for (;;) {
-    if (mbar_wait_hint(bar, parity, kSuspendHintNs)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     pump();
     const long long el = clock64() - t0;
     if (el > next_poll) {
@@ -270,8 +260,8 @@ __device__ bool wait_mbar(const KernelArgs &a, uint64_t *bar, uint32_t parity, u
 // full mbarrier, after the slot's empty mbarrier says all 16 consumer warps
 // released its previous tile.  Weights do not depend on activations, so the
 // stream runs ahead across stage, layer and step boundaries while the
-// consumers wait for other SMs.  Its state lives in registers; its waits
-// sleep in hardware (bounded).
+// consumers wait for other SMs.  Its state lives in registers; its waits are
+// bounded.
 struct Producer {
   const KernelArgs &a;
   Smem s;
@@ -358,7 +348,7 @@ struct Producer {
     const uint32_t first = T > NS ? T - NS : 0;
     for (uint32_t t = first; t < T; ++t) {
       const long long t0 = clock64();
-      while (!mbar_wait_hint(&s.full[t % NS], (t / NS) & 1, kSuspendHintNs))
+      while (!mbar_try_wait(&s.full[t % NS], (t / NS) & 1))
         if (clock64() - t0 > (long long)a.watchdog_ns * 2) break;
     }
   }
@@ -376,6 +366,15 @@ struct Consumer {
   uint32_t gl = 0;        // global layer index step * n_layers + l (parity of the buffers)
   uint32_t lm_count = 0;
   uint32_t nsig = 0;      // signals this CTA has made (grid-barrier mode)
+  bool tracing = false;   // profiling build: this SM records the current step
+#ifdef KIE_PROFILE
+  __device__ void trace_put(int type, int arg) {
+    const int n = s.misc->tn;
+    if (n < a.trace_cap) a.trace[1 + n] = (static_cast<unsigned long long>(clock64()) << 8) |
+                                          uint32_t(((type & 15) << 4) | (arg & 15));
+    s.misc->tn = n + 1;
+  }
+#endif
 
   __device__ Consumer(const KernelArgs &a_, Smem s_, int tid_, int cta_)
       : a(a_), s(s_), tid(tid_), warp(tid_ >> 5), lane(tid_ & 31), cta(cta_) {}
@@ -395,7 +394,9 @@ struct Consumer {
         slot = SY_GRID;
         target = nsig * a.n_ctas;
       }
+      KT(TE_GATE_BEGIN, pkind);
       if (!wait_counter(a, sync_at(a, slot), target, where, [] {})) s.misc->abort = 1;
+      KT(TE_GATE_END, pkind);
 #ifdef KIE_PROFILE
       s.misc->prof[PF_GATE] += clock64() - t0;
       s.misc->prof[PF_GATE_K + pkind] += clock64() - t0;
@@ -408,7 +409,9 @@ struct Consumer {
 
   __device__ void signal(int slot) {
     KP_BEGIN(t_sig);
+    KT(TE_SIGNAL_BEGIN, 0);
     cbar();
+    KT(TE_SIGNAL_END, 0);
     ++nsig;
     if (tid == 0) red_release_add(sync_at(a, a.grid_sync ? int(SY_GRID) : slot), 1u);
     KP_END(t_sig, PF_SIGNAL);
@@ -451,6 +454,7 @@ struct Consumer {
   __device__ void stage_norm(Src src, const float *gain, int n, int seg, float *own = nullptr,
                              int own_lo = 0, int own_hi = 0) {
     KP_BEGIN(t_norm);
+    KT(TE_NORM_BEGIN, 0);
     const int ng = n >> 2;
     float4 *vb = reinterpret_cast<float4 *>(s.vbuf);
     float4 *gb = vb + ng;   // the gains, staged beside the input
@@ -488,6 +492,7 @@ struct Consumer {
       }
     }
     cbar();
+    KT(TE_NORM_END, 0);
     KP_END(t_norm, PF_STAGE);
   }
 
@@ -503,6 +508,7 @@ struct Consumer {
   template <bool MULTI>
   __device__ void gemv_impl(int k, const float *vin, bool vin_global) {
     KP_BEGIN(t_gemv);
+    KT(TE_STAGE_BEGIN, k);
     const StageShape sh = a.shape[k];
     const StageCta &c = s.misc->sc[k];
     const int rg = warp / sh.nseg, split = warp - rg * sh.nseg;
@@ -556,7 +562,9 @@ struct Consumer {
 #ifdef KIE_PROFILE
             const long long tw = (lane == 0) ? clock64() : 0ll;
 #endif
+            KT(TE_TILE_WAIT, 0);
             if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [] {});
+            KT(TE_TILE_READY, 0);
 #ifdef KIE_PROFILE
             if (lane == 0) {
               const long long dt = clock64() - tw;
@@ -571,16 +579,19 @@ struct Consumer {
             } else {
               const int rows = min(sh.R, b.nrows - (t0 + bt) * sh.R);
               const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes;
+              uint4 wv[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                wv[i] = crow[i] < rows ? *reinterpret_cast<const uint4 *>(tile + off[i])
+                                       : make_uint4(0u, 0u, 0u, 0u);
+              KT(TE_TILE_LOADED, (wv[0].x ^ wv[1].y ^ wv[2].z ^ wv[3].w) == 0x12345678u);
               float2 d2[4];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                d2[i] = make_float2(0.f, 0.f);
-                if (crow[i] < rows)
-                  d2[i] = dot8x2<T>(*reinterpret_cast<const uint4 *>(tile + off[i]), vr[i], d2[i]);
-              }
+              for (int i = 0; i < 4; ++i) d2[i] = dot8x2<T>(wv[i], vr[i], make_float2(0.f, 0.f));
               if (!MULTI) {
                 const float2 q = __fadd2_rn(__fadd2_rn(d2[0], d2[1]), __fadd2_rn(d2[2], d2[3]));
                 val[bt] += q.x + q.y;
+                KT(TE_TILE_MATH, val[bt] != val[bt]);
               } else {
                 // value index: tile bt of the batch, row crow[i] - row0 of the
                 // warp's rows (uniform across lanes); < 4 because batch * rpw == 4
@@ -595,6 +606,7 @@ struct Consumer {
               }
               __syncwarp();
               if (lane == 0) mbar_arrive(&s.empty[slot]);
+              KT(TE_TILE_DONE, 0);
               if (++slot == uint32_t(a.ring_slots)) { slot = 0; phase ^= 1u; }
             }
           }
@@ -625,6 +637,7 @@ struct Consumer {
     }
     Tbase += c.ntiles;
     cbar();
+    KT(TE_STAGE_END, k);
     KP_END(t_gemv, k == ST_LM ? PF_LM : PF_GEMV);
     KP_END(t_gemv, PF_GEMV_K + k);
   }
@@ -682,7 +695,9 @@ struct Consumer {
 
   __device__ void attention(KvWords &pre) {
     KP_BEGIN(t_attn);
+    KT(TE_ATTN, 0);
     attention_body(pre);
+    KT(TE_ATTN, 3);
     KP_END(t_attn, PF_ATTN);
   }
 
@@ -799,6 +814,7 @@ struct Consumer {
         }
       }
     }
+    KT(TE_ATTN, 1);
     const int st = dh + 2;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -832,6 +848,7 @@ struct Consumer {
     // every split of the group publishes its partial, then each CTA of the
     // group loads all of them into shared memory (one coalesced pass) and
     // merges them (log-sum-exp) into the group's attention output
+    KT(TE_ATTN, 2);
     signal(SY_QG0 + Hkv + g);
     if (!gate(SY_QG0 + Hkv + g, (gl + 1) * uint32_t(ngroup), 0x28, 5)) return;
     float *pb = s.vbuf;   // [G][nsplit][st]
@@ -865,6 +882,7 @@ struct Consumer {
   // in shared memory, then every group is added to acc with one vector atomic.
   __device__ void gemv_cols(int k, const float *svals, float *acc) {
     KP_BEGIN(t_gemv);
+    KT(TE_STAGE_BEGIN, k);
     const StageShape sh = a.shape[k];
     const StageCta &c = s.misc->sc[k];
     const int ngrp = sh.K >> 2;                  // 4-element groups of the output
@@ -884,7 +902,9 @@ struct Consumer {
 #ifdef KIE_PROFILE
         const long long tw = (lane == 0) ? clock64() : 0ll;
 #endif
+        KT(TE_TILE_WAIT, 0);
         if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [] {});
+        KT(TE_TILE_READY, 0);
 #ifdef KIE_PROFILE
         if (lane == 0) {
           const long long dt = clock64() - tw;
@@ -901,21 +921,29 @@ struct Consumer {
         const int rows = min(sh.R, b.nrows - t * sh.R);
         const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes;
         const float *sv = svals + b.lrow0 + t * sh.R;
-        for (int r = ph; r < rows; r += sh.nseg) {
-          const float x = sv[r];
-          const float2 xx = make_float2(x, x);
-          const uint8_t *row = tile + size_t(r) * sh.K * 2;
+        // this thread's rows of the tile are ph, ph + nseg, ... (at most 8:
+        // a tile holds 8 * nseg rows of at least 2048 / nseg outputs)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (j < sh.cps) {
-              const uint2 w = *reinterpret_cast<const uint2 *>(row + size_t(gi + tpr * j) * 8);
-              acc4[j][0] = __ffma2_rn(Store<T>::pair(w.x), xx, acc4[j][0]);
-              acc4[j][1] = __ffma2_rn(Store<T>::pair(w.y), xx, acc4[j][1]);
+        for (int q = 0; q < 8; ++q) {
+          const int r = ph + q * sh.nseg;
+          if (r < rows) {
+            const float x = sv[r];
+            const float2 xx = make_float2(x, x);
+            const uint8_t *row = tile + size_t(r) * sh.K * 2;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (j < sh.cps) {
+                const uint2 w = *reinterpret_cast<const uint2 *>(row + size_t(gi + tpr * j) * 8);
+                acc4[j][0] = __ffma2_rn(Store<T>::pair(w.x), xx, acc4[j][0]);
+                acc4[j][1] = __ffma2_rn(Store<T>::pair(w.y), xx, acc4[j][1]);
+              }
             }
           }
         }
+        KT(TE_TILE_MATH, acc4[0][0].x != acc4[0][0].x);
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.empty[slot]);
+        KT(TE_TILE_DONE, 0);
         if (++slot == uint32_t(a.ring_slots)) { slot = 0; phase ^= 1u; }
       }
       float *dst = acc + b.out_off;
@@ -942,6 +970,7 @@ struct Consumer {
     }
     Tbase += c.ntiles;
     cbar();
+    KT(TE_STAGE_END, k);
     KP_END(t_gemv, PF_GEMV);
     KP_END(t_gemv, PF_GEMV_K + k);
   }
@@ -1008,8 +1037,12 @@ struct Consumer {
         goto done;
       }
       const bool lm = a.logits_every_step || step == a.n_steps - 1;
+#ifdef KIE_PROFILE
+      tracing = a.trace && cta == a.trace_cta && step == a.trace_step;
+#endif
       for (l = 0; l < L; ++l) {
         gl = uint32_t(step) * L + l;
+        KT(TE_LAYER, l & 15);
         const uint32_t cur = gl & 1u, prev = (gl - 1) & 1u;
         // ---------------- RMSNorm + q/k/v rows of the group
         // (every CTA's down contribution to the previous layer is in)
@@ -1084,6 +1117,7 @@ struct Consumer {
         signal(SY_S2);
       }
       if (lm) {
+        KT(TE_LAYER, 15);
         ++lm_count;
         const uint32_t last = gl & 1u;   // parity of the last layer
         if (!gate(SY_S2, (gl + 1) * nc, 0x60, 1)) goto done;
@@ -1158,6 +1192,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
     s.misc->flag = 0;
     for (int i = 0; i < kProfSlots; ++i) s.misc->prof[i] = 0;
     for (int i = 0; i < kConsumerWarps; ++i) s.misc->wwait[i] = 0;
+    s.misc->tn = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -1196,6 +1231,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
   }
   __syncthreads();
   if (a.prof && tid < kProfSlots) a.prof[size_t(cta) * kProfSlots + tid] = s.misc->prof[tid];
+  if (a.trace && cta == a.trace_cta && tid == 0) a.trace[0] = uint32_t(s.misc->tn);
 #endif
 }
 

@@ -169,6 +169,20 @@ int kie_copy_kv(const kie_ctx *ctx, int32_t layer, int32_t kv_head, int32_t pos0
  * n_words must be >= 32 * n_ctas. */
 int kie_get_profile(const kie_ctx *ctx, uint64_t *out, int32_t n_words);
 
+/* Event trace of one SM over one decode step of later launches (profiling
+ * build only; the normal build returns KIE_ERR_INVALID): step = index of the
+ * step inside a launch, -1 to stop tracing.  The SM's thread 0 records
+ * 64-bit events (SM clock << 8) | (type << 4) | argument: 0 layer start
+ * (argument layer & 15, 15 = LM head), 1/2 wait for other SMs begins/ends
+ * (argument: counter kind as in kie_get_profile), 3/4 end-of-stage barrier,
+ * 5/6 RMSNorm staging, 7/8 weight stage (argument: QKV 0, O 1, gate/up 2,
+ * down 3, mix 4, LM 5), 9/10 waiting for a weight tile, 11 tile released,
+ * 12 attention (0 begin, 1 positions folded, 2 partials written, 3 merged).
+ * kie_get_trace copies out[0] = number of events, out[1..] the events;
+ * n_words <= 65537 are copied. */
+int kie_trace_request(kie_ctx *ctx, int32_t cta, int32_t step);
+int kie_get_trace(const kie_ctx *ctx, uint64_t *out, int32_t n_words);
+
 /* Test hooks for the device watchdog (no effect unless called).
  *   watchdog_ms: limit of every in-kernel wait (default 2000, env KIE_WATCHDOG_MS).
  *   skip_signal_cta: if >= 0, that CTA never signals the first stage of the
