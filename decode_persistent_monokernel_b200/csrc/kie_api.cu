@@ -109,24 +109,15 @@ const char *make_shape(int K, int in_len, int out_len, StageShape &s) {
   s.K = K;
   s.in_len = in_len;
   s.out_len = out_len;
-  const int max_rows = kSlotBytes / (2 * K);
-  if (K % 8 || max_rows < 1) return "a weight row must be a multiple of 8 elements and fit one 32 KB slot";
-  const int limit = (K % 256 == 0) ? 64 : 16;
-  int R = 1;
-  while (R * 2 <= std::min(limit, max_rows)) R *= 2;
-  s.R = R;
-  if (R >= kConsumerWarps) {
-    s.nseg = 1;
-    s.rpw = R / kConsumerWarps;
-  } else {
-    int S = kConsumerWarps / R;
-    while (S > 1 && (K / 8) % S) S >>= 1;
-    s.nseg = S;
-    s.rpw = 1;
-  }
-  s.cps = K / 8 / s.nseg;
-  if (s.rpw * s.cps > 128) return "row split leaves more than 4 chunks per lane";
-  if (s.rpw > 1 && s.cps % 32) return "multi-row warps need rows of a multiple of 256 elements";
+  // Each of the 16 consumer warps owns K/16 columns of every row and each
+  // lane 8 of those, so K/128 lanes share a row: one 16-byte load per lane
+  // covers 4096/K rows, and four of them cover R = 16384/K rows, one 32 KB
+  // tile.
+  if (K % 128 || K < 128 || K > 4096) return "row length must be a multiple of 128, at most 4096";
+  s.R = 16384 / K;
+  s.nseg = 1;    // one (shared-memory atomic) sum per row
+  s.rpw = 1;
+  s.cps = 1;
   return nullptr;
 }
 
@@ -409,7 +400,7 @@ static const char *validate(const kie_model_desc *m) {
   if (m->n_heads * m->head_dim != m->d_model) return "n_heads * head_dim must equal d_model";
   if ((m->d_model / nl) % 8 || (m->ffn_dim / nl) % 8) return "lane width and lane ffn must be multiples of 8";
   if ((m->d_model / nl) % 128) return "lane width (d_model / n_lanes) must be a multiple of 128";
-  if (m->d_model > 8192) return "d_model above 8192 is not supported";
+  if (m->d_model > 4096) return "d_model above 4096 is not supported";
   if (nl > 1 && m->lane_delay < 2) return "lane_delay must be >= 2";
   if (nl > 64) return "at most 64 lanes";
   if (!(m->rms_eps >= 0.f) || !(m->rope_theta > 0.f)) return "bad rms_eps or rope_theta";

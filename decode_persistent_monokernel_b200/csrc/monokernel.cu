@@ -107,6 +107,9 @@ __device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t *p, uint32_t v) {
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
 }
+__device__ __forceinline__ void sred_add(float *p, float v) {
+  asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(v) : "memory");
+}
 __device__ __forceinline__ void red_add_v4(float *p, float4 v) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y),
                "f"(v.z), "f"(v.w)
@@ -169,7 +172,7 @@ __device__ __forceinline__ float2 dot8x2(uint4 w, const float2 (&x)[4], float2 a
 struct Misc {
   StageCta sc[ST_COUNT];
   Block blk[kMaxBlocksPerCta];
-  float red_sq[4 * kConsumerWarps];  // per-warp sums of squares while staging
+  __align__(16) float red_sq[4 * kConsumerWarps];  // per-warp sums of squares while staging
   float red_v[kConsumerWarps];
   int32_t red_i[kConsumerWarps];
   volatile int32_t abort;  // a consumer saw a failed wait
@@ -177,6 +180,8 @@ struct Misc {
   long long prof[kProfSlots];
   long long wwait[kConsumerWarps];   // profiling build: tile waits per consumer warp
   int32_t tn;                        // profiling build: trace events recorded
+  float fac[4 * 32];   // attention: per-head scale factors of warps or splits
+  float hs[8];         // attention: per-head running maximum and sum
 };
 
 // Scalars of the column stages: the merged attention output of the CTA's KV
@@ -480,11 +485,20 @@ struct Consumer {
     for (int q = 0; q * kNC < ng; ++q) {
       const int j = tid + q * kNC;
       if (j < ng) {
-        // the slice holding element 4j covers warps' 128-element ranges
-        // e = e0, e0 + 128, ...; range e was summed into red_sq[e / 2048 * 16 + e % 2048 / 128]
+        // the slice holding element 4j covers the warps' 128-element ranges
+        // e0 / 128 .. (e0 + seg) / 128 - 1 of red_sq, which are contiguous
         const int e0 = (4 * j) / seg * seg;
+        const int i0 = e0 >> 7, n = seg >> 7;
         float tot = 0.f;
-        for (int e = e0; e < e0 + seg; e += 128) tot += s.misc->red_sq[(e >> 11) * kConsumerWarps + ((e >> 7) & 15)];
+        if ((n & 3) == 0) {
+          const float4 *rq = reinterpret_cast<const float4 *>(s.misc->red_sq + i0);
+          for (int i = 0; i < (n >> 2); ++i) {
+            const float4 r4 = rq[i];
+            tot += (r4.x + r4.y) + (r4.z + r4.w);
+          }
+        } else {
+          for (int i = 0; i < n; ++i) tot += s.misc->red_sq[i0 + i];
+        }
         const float r = rsqrtf(tot / float(seg) + a.rms_eps);
         const float4 g = gb[j];
         const float4 v = vb[j];
@@ -496,145 +510,144 @@ struct Consumer {
     KP_END(t_norm, PF_STAGE);
   }
 
-  // ---- GEMV over the stage's tiles: partial sums into s.part
-  // Every consumer warp waits on every tile in order and handles its row group
-  // and column split; its slice of the input vector stays in registers for
-  // the whole block.  `vin` is the stage input (shared or global memory).
-  __device__ void gemv(int k, const float *vin, bool vin_global) {
-    if (a.shape[k].rpw > 1) gemv_impl<true>(k, vin, vin_global);
-    else gemv_impl<false>(k, vin, vin_global);
+  // ---- row stages: part[row] = W[row, :] . vin over the stage's tiles
+  // Warp w owns columns [w*K/16, (w+1)*K/16) of every row; lane l covers the
+  // 8 columns col0 = w*K/16 + (l % lpr)*8 (lpr = K/128 lanes per row) of rows
+  // l / lpr + q * (32 / lpr), q = 0..3, of each tile: one 16-byte shared load
+  // per q, 8 fp32 inputs in registers.  The tile after the current one is
+  // waited for and loaded before the current one's arithmetic (one-tile
+  // software pipeline, across block boundaries too); a tile's slot is
+  // released once its words have been used.  Each row's partial sums are
+  // reduced across its lpr lanes (transposed butterfly) and added into
+  // part[row] with shared-memory atomics: part must be zero on entry
+  // (rowsum_clear leaves it so).
+  struct Words4 {
+    uint4 q[4];
+  };
+  struct Inputs8 {
+    float2 v[4];
+  };
+
+  // Waits (warp-wide outcome) for the weight tile in the current ring slot.
+  __device__ bool tile_wait(int k) {
+    bool got = true;
+    KT(TE_TILE_WAIT, 0);
+    if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [] {});
+    KT(TE_TILE_READY, 0);
+    return __shfl_sync(0xffffffffu, got, 0);
+  }
+  __device__ void slot_advance() {
+    if (++slot == uint32_t(a.ring_slots)) { slot = 0; phase ^= 1u; }
+  }
+  // This lane's four 16-byte chunks of the tile in the current slot (rows
+  // lrow + q * rpl; zero beyond the tile's `rows`).
+  __device__ Words4 row_words(uint32_t off0, int lrow, int rpl, int rows) const {
+    Words4 w;
+    const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes + off0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      w.q[q] = (lrow + q * rpl < rows) ? *reinterpret_cast<const uint4 *>(tile + q * 8192)
+                                       : make_uint4(0u, 0u, 0u, 0u);
+    return w;
+  }
+  __device__ Inputs8 row_inputs(const float *vin, int in_off, int col0) const {
+    const float4 *src = reinterpret_cast<const float4 *>(vin + in_off + col0);
+    const float4 x0 = src[0], x1 = src[1];
+    Inputs8 x;
+    x.v[0] = make_float2(x0.x, x0.y); x.v[1] = make_float2(x0.z, x0.w);
+    x.v[2] = make_float2(x1.x, x1.y); x.v[3] = make_float2(x1.z, x1.w);
+    return x;
+  }
+  // The tile after (bi, t) of the stage's blocks, skipping empty blocks.
+  __device__ void next_tile(int b0, int nblk, int R, int &bi, int &t) const {
+    ++t;
+    if (t * R >= s.misc->blk[b0 + bi].nrows) { ++bi; t = 0; }
+    while (bi < nblk && s.misc->blk[b0 + bi].nrows == 0) ++bi;
   }
 
-  template <bool MULTI>
-  __device__ void gemv_impl(int k, const float *vin, bool vin_global) {
+  __device__ void gemv(int k, const float *vin) {
     KP_BEGIN(t_gemv);
     KT(TE_STAGE_BEGIN, k);
-    const StageShape sh = a.shape[k];
     const StageCta &c = s.misc->sc[k];
-    const int rg = warp / sh.nseg, split = warp - rg * sh.nseg;
-    const int row0 = rg * sh.rpw;               // first row of this warp inside a tile
-    const bool active = row0 < sh.R;
-    const int nchunk = sh.rpw * sh.cps;         // chunks this warp covers per tile (<= 128)
-    // Per-lane chunk layout, the same for every tile of the stage: byte offset
-    // inside the tile, row inside the tile (INT_MAX if unused), input column.
-    uint32_t off[4];
-    int crow[4], ccol[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int ci = lane + 32 * i;
-      const int rr = ci / sh.cps, cc = ci - rr * sh.cps;
-      const bool valid = active && ci < nchunk;
-      crow[i] = valid ? row0 + rr : 0x7fffffff;
-      ccol[i] = (split * sh.cps + cc) * 8;
-      off[i] = uint32_t((row0 + rr) * sh.K + ccol[i]) * 2u;
-    }
+    const int K = a.shape[k].K, R = a.shape[k].R;
+    const int lsh = __ffs(K >> 7) - 1;          // log2(lanes per row)
+    const int lpr = 1 << lsh;
+    const int lrow = lane >> lsh;               // this lane's row within a load
+    const int rpl = 32 >> lsh;                  // rows per load
+    const int col0 = warp * (K >> 4) + ((lane & (lpr - 1)) << 3);
+    const uint32_t off0 = uint32_t(lrow * K + col0) * 2u;   // + q * 8192 bytes
+    const int nblk = c.nblk, b0 = c.blk_begin;
     bool ok = !aborted();
-    for (int bi = 0; bi < c.nblk && ok; ++bi) {
-      const Block b = s.misc->blk[c.blk_begin + bi];
-      // this warp's slice of the input vector, kept in registers for the block
-      float2 vr[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (crow[i] != 0x7fffffff) {
-          const float *src = vin + b.in_off + ccol[i];
-          float4 x0, x1;
-          if (vin_global) { x0 = __ldcg(reinterpret_cast<const float4 *>(src)); x1 = __ldcg(reinterpret_cast<const float4 *>(src) + 1); }
-          else { x0 = reinterpret_cast<const float4 *>(src)[0]; x1 = reinterpret_cast<const float4 *>(src)[1]; }
-          vr[i][0] = make_float2(x0.x, x0.y); vr[i][1] = make_float2(x0.z, x0.w);
-          vr[i][2] = make_float2(x1.x, x1.y); vr[i][3] = make_float2(x1.z, x1.w);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) vr[i][e] = make_float2(0.f, 0.f);
-        }
-      }
-      // Tiles go in batches of `batch` (4 / rpw) tiles: each tile's dot
-      // products are folded into one value per (tile, row) and its slot is
-      // released at once; the batch's 4 values are then reduced across the
-      // warp together (transposed butterfly: 6 shuffles for 4 values).
-      const int ntile = (b.nrows + sh.R - 1) / sh.R;
-      const int batch = MULTI ? 4 / sh.rpw : 4;
-      for (int t0 = 0; t0 < ntile && ok; t0 += batch) {
-        float val[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int bt = 0; bt < 4; ++bt) {
-          if (bt < batch && t0 + bt < ntile) {
-            bool got = true;
-#ifdef KIE_PROFILE
-            const long long tw = (lane == 0) ? clock64() : 0ll;
-#endif
-            KT(TE_TILE_WAIT, 0);
-            if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [] {});
-            KT(TE_TILE_READY, 0);
-#ifdef KIE_PROFILE
-            if (lane == 0) {
-              const long long dt = clock64() - tw;
-              if (tid == 0) s.misc->prof[PF_FULLWAIT] += dt;
-              s.misc->wwait[warp] += dt;
-            }
-#endif
-            got = __shfl_sync(0xffffffffu, got, 0);
-            if (!got) {
-              s.misc->abort = 1;
-              ok = false;
-            } else {
-              const int rows = min(sh.R, b.nrows - (t0 + bt) * sh.R);
-              const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes;
-              uint4 wv[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                wv[i] = crow[i] < rows ? *reinterpret_cast<const uint4 *>(tile + off[i])
-                                       : make_uint4(0u, 0u, 0u, 0u);
-              KT(TE_TILE_LOADED, (wv[0].x ^ wv[1].y ^ wv[2].z ^ wv[3].w) == 0x12345678u);
-              float2 d2[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) d2[i] = dot8x2<T>(wv[i], vr[i], make_float2(0.f, 0.f));
-              if (!MULTI) {
-                const float2 q = __fadd2_rn(__fadd2_rn(d2[0], d2[1]), __fadd2_rn(d2[2], d2[3]));
-                val[bt] += q.x + q.y;
-                KT(TE_TILE_MATH, val[bt] != val[bt]);
-              } else {
-                // value index: tile bt of the batch, row crow[i] - row0 of the
-                // warp's rows (uniform across lanes); < 4 because batch * rpw == 4
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const int vidx = bt * sh.rpw + (crow[i] - row0);
-                  const float d = d2[i].x + d2[i].y;
-#pragma unroll
-                  for (int j = 0; j < 4; ++j)
-                    if (crow[i] < rows && j == vidx) val[j] += d;
-                }
-              }
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&s.empty[slot]);
-              KT(TE_TILE_DONE, 0);
-              if (++slot == uint32_t(a.ring_slots)) { slot = 0; phase ^= 1u; }
-            }
-          }
-        }
-        if (!ok) break;
-        // transposed butterfly: after it, lane l holds the warp sum of value (l >> 3) & 3
-        const bool b4 = lane & 16, b3 = lane & 8;
-        const float r0 = __shfl_xor_sync(0xffffffffu, b4 ? val[0] : val[2], 16);
-        const float r1 = __shfl_xor_sync(0xffffffffu, b4 ? val[1] : val[3], 16);
-        const float k0 = (b4 ? val[2] : val[0]) + r0;
-        const float k1 = (b4 ? val[3] : val[1]) + r1;
-        const float r2 = __shfl_xor_sync(0xffffffffu, b3 ? k0 : k1, 8);
-        float v = (b3 ? k1 : k0) + r2;
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        if (active && (lane & 7) == 0) {
-          const int vi = lane >> 3;                        // value index 0..3
-          const int bt = MULTI ? vi / sh.rpw : vi;          // tile within the batch
-          const int r = MULTI ? vi - bt * sh.rpw : 0;       // row within the warp's rows
-          const int t = t0 + bt;
-          if (t < ntile && r < sh.rpw) {
-            const int rows = min(sh.R, b.nrows - t * sh.R);
-            if (row0 + r < rows) s.part[(b.lrow0 + t * sh.R + row0 + r) * sh.nseg + split] = v;
-          }
-        }
-      }
+    int bi = 0, t = 0;
+    while (bi < nblk && s.misc->blk[b0 + bi].nrows == 0) ++bi;
+    Words4 w{}, wn{};
+    Inputs8 x{};
+    int rows = 0;
+    if (bi < nblk && ok) {
+      x = row_inputs(vin, s.misc->blk[b0 + bi].in_off, col0);
+      rows = min(R, s.misc->blk[b0 + bi].nrows);
+      ok = tile_wait(k);
+      if (ok) w = row_words(off0, lrow, rpl, rows);
+      slot_advance();
     }
+    while (ok && bi < nblk) {
+      const uint32_t held = slot == 0 ? uint32_t(a.ring_slots) - 1 : slot - 1;
+      int nbi = bi, nt = t;
+      next_tile(b0, nblk, R, nbi, nt);
+      const bool more = nbi < nblk;
+      int nrows = 0;
+      if (more) {
+        nrows = min(R, s.misc->blk[b0 + nbi].nrows - nt * R);
+        ok = tile_wait(k);
+        if (ok) wn = row_words(off0, lrow, rpl, nrows);
+        slot_advance();
+      }
+      // arithmetic of the current tile: four 8-term dot products
+      float p[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 d = dot8x2<T>(w.q[q], x.v, make_float2(0.f, 0.f));
+        p[q] = d.x + d.y;
+      }
+      KT(TE_TILE_MATH, p[0] != p[0]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.empty[held]);
+      KT(TE_TILE_DONE, 0);
+      // reduce each row over its lpr lanes, then one shared atomic per row
+      float *prow = s.part + s.misc->blk[b0 + bi].lrow0 + t * R + lrow;   // + value * rpl
+      if (lsh == 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (lrow + q * rpl < rows) sred_add(prow + q * rpl, p[q]);
+      } else {
+        const int h = lpr >> 1;
+        const bool hi = lane & h;
+        const float s0 = __shfl_xor_sync(0xffffffffu, hi ? p[0] : p[2], h);
+        const float s1 = __shfl_xor_sync(0xffffffffu, hi ? p[1] : p[3], h);
+        const float a0 = (hi ? p[2] : p[0]) + s0;   // value 2 if hi else 0
+        const float a1 = (hi ? p[3] : p[1]) + s1;   // value 3 if hi else 1
+        const int v0 = hi ? 2 : 0;
+        if (lsh == 1) {
+          if (lrow + v0 * rpl < rows) sred_add(prow + v0 * rpl, a0);
+          if (lrow + (v0 + 1) * rpl < rows) sred_add(prow + (v0 + 1) * rpl, a1);
+        } else {
+          const int h2 = lpr >> 2;
+          const bool hi2 = lane & h2;
+          const float s2 = __shfl_xor_sync(0xffffffffu, hi2 ? a0 : a1, h2);
+          float v = (hi2 ? a1 : a0) + s2;          // value v0 + hi2
+          for (int o = lpr >> 3; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          const int vi = v0 + (hi2 ? 1 : 0);
+          if ((lane & (h2 - 1)) == 0 && lrow + vi * rpl < rows) sred_add(prow + vi * rpl, v);
+        }
+      }
+      if (!ok || !more) break;
+      if (nbi != bi) x = row_inputs(vin, s.misc->blk[b0 + nbi].in_off, col0);
+      w = wn;
+      bi = nbi;
+      t = nt;
+      rows = nrows;
+    }
+    if (!ok) s.misc->abort = 1;
     Tbase += c.ntiles;
     cbar();
     KT(TE_STAGE_END, k);
@@ -642,9 +655,11 @@ struct Consumer {
     KP_END(t_gemv, PF_GEMV_K + k);
   }
 
-  __device__ float rowsum(int i, int nseg) const {
-    float v = 0.f;
-    for (int sg = 0; sg < nseg; ++sg) v += s.part[i * nseg + sg];
+  // Sum of row i of the last row stage (its shared-memory accumulator), which
+  // is cleared for the next stage.  Each row is read by exactly one thread.
+  __device__ float rowsum(int i) const {
+    const float v = s.part[i];
+    s.part[i] = 0.f;
     return v;
   }
 
@@ -686,28 +701,25 @@ struct Consumer {
       }
     }
   }
-  // Issued before the q/k/v gate: the cache rows do not depend on this step.
-  __device__ void attention_prefetch(KvWords &w) const {
-    int j0, j1, split, nsplit;
-    kv_range(j0, j1, split, nsplit);
-    kv_load(w, j0 + warp, j1);
-  }
-
-  __device__ void attention(KvWords &pre) {
+  __device__ void attention() {
     KP_BEGIN(t_attn);
     KT(TE_ATTN, 0);
-    attention_body(pre);
+    attention_body();
     KT(TE_ATTN, 3);
     KP_END(t_attn, PF_ATTN);
   }
 
-  __device__ void attention_body(KvWords &kw) {
+  __device__ void attention_body() {
     const int dh = a.head_dim, half = dh >> 1;
     const int Hkv = a.n_kv_heads, G = a.n_heads / a.n_kv_heads;
     const int g = cta % Hkv;
     const int ngroup = (a.n_ctas - 1 - g) / Hkv + 1;      // CTAs of this KV group
     int j0, j1, split, nsplit;
     kv_range(j0, j1, split, nsplit);
+    // the first cached rows (already pulled into L2 by the producer) are
+    // requested together with this step's q/k/v
+    KvWords kw;
+    kv_load(kw, j0 + warp, j1);
     const bool active = split < nsplit;
     const bool writer = (split == nsplit - 1);  // its range holds position p
     float *qs = s.vbuf;              // [G][dh] roped, scaled queries
@@ -743,8 +755,7 @@ struct Consumer {
     cbar();
     // Online softmax, kU positions per iteration: their score reductions are
     // independent and one rescale covers them.  The next iteration's rows are
-    // requested before this one's arithmetic (the first ones were requested
-    // before the q/k/v gate).
+    // requested before this one's arithmetic.
     const int dpl = dh >> 5;  // dims per lane: 4 (dh 128) or 2 (dh 64)
     float m[4], lsum[4], o[4][4];
 #pragma unroll
@@ -827,23 +838,30 @@ struct Consumer {
       }
     }
     cbar();
-    // combine the warps into this CTA's partial for each query head
+    // combine the warps into this CTA's partial for each query head: warp i
+    // finds head i's running maximum over the 16 warps and each warp's scale
+    // factor once; then every output element is a 16-term weighted sum
+    float *fac = s.misc->fac, *hs = s.misc->hs;
+    if (warp < G) {
+      const int i = warp;
+      const float mw = lane < kConsumerWarps ? wst[(size_t(lane) * G + i) * st + dh] : -INFINITY;
+      float M = mw;
+      for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float f = mw == -INFINITY ? 0.f : expf(mw - M);
+      float L = lane < kConsumerWarps ? f * wst[(size_t(lane) * G + i) * st + dh + 1] : 0.f;
+      for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+      fac[i * 32 + lane] = f;
+      if (lane == 0) { hs[2 * i] = M; hs[2 * i + 1] = L; }
+    }
+    cbar();
     for (int idx = tid; idx < (active ? G * dh : 0); idx += kNC) {
       const int i = idx / dh, d = idx - i * dh;
-      float M = -INFINITY;
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, wst[(size_t(w) * G + i) * st + dh]);
-      float Ls = 0.f, O = 0.f;
-      if (M != -INFINITY) {
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float *ws = wst + (size_t(w) * G + i) * st;
-          const float f = expf(ws[dh] - M);
-          Ls += ws[dh + 1] * f;
-          O += ws[d] * f;
-        }
-      }
+      float O = 0.f;
+#pragma unroll 4
+      for (int w = 0; w < kConsumerWarps; ++w) O = fmaf(fac[i * 32 + w], wst[(size_t(w) * G + i) * st + d], O);
       float *dst = a.attn_part + (size_t(g * G + i) * a.max_split + split) * st;
       dst[d] = O;
-      if (d == 0) { dst[dh] = M; dst[dh + 1] = Ls; }
+      if (d == 0) { dst[dh] = hs[2 * i]; dst[dh + 1] = hs[2 * i + 1]; }
     }
     // every split of the group publishes its partial, then each CTA of the
     // group loads all of them into shared memory (one coalesced pass) and
@@ -857,20 +875,30 @@ struct Consumer {
       for (int q = tid; q < nsplit * st; q += kNC) pb[(size_t(i) * nsplit) * st + q] = __ldcg(src + q);
     }
     cbar();
+    // log-sum-exp merge of the splits: warp i computes head i's weights
+    // exp(m_s - M) / sum_s l_s exp(m_s - M) once (lane = split), then every
+    // output element is an nsplit-term weighted sum.  The split holding
+    // position p is never empty, so the denominator is positive.
+    if (warp < G) {
+      const int i = warp;
+      const float *src = pb + size_t(i) * nsplit * st;
+      const float ms = lane < nsplit ? src[size_t(lane) * st + dh] : -INFINITY;
+      float M = ms;
+      for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float f = ms == -INFINITY ? 0.f : expf(ms - M);
+      float L = lane < nsplit ? f * src[size_t(lane) * st + dh + 1] : 0.f;
+      for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+      fac[i * 32 + lane] = f / L;
+    }
+    cbar();
     float *og = s.svec;   // [G * dh] merged attention output of the group
     for (int idx = tid; idx < G * dh; idx += kNC) {
       const int i = idx / dh, d = idx - i * dh;
       const float *src = pb + size_t(i) * nsplit * st;
-      float M = -INFINITY;
-      for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, src[size_t(sp) * st + dh]);
-      float Ls = 0.f, O = 0.f;
-      for (int sp = 0; sp < nsplit; ++sp) {
-        const float *ps = src + size_t(sp) * st;
-        const float f = expf(ps[dh] - M);
-        Ls += ps[dh + 1] * f;
-        O += ps[d] * f;
-      }
-      og[idx] = O / Ls;
+      float O = 0.f;
+#pragma unroll 4
+      for (int sp = 0; sp < nsplit; ++sp) O = fmaf(fac[i * 32 + sp], src[size_t(sp) * st + d], O);
+      og[idx] = O;
     }
     cbar();
   }
@@ -878,9 +906,41 @@ struct Consumer {
   // ---- column stages (O, down): out[:] += sum_i svals[i] * W_i[:]
   // W_i are the stage's streamed rows (columns of the canonical matrix), svals
   // the matching scalars in shared memory (index = local row).  Each thread
-  // accumulates 4-element output groups over its row phase; phases are summed
-  // in shared memory, then every group is added to acc with one vector atomic.
+  // owns CPS 4-element output groups and a phase of the tile's rows: rows
+  // ph, ph + nseg, ... (8 / CPS of them: a tile holds 8 * nseg / CPS rows).
+  // Its words and row scalars of the next tile are loaded before the current
+  // tile's arithmetic (one-tile software pipeline across blocks).  At the end
+  // of a block, phases are summed in shared memory (nseg > 1) and every group
+  // is added to the fp32 accumulator with one vector atomic.
+  template <int CPS>
+  struct ColWords {
+    uint2 w[8 / CPS][CPS];
+  };
+
+  template <int CPS>
+  __device__ ColWords<CPS> col_words(const StageShape &sh, int ph, int gi, int tpr, int rows) const {
+    ColWords<CPS> cw;
+    const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes;
+#pragma unroll
+    for (int q = 0; q < 8 / CPS; ++q) {
+      const int r = ph + q * sh.nseg;
+      const bool in = r < rows;
+      const uint8_t *row = tile + size_t(r) * sh.K * 2;
+#pragma unroll
+      for (int j = 0; j < CPS; ++j)
+        cw.w[q][j] = in ? *reinterpret_cast<const uint2 *>(row + size_t(gi + tpr * j) * 8)
+                        : make_uint2(0u, 0u);
+    }
+    return cw;
+  }
+
   __device__ void gemv_cols(int k, const float *svals, float *acc) {
+    if (a.shape[k].cps == 1) gemv_cols_impl<1>(k, svals, acc);
+    else gemv_cols_impl<2>(k, svals, acc);
+  }
+
+  template <int CPS>
+  __device__ void gemv_cols_impl(int k, const float *svals, float *acc) {
     KP_BEGIN(t_gemv);
     KT(TE_STAGE_BEGIN, k);
     const StageShape sh = a.shape[k];
@@ -888,86 +948,84 @@ struct Consumer {
     const int ngrp = sh.K >> 2;                  // 4-element groups of the output
     const int tpr = sh.nseg > 1 ? ngrp : kNC;    // threads per row phase
     const int ph = tid / tpr, gi = tid - ph * tpr;
+    const int nblk = c.nblk, b0 = c.blk_begin, R = sh.R;
     // A failed wait stops this warp's tile work, but every warp still goes
     // through the same barriers so that none is left waiting.
     bool ok = !aborted();
-    for (int bi = 0; bi < c.nblk; ++bi) {
-      const Block b = s.misc->blk[c.blk_begin + bi];
-      float2 acc4[4][2];   // output group j: elements (0,1) and (2,3)
+    int bi = 0, t = 0;
+    while (bi < nblk && s.misc->blk[b0 + bi].nrows == 0) ++bi;
+    ColWords<CPS> cw{}, cn{};
+    float2 acc2[CPS][2];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc4[j][0] = acc4[j][1] = make_float2(0.f, 0.f);
-      const int ntile = (b.nrows + sh.R - 1) / sh.R;
-      for (int t = 0; t < ntile && ok; ++t) {
-        bool got = true;
-#ifdef KIE_PROFILE
-        const long long tw = (lane == 0) ? clock64() : 0ll;
-#endif
-        KT(TE_TILE_WAIT, 0);
-        if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [] {});
-        KT(TE_TILE_READY, 0);
-#ifdef KIE_PROFILE
-        if (lane == 0) {
-          const long long dt = clock64() - tw;
-          if (tid == 0) s.misc->prof[PF_FULLWAIT] += dt;
-          s.misc->wwait[warp] += dt;
-        }
-#endif
-        got = __shfl_sync(0xffffffffu, got, 0);
-        if (!got) {
-          s.misc->abort = 1;
-          ok = false;
-          break;
-        }
-        const int rows = min(sh.R, b.nrows - t * sh.R);
-        const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes;
-        const float *sv = svals + b.lrow0 + t * sh.R;
-        // this thread's rows of the tile are ph, ph + nseg, ... (at most 8:
-        // a tile holds 8 * nseg rows of at least 2048 / nseg outputs)
+    for (int j = 0; j < CPS; ++j) acc2[j][0] = acc2[j][1] = make_float2(0.f, 0.f);
+    int rows = 0;
+    if (bi < nblk) {
+      rows = min(R, s.misc->blk[b0 + bi].nrows);
+      if (ok) ok = tile_wait(k);
+      if (ok) cw = col_words<CPS>(sh, ph, gi, tpr, rows);
+      slot_advance();
+    }
+    while (bi < nblk) {
+      const uint32_t held = slot == 0 ? uint32_t(a.ring_slots) - 1 : slot - 1;
+      int nbi = bi, nt = t, nrows = 0;
+      next_tile(b0, nblk, R, nbi, nt);
+      const bool more = nbi < nblk;
+      if (more) {
+        nrows = min(R, s.misc->blk[b0 + nbi].nrows - nt * R);
+        if (ok) ok = tile_wait(k);
+        if (ok) cn = col_words<CPS>(sh, ph, gi, tpr, nrows);
+        slot_advance();
+      }
+      if (ok) {
+        const float *sv = svals + s.misc->blk[b0 + bi].lrow0 + t * R;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < 8 / CPS; ++q) {
           const int r = ph + q * sh.nseg;
-          if (r < rows) {
-            const float x = sv[r];
-            const float2 xx = make_float2(x, x);
-            const uint8_t *row = tile + size_t(r) * sh.K * 2;
+          const float xv = r < rows ? sv[r] : 0.f;
+          const float2 xx = make_float2(xv, xv);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              if (j < sh.cps) {
-                const uint2 w = *reinterpret_cast<const uint2 *>(row + size_t(gi + tpr * j) * 8);
-                acc4[j][0] = __ffma2_rn(Store<T>::pair(w.x), xx, acc4[j][0]);
-                acc4[j][1] = __ffma2_rn(Store<T>::pair(w.y), xx, acc4[j][1]);
-              }
-            }
+          for (int j = 0; j < CPS; ++j) {
+            acc2[j][0] = __ffma2_rn(Store<T>::pair(cw.w[q][j].x), xx, acc2[j][0]);
+            acc2[j][1] = __ffma2_rn(Store<T>::pair(cw.w[q][j].y), xx, acc2[j][1]);
           }
         }
-        KT(TE_TILE_MATH, acc4[0][0].x != acc4[0][0].x);
+        KT(TE_TILE_MATH, acc2[0][0].x != acc2[0][0].x);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s.empty[slot]);
+        if (lane == 0) mbar_arrive(&s.empty[held]);
         KT(TE_TILE_DONE, 0);
-        if (++slot == uint32_t(a.ring_slots)) { slot = 0; phase ^= 1u; }
       }
-      float *dst = acc + b.out_off;
-      if (sh.nseg == 1) {
-        if (ok) {
+      if (nbi != bi) {
+        // the block is complete: add its groups into the accumulator
+        float *dst = acc + s.misc->blk[b0 + bi].out_off;
+        if (sh.nseg == 1) {
+          if (ok) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (j < sh.cps)
+            for (int j = 0; j < CPS; ++j)
               red_add_v4(dst + 4 * (gi + tpr * j),
-                         make_float4(acc4[j][0].x, acc4[j][0].y, acc4[j][1].x, acc4[j][1].y));
+                         make_float4(acc2[j][0].x, acc2[j][0].y, acc2[j][1].x, acc2[j][1].y));
+          }
+        } else {
+          // several row phases: add them up in shared memory first (CPS == 1)
+          float4 *scr = reinterpret_cast<float4 *>(s.vbuf);
+          scr[ph * ngrp + gi] = make_float4(acc2[0][0].x, acc2[0][0].y, acc2[0][1].x, acc2[0][1].y);
+          cbar();
+          if (tid < ngrp && !aborted()) {
+            float4 v = scr[tid];
+            for (int q = 1; q < sh.nseg; ++q) v = add4(v, scr[q * ngrp + tid]);
+            red_add_v4(dst + 4 * tid, v);
+          }
+          cbar();
         }
-      } else {
-        // several row phases: add them up in shared memory first (cps == 1)
-        float4 *scr = reinterpret_cast<float4 *>(s.vbuf);
-        scr[ph * ngrp + gi] = make_float4(acc4[0][0].x, acc4[0][0].y, acc4[0][1].x, acc4[0][1].y);
-        cbar();
-        if (tid < ngrp && !aborted()) {
-          float4 v = scr[tid];
-          for (int q = 1; q < sh.nseg; ++q) v = add4(v, scr[q * ngrp + tid]);
-          red_add_v4(dst + 4 * tid, v);
-        }
-        cbar();
+#pragma unroll
+        for (int j = 0; j < CPS; ++j) acc2[j][0] = acc2[j][1] = make_float2(0.f, 0.f);
       }
+      if (!more) break;
+      cw = cn;
+      bi = nbi;
+      t = nt;
+      rows = nrows;
     }
+    if (!ok) s.misc->abort = 1;
     Tbase += c.ntiles;
     cbar();
     KT(TE_STAGE_END, k);
@@ -978,13 +1036,12 @@ struct Consumer {
   // ---- LM head epilogue: logits and the CTA's share of the argmax
   __device__ void lm_epilogue() {
     const StageCta &c = s.misc->sc[ST_LM];
-    const int nseg = a.shape[ST_LM].nseg;
     // bidx starts at a row of this CTA so that the key always names a valid
     // token; a NaN logit never wins a comparison and raises DE_NONFINITE.
     float best = -INFINITY;
     int bidx = c.row0;
     for (int i = tid; i < c.nout; i += kNC) {
-      const float v = rowsum(i, nseg);
+      const float v = rowsum(i);
       const int row = c.row0 + i;
       if (a.logits_out) a.logits_out[size_t(step) * a.vocab + row] = v;
       if (v != v) raise_error(a, DE_NONFINITE | (uint32_t(step & 0xffff) << 8));
@@ -1049,14 +1106,13 @@ struct Consumer {
         if (gl > 0 && !gate(SY_S2, gl * nc, 0x10, 1)) goto done;
         stage_norm([=](int j) { return xin4(j); }, a.gain_attn + size_t(l) * d, d, a.lane_width,
                    a.xres + size_t(cur) * d, own_lo, own_hi);
-        gemv(ST_QKV, s.vbuf, false);
+        gemv(ST_QKV, s.vbuf);
         if (aborted()) goto done;
         {
           const StageCta &c = s.misc->sc[ST_QKV];
-          const int nseg = a.shape[ST_QKV].nseg;
           for (int bi = 0; bi < c.nblk; ++bi) {
             const Block b = s.misc->blk[c.blk_begin + bi];
-            for (int i = tid; i < b.nrows; i += kNC) a.qkv[b.out_off + i] = rowsum(b.lrow0 + i, nseg);
+            for (int i = tid; i < b.nrows; i += kNC) a.qkv[b.out_off + i] = rowsum(b.lrow0 + i);
           }
         }
         if (!(a.skip_signal_cta == cta && step == 0 && l == 0)) signal(SY_QG0 + g);
@@ -1066,20 +1122,15 @@ struct Consumer {
           for (int j = tid; j < (d >> 2); j += kNC)
             reinterpret_cast<float4 *>(s.vbuf)[j] = add4(__ldcg(uo + j), __ldcg(ud + j));
           cbar();
-          gemv(ST_MIX, s.vbuf, false);
+          gemv(ST_MIX, s.vbuf);
           if (aborted()) goto done;
           const StageCta &c = s.misc->sc[ST_MIX];
-          const int nseg = a.shape[ST_MIX].nseg;
           float *dst = a.dsum + size_t((l - 1) % delta) * d;
-          for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(i, nseg);
+          for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(i);
         }
         // ---------------- attention of the group, merged in every group CTA
-        {
-          KvWords kw;
-          attention_prefetch(kw);
-          if (!gate(SY_QG0 + g, (gl + 1) * ng, 0x20, 4)) goto done;
-          attention(kw);
-        }
+        if (!gate(SY_QG0 + g, (gl + 1) * ng, 0x20, 4)) goto done;
+        attention();
         if (aborted()) goto done;
         // ---------------- O projection over the group's attention outputs
         gemv_cols(ST_O, s.svec + s.misc->sc[ST_O].row0, a.acc_o + size_t(cur) * d);
@@ -1099,14 +1150,13 @@ struct Consumer {
           stage_norm([=](int j) { return add4(__ldcg(xr + j), __ldcg(ao + j)); },
                      a.gain_ffn + size_t(l) * d, d, a.lane_width);
         }
-        gemv(ST_GU, s.vbuf, false);
+        gemv(ST_GU, s.vbuf);
         if (aborted()) goto done;
         {
           const StageCta &c = s.misc->sc[ST_GU];
-          const int nseg = a.shape[ST_GU].nseg;
           float *h = s.svec + kSvecO;
           for (int i = tid; i < c.nout; i += kNC) {
-            const float gt = rowsum(i, nseg), up = rowsum(c.nout + i, nseg);
+            const float gt = rowsum(i), up = rowsum(c.nout + i);
             h[i] = gt / (1.f + expf(-gt)) * up;
           }
           cbar();
@@ -1127,12 +1177,11 @@ struct Consumer {
           for (int j = tid; j < (d >> 2); j += kNC)
             reinterpret_cast<float4 *>(s.vbuf)[j] = add4(__ldcg(uo + j), __ldcg(ud + j));
           cbar();
-          gemv(ST_MIX, s.vbuf, false);
+          gemv(ST_MIX, s.vbuf);
           if (aborted()) goto done;
           const StageCta &c = s.misc->sc[ST_MIX];
-          const int nseg = a.shape[ST_MIX].nseg;
           float *dst = a.dsum + size_t((L - 1) % delta) * d;
-          for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(i, nseg);
+          for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(i);
           signal(SY_MIXF);
           if (!gate(SY_MIXF, lm_count * nc, 0x70, 2)) goto done;
         }
@@ -1148,7 +1197,7 @@ struct Consumer {
               },
               a.gain_final, d, d);
         }
-        gemv(ST_LM, s.vbuf, false);
+        gemv(ST_LM, s.vbuf);
         if (aborted()) goto done;
         lm_epilogue();
         signal(SY_TOK);
@@ -1180,6 +1229,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
   s.svec = s.part + a.part_floats;
   s.misc = reinterpret_cast<Misc *>(s.svec + kSvecFloats);
 
+  for (int i = tid; i < a.part_floats; i += kThreads) s.part[i] = 0.f;   // row sums start at zero
   const int b0 = a.cta_blk_begin[cta], b1 = a.cta_blk_begin[cta + 1];
   for (int i = tid; i < b1 - b0; i += kThreads) s.misc->blk[i] = a.blocks[b0 + i];
   if (tid < ST_COUNT) s.misc->sc[tid] = a.stage_cta[tid * a.n_ctas + cta];
