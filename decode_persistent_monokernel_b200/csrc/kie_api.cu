@@ -320,6 +320,11 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
   int vb = 2 * d;   // normalised input and its gains
   vb = std::max(vb, (G + 2) * dh + kConsumerWarps * G * (dh + 2));   // attention scratch
   vb = std::max(vb, G * std::min((n_ctas + Hkv - 1) / Hkv, kMaxSplit) * (dh + 2));  // group partials
+  for (int g = 0; g < Hkv; ++g) {   // merge staging: (m, l) of every split + own output columns
+    const int ng = (n_ctas - 1 - g) / Hkv + 1;
+    const int nr = (G * dh + ng - 1) / ng;
+    vb = std::max(vb, 2 * G * kMaxSplit + std::min(ng, kMaxSplit) * nr);
+  }
   for (int k : {int(ST_O), int(ST_D)})                               // column-stage phases
     vb = std::max(vb, P.shape[k].nseg * P.shape[k].K);
   P.vbuf_floats = (vb + 3) / 4 * 4;

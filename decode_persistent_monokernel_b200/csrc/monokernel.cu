@@ -60,7 +60,7 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
                : "memory");
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t *b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
   uint32_t ok;
@@ -536,6 +536,14 @@ struct Consumer {
     KT(TE_TILE_READY, 0);
     return __shfl_sync(0xffffffffu, got, 0);
   }
+  // Hands ring slot `sl` back to the producer as soon as this warp has
+  // loaded its words from it: __syncwarp orders every lane's loads before
+  // lane 0's arrive, whose release semantics order them before the producer
+  // can observe the arrival and overwrite the slot.
+  __device__ void release_slot(uint32_t sl) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[sl]);
+  }
   __device__ void slot_advance() {
     if (++slot == uint32_t(a.ring_slots)) { slot = 0; phase ^= 1u; }
   }
@@ -587,22 +595,26 @@ struct Consumer {
       x = row_inputs(vin, s.misc->blk[b0 + bi].in_off, col0);
       rows = min(R, s.misc->blk[b0 + bi].nrows);
       ok = tile_wait(k);
-      if (ok) w = row_words(off0, lrow, rpl, rows);
+      if (ok) {
+        w = row_words(off0, lrow, rpl, rows);
+        release_slot(slot);
+      }
       slot_advance();
     }
     while (ok && bi < nblk) {
-      const uint32_t held = slot == 0 ? uint32_t(a.ring_slots) - 1 : slot - 1;
       int nbi = bi, nt = t;
       next_tile(b0, nblk, R, nbi, nt);
       const bool more = nbi < nblk;
       int nrows = 0;
+      uint32_t nslot = slot;
       if (more) {
         nrows = min(R, s.misc->blk[b0 + nbi].nrows - nt * R);
         ok = tile_wait(k);
         if (ok) wn = row_words(off0, lrow, rpl, nrows);
         slot_advance();
       }
-      // arithmetic of the current tile: four 8-term dot products
+      // arithmetic of the current tile (already released): four 8-term dot
+      // products, while the next tile's loads are in flight
       float p[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -610,8 +622,8 @@ struct Consumer {
         p[q] = d.x + d.y;
       }
       KT(TE_TILE_MATH, p[0] != p[0]);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.empty[held]);
+      // the next tile's words are in registers: hand its slot back at once
+      if (more && ok) release_slot(nslot);
       KT(TE_TILE_DONE, 0);
       // reduce each row over its lpr lanes, then one shared atomic per row
       float *prow = s.part + s.misc->blk[b0 + bi].lrow0 + t * R + lrow;   // + value * rpl
@@ -869,35 +881,42 @@ struct Consumer {
     KT(TE_ATTN, 2);
     signal(SY_QG0 + Hkv + g);
     if (!gate(SY_QG0 + Hkv + g, (gl + 1) * uint32_t(ngroup), 0x28, 5)) return;
-    float *pb = s.vbuf;   // [G][nsplit][st]
-    for (int i = 0; i < G; ++i) {
-      const float *src = a.attn_part + size_t(g * G + i) * a.max_split * st;
-      for (int q = tid; q < nsplit * st; q += kNC) pb[(size_t(i) * nsplit) * st + q] = __ldcg(src + q);
+    // This SM's O projection reads only the merged outputs [r0, r0 + nr) of
+    // the group's G*dh: stage every split's (m, l) and those output columns.
+    const int r0 = s.misc->sc[ST_O].row0, nr = s.misc->sc[ST_O].nout;
+    float *pml = s.vbuf;                       // [G][nsplit][2]
+    float *po = pml + 2 * G * kMaxSplit;       // [nsplit][nr]
+    for (int q = tid; q < 2 * G * nsplit; q += kNC) {
+      const int i = q / (2 * nsplit), r = q - i * 2 * nsplit;
+      pml[q] = __ldcg(a.attn_part + (size_t(g * G + i) * a.max_split + (r >> 1)) * st + dh + (r & 1));
+    }
+    for (int q = tid; q < nsplit * nr; q += kNC) {
+      const int sp = q / nr, idx = r0 + (q - sp * nr);
+      const int i = idx / dh, d = idx - i * dh;
+      po[q] = __ldcg(a.attn_part + (size_t(g * G + i) * a.max_split + sp) * st + d);
     }
     cbar();
     // log-sum-exp merge of the splits: warp i computes head i's weights
     // exp(m_s - M) / sum_s l_s exp(m_s - M) once (lane = split), then every
-    // output element is an nsplit-term weighted sum.  The split holding
-    // position p is never empty, so the denominator is positive.
+    // needed output element is an nsplit-term weighted sum.  The split
+    // holding position p is never empty, so the denominator is positive.
     if (warp < G) {
       const int i = warp;
-      const float *src = pb + size_t(i) * nsplit * st;
-      const float ms = lane < nsplit ? src[size_t(lane) * st + dh] : -INFINITY;
+      const float ms = lane < nsplit ? pml[(i * nsplit + lane) * 2] : -INFINITY;
       float M = ms;
       for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
       const float f = ms == -INFINITY ? 0.f : expf(ms - M);
-      float L = lane < nsplit ? f * src[size_t(lane) * st + dh + 1] : 0.f;
+      float L = lane < nsplit ? f * pml[(i * nsplit + lane) * 2 + 1] : 0.f;
       for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
       fac[i * 32 + lane] = f / L;
     }
     cbar();
-    float *og = s.svec;   // [G * dh] merged attention output of the group
-    for (int idx = tid; idx < G * dh; idx += kNC) {
-      const int i = idx / dh, d = idx - i * dh;
-      const float *src = pb + size_t(i) * nsplit * st;
+    float *og = s.svec;   // [G * dh] merged attention output of the group (rows r0.. used)
+    for (int q = tid; q < nr; q += kNC) {
+      const int idx = r0 + q, i = idx / dh;
       float O = 0.f;
 #pragma unroll 4
-      for (int sp = 0; sp < nsplit; ++sp) O = fmaf(fac[i * 32 + sp], src[size_t(sp) * st + d], O);
+      for (int sp = 0; sp < nsplit; ++sp) O = fmaf(fac[i * 32 + sp], po[sp * nr + q], O);
       og[idx] = O;
     }
     cbar();
@@ -962,14 +981,17 @@ struct Consumer {
     if (bi < nblk) {
       rows = min(R, s.misc->blk[b0 + bi].nrows);
       if (ok) ok = tile_wait(k);
-      if (ok) cw = col_words<CPS>(sh, ph, gi, tpr, rows);
+      if (ok) {
+        cw = col_words<CPS>(sh, ph, gi, tpr, rows);
+        release_slot(slot);
+      }
       slot_advance();
     }
     while (bi < nblk) {
-      const uint32_t held = slot == 0 ? uint32_t(a.ring_slots) - 1 : slot - 1;
       int nbi = bi, nt = t, nrows = 0;
       next_tile(b0, nblk, R, nbi, nt);
       const bool more = nbi < nblk;
+      const uint32_t nslot = slot;
       if (more) {
         nrows = min(R, s.misc->blk[b0 + nbi].nrows - nt * R);
         if (ok) ok = tile_wait(k);
@@ -990,10 +1012,9 @@ struct Consumer {
           }
         }
         KT(TE_TILE_MATH, acc2[0][0].x != acc2[0][0].x);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.empty[held]);
-        KT(TE_TILE_DONE, 0);
       }
+      if (more && ok) release_slot(nslot);
+      KT(TE_TILE_DONE, 0);
       if (nbi != bi) {
         // the block is complete: add its groups into the accumulator
         float *dst = acc + s.misc->blk[b0 + bi].out_off;
