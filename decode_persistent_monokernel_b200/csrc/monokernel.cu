@@ -529,7 +529,7 @@ struct Consumer {
   };
 
   // Waits (warp-wide outcome) for the weight tile in the current ring slot.
-  __device__ bool tile_wait(int k) {
+  __device__ __forceinline__ bool tile_wait(int k) {
     bool got = true;
     KT(TE_TILE_WAIT, 0);
     if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [] {});
@@ -540,25 +540,14 @@ struct Consumer {
   // loaded its words from it: __syncwarp orders every lane's loads before
   // lane 0's arrive, whose release semantics order them before the producer
   // can observe the arrival and overwrite the slot.
-  __device__ void release_slot(uint32_t sl) {
+  __device__ __forceinline__ void release_slot(uint32_t sl) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.empty[sl]);
   }
   __device__ void slot_advance() {
     if (++slot == uint32_t(a.ring_slots)) { slot = 0; phase ^= 1u; }
   }
-  // This lane's four 16-byte chunks of the tile in the current slot (rows
-  // lrow + q * rpl; zero beyond the tile's `rows`).
-  __device__ Words4 row_words(uint32_t off0, int lrow, int rpl, int rows) const {
-    Words4 w;
-    const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes + off0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      w.q[q] = (lrow + q * rpl < rows) ? *reinterpret_cast<const uint4 *>(tile + q * 8192)
-                                       : make_uint4(0u, 0u, 0u, 0u);
-    return w;
-  }
-  __device__ Inputs8 row_inputs(const float *vin, int in_off, int col0) const {
+  __device__ __forceinline__ Inputs8 row_inputs(const float *vin, int in_off, int col0) const {
     const float4 *src = reinterpret_cast<const float4 *>(vin + in_off + col0);
     const float4 x0 = src[0], x1 = src[1];
     Inputs8 x;
@@ -573,91 +562,118 @@ struct Consumer {
     while (bi < nblk && s.misc->blk[b0 + bi].nrows == 0) ++bi;
   }
 
-  __device__ void gemv(int k, const float *vin) {
+  __device__ void gemv(int k, const float *vin) { gemv_rows(k, vin); }
+
+  struct Dots4 {
+    float p[4];
+  };
+  __device__ __forceinline__ Dots4 row_tile_dots(const Words4 &w, const Inputs8 &x) const {
+    Dots4 d4;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 d = dot8x2<T>(w.q[q], x.v, make_float2(0.f, 0.f));
+      d4.p[q] = d.x + d.y;
+    }
+    return d4;
+  }
+  // Reduces one tile's four dot products over the LPR lanes of each row and
+  // adds them into the rows' shared-memory sums (`rows` < R only for the last
+  // tile of a block).
+  __device__ __forceinline__ void row_tile_reduce(const Dots4 &d4, float *prow, int lrow, int rows,
+                                                  bool full, int LSH) {
+    const int LPR = 1 << LSH, RPL = 32 >> LSH;
+    const float *p = d4.p;
+    KT(TE_TILE_MATH, p[0] != p[0]);
+    if (LSH == 0) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (full || lrow + q * RPL < rows) sred_add(prow + q * RPL, p[q]);
+    } else {
+      const int H = LPR >> 1;
+      const bool hi = lane & H;
+      const float s0 = __shfl_xor_sync(0xffffffffu, hi ? p[0] : p[2], H);
+      const float s1 = __shfl_xor_sync(0xffffffffu, hi ? p[1] : p[3], H);
+      const float a0 = (hi ? p[2] : p[0]) + s0;   // value 2 if hi else 0
+      const float a1 = (hi ? p[3] : p[1]) + s1;   // value 3 if hi else 1
+      const int v0 = hi ? 2 : 0;
+      if (LSH == 1) {
+        if (full || lrow + v0 * RPL < rows) sred_add(prow + v0 * RPL, a0);
+        if (full || lrow + (v0 + 1) * RPL < rows) sred_add(prow + (v0 + 1) * RPL, a1);
+      } else {
+        const int H2 = LPR >> 2;
+        const bool hi2 = lane & H2;
+        const float s2 = __shfl_xor_sync(0xffffffffu, hi2 ? a0 : a1, H2);
+        float v = (hi2 ? a1 : a0) + s2;           // value v0 + hi2
+        for (int o = LPR >> 3; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        const int vi = v0 + (hi2 ? 1 : 0);
+        if ((lane & (H2 - 1)) == 0 && (full || lrow + vi * RPL < rows)) sred_add(prow + vi * RPL, v);
+      }
+    }
+  }
+
+  // This lane's words of the tile in the current ring slot; the slot index
+  // is returned in `sl` and the ring position advanced.
+  __device__ __forceinline__ Words4 row_fetch(int k, uint32_t off0, int lrow, int rows, bool full,
+                                              uint32_t &sl, bool &ok, int RPL) {
+    Words4 w;
+    sl = slot;
+    ok = ok && tile_wait(k);
+    const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes + off0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      w.q[q] = (ok && (full || lrow + q * RPL < rows)) ? *reinterpret_cast<const uint4 *>(tile + q * 8192)
+                                                      : make_uint4(0u, 0u, 0u, 0u);
+    slot_advance();
+    return w;
+  }
+
+  // Row stage (K/128 lanes per row).  Tiles of a block are processed in pairs
+  // with two register sets (no copies): the next tile is fetched before the
+  // current one's arithmetic and its slot handed back right after it.
+  __device__ void gemv_rows(int k, const float *vin) {
     KP_BEGIN(t_gemv);
     KT(TE_STAGE_BEGIN, k);
     const StageCta &c = s.misc->sc[k];
     const int K = a.shape[k].K, R = a.shape[k].R;
-    const int lsh = __ffs(K >> 7) - 1;          // log2(lanes per row)
-    const int lpr = 1 << lsh;
-    const int lrow = lane >> lsh;               // this lane's row within a load
-    const int rpl = 32 >> lsh;                  // rows per load
-    const int col0 = warp * (K >> 4) + ((lane & (lpr - 1)) << 3);
+    const int LSH = __ffs(K >> 7) - 1;         // log2 of the lanes that share a row
+    const int LPR = 1 << LSH, RPL = 32 >> LSH;
+    const int lrow = lane >> LSH;               // this lane's row within a load
+    const int col0 = warp * (K >> 4) + ((lane & (LPR - 1)) << 3);
     const uint32_t off0 = uint32_t(lrow * K + col0) * 2u;   // + q * 8192 bytes
-    const int nblk = c.nblk, b0 = c.blk_begin;
     bool ok = !aborted();
-    int bi = 0, t = 0;
-    while (bi < nblk && s.misc->blk[b0 + bi].nrows == 0) ++bi;
-    Words4 w{}, wn{};
-    Inputs8 x{};
-    int rows = 0;
-    if (bi < nblk && ok) {
-      x = row_inputs(vin, s.misc->blk[b0 + bi].in_off, col0);
-      rows = min(R, s.misc->blk[b0 + bi].nrows);
-      ok = tile_wait(k);
-      if (ok) {
-        w = row_words(off0, lrow, rpl, rows);
-        release_slot(slot);
+    for (int bi = 0; bi < c.nblk && ok; ++bi) {
+      const Block b = s.misc->blk[c.blk_begin + bi];
+      if (b.nrows == 0) continue;
+      const Inputs8 x = row_inputs(vin, b.in_off, col0);
+      const int n = (b.nrows + R - 1) / R;     // tiles of the block; the last may be partial
+      const int last_rows = b.nrows - (n - 1) * R;
+      float *prow0 = s.part + b.lrow0 + lrow;
+      uint32_t sa = 0, sb = 0;
+      Words4 wa = row_fetch(k, off0, lrow, n == 1 ? last_rows : R, n > 1, sa, ok, RPL);
+      if (ok) release_slot(sa);
+      for (int t = 0; t < n && ok; t += 2) {
+        // tile t in wa (released), tile t + 1 into wb
+        const bool has_b = t + 1 < n;
+        const bool b_full = t + 1 < n - 1;
+        Words4 wb{};
+        if (has_b) wb = row_fetch(k, off0, lrow, b_full ? R : last_rows, b_full, sb, ok, RPL);
+        const bool a_full = t < n - 1;
+        // the slot goes back before the shared atomics, whose completion the
+        // arrive's release semantics would otherwise wait for
+        const Dots4 da = row_tile_dots(wa, x);
+        if (has_b && ok) release_slot(sb);
+        row_tile_reduce(da, prow0 + t * R, lrow, a_full ? R : last_rows, a_full, LSH);
+        KT(TE_TILE_DONE, 0);
+        if (!has_b || !ok) break;
+        // tile t + 1 in wb (released), tile t + 2 into wa
+        const bool has_a = t + 2 < n;
+        const bool a2_full = t + 2 < n - 1;
+        if (has_a) wa = row_fetch(k, off0, lrow, a2_full ? R : last_rows, a2_full, sa, ok, RPL);
+        const Dots4 db = row_tile_dots(wb, x);
+        if (has_a && ok) release_slot(sa);
+        row_tile_reduce(db, prow0 + (t + 1) * R, lrow, b_full ? R : last_rows, b_full, LSH);
+        KT(TE_TILE_DONE, 0);
       }
-      slot_advance();
-    }
-    while (ok && bi < nblk) {
-      int nbi = bi, nt = t;
-      next_tile(b0, nblk, R, nbi, nt);
-      const bool more = nbi < nblk;
-      int nrows = 0;
-      uint32_t nslot = slot;
-      if (more) {
-        nrows = min(R, s.misc->blk[b0 + nbi].nrows - nt * R);
-        ok = tile_wait(k);
-        if (ok) wn = row_words(off0, lrow, rpl, nrows);
-        slot_advance();
-      }
-      // arithmetic of the current tile (already released): four 8-term dot
-      // products, while the next tile's loads are in flight
-      float p[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 d = dot8x2<T>(w.q[q], x.v, make_float2(0.f, 0.f));
-        p[q] = d.x + d.y;
-      }
-      KT(TE_TILE_MATH, p[0] != p[0]);
-      // the next tile's words are in registers: hand its slot back at once
-      if (more && ok) release_slot(nslot);
-      KT(TE_TILE_DONE, 0);
-      // reduce each row over its lpr lanes, then one shared atomic per row
-      float *prow = s.part + s.misc->blk[b0 + bi].lrow0 + t * R + lrow;   // + value * rpl
-      if (lsh == 0) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (lrow + q * rpl < rows) sred_add(prow + q * rpl, p[q]);
-      } else {
-        const int h = lpr >> 1;
-        const bool hi = lane & h;
-        const float s0 = __shfl_xor_sync(0xffffffffu, hi ? p[0] : p[2], h);
-        const float s1 = __shfl_xor_sync(0xffffffffu, hi ? p[1] : p[3], h);
-        const float a0 = (hi ? p[2] : p[0]) + s0;   // value 2 if hi else 0
-        const float a1 = (hi ? p[3] : p[1]) + s1;   // value 3 if hi else 1
-        const int v0 = hi ? 2 : 0;
-        if (lsh == 1) {
-          if (lrow + v0 * rpl < rows) sred_add(prow + v0 * rpl, a0);
-          if (lrow + (v0 + 1) * rpl < rows) sred_add(prow + (v0 + 1) * rpl, a1);
-        } else {
-          const int h2 = lpr >> 2;
-          const bool hi2 = lane & h2;
-          const float s2 = __shfl_xor_sync(0xffffffffu, hi2 ? a0 : a1, h2);
-          float v = (hi2 ? a1 : a0) + s2;          // value v0 + hi2
-          for (int o = lpr >> 3; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          const int vi = v0 + (hi2 ? 1 : 0);
-          if ((lane & (h2 - 1)) == 0 && lrow + vi * rpl < rows) sred_add(prow + vi * rpl, v);
-        }
-      }
-      if (!ok || !more) break;
-      if (nbi != bi) x = row_inputs(vin, s.misc->blk[b0 + nbi].in_off, col0);
-      w = wn;
-      bi = nbi;
-      t = nt;
-      rows = nrows;
     }
     if (!ok) s.misc->abort = 1;
     Tbase += c.ntiles;
@@ -958,6 +974,34 @@ struct Consumer {
     else gemv_cols_impl<2>(k, svals, acc);
   }
 
+  // Accumulates one tile (its rows ph, ph + nseg, ...) into acc2.
+  template <int CPS>
+  __device__ __forceinline__ void col_tile_math(const ColWords<CPS> &cw, const float *sv, int ph,
+                                                int nseg, int rows, float2 (&acc2)[CPS][2]) const {
+#pragma unroll
+    for (int q = 0; q < 8 / CPS; ++q) {
+      const int r = ph + q * nseg;
+      const float xv = r < rows ? sv[r] : 0.f;
+      const float2 xx = make_float2(xv, xv);
+#pragma unroll
+      for (int j = 0; j < CPS; ++j) {
+        acc2[j][0] = __ffma2_rn(Store<T>::pair(cw.w[q][j].x), xx, acc2[j][0]);
+        acc2[j][1] = __ffma2_rn(Store<T>::pair(cw.w[q][j].y), xx, acc2[j][1]);
+      }
+    }
+  }
+
+  template <int CPS>
+  __device__ __forceinline__ ColWords<CPS> col_fetch(int k, const StageShape &sh, int ph, int gi,
+                                                     int tpr, int rows, uint32_t &sl, bool &ok) {
+    ColWords<CPS> cw{};
+    sl = slot;
+    ok = ok && tile_wait(k);
+    if (ok) cw = col_words<CPS>(sh, ph, gi, tpr, rows);
+    slot_advance();
+    return cw;
+  }
+
   template <int CPS>
   __device__ void gemv_cols_impl(int k, const float *svals, float *acc) {
     KP_BEGIN(t_gemv);
@@ -967,84 +1011,59 @@ struct Consumer {
     const int ngrp = sh.K >> 2;                  // 4-element groups of the output
     const int tpr = sh.nseg > 1 ? ngrp : kNC;    // threads per row phase
     const int ph = tid / tpr, gi = tid - ph * tpr;
-    const int nblk = c.nblk, b0 = c.blk_begin, R = sh.R;
+    const int R = sh.R;
     // A failed wait stops this warp's tile work, but every warp still goes
     // through the same barriers so that none is left waiting.
     bool ok = !aborted();
-    int bi = 0, t = 0;
-    while (bi < nblk && s.misc->blk[b0 + bi].nrows == 0) ++bi;
-    ColWords<CPS> cw{}, cn{};
-    float2 acc2[CPS][2];
+    for (int bi = 0; bi < c.nblk; ++bi) {
+      const Block b = s.misc->blk[c.blk_begin + bi];
+      if (b.nrows == 0) continue;
+      const int n = (b.nrows + R - 1) / R;
+      const int last_rows = b.nrows - (n - 1) * R;
+      const float *sv0 = svals + b.lrow0;
+      float2 acc2[CPS][2];
 #pragma unroll
-    for (int j = 0; j < CPS; ++j) acc2[j][0] = acc2[j][1] = make_float2(0.f, 0.f);
-    int rows = 0;
-    if (bi < nblk) {
-      rows = min(R, s.misc->blk[b0 + bi].nrows);
-      if (ok) ok = tile_wait(k);
-      if (ok) {
-        cw = col_words<CPS>(sh, ph, gi, tpr, rows);
-        release_slot(slot);
+      for (int j = 0; j < CPS; ++j) acc2[j][0] = acc2[j][1] = make_float2(0.f, 0.f);
+      uint32_t sa = 0, sb = 0;
+      ColWords<CPS> ca = col_fetch<CPS>(k, sh, ph, gi, tpr, n == 1 ? last_rows : R, sa, ok);
+      if (ok) release_slot(sa);
+      for (int t = 0; t < n && ok; t += 2) {
+        const bool has_b = t + 1 < n;
+        const int rows_b = t + 1 < n - 1 ? R : last_rows;
+        ColWords<CPS> cb{};
+        if (has_b) cb = col_fetch<CPS>(k, sh, ph, gi, tpr, rows_b, sb, ok);
+        col_tile_math<CPS>(ca, sv0 + t * R, ph, sh.nseg, t < n - 1 ? R : last_rows, acc2);
+        KT(TE_TILE_MATH, 0);
+        if (!has_b || !ok) break;
+        release_slot(sb);
+        KT(TE_TILE_DONE, 0);
+        const bool has_a = t + 2 < n;
+        if (has_a) ca = col_fetch<CPS>(k, sh, ph, gi, tpr, t + 2 < n - 1 ? R : last_rows, sa, ok);
+        col_tile_math<CPS>(cb, sv0 + (t + 1) * R, ph, sh.nseg, rows_b, acc2);
+        if (has_a && ok) release_slot(sa);
+        KT(TE_TILE_DONE, 0);
       }
-      slot_advance();
-    }
-    while (bi < nblk) {
-      int nbi = bi, nt = t, nrows = 0;
-      next_tile(b0, nblk, R, nbi, nt);
-      const bool more = nbi < nblk;
-      const uint32_t nslot = slot;
-      if (more) {
-        nrows = min(R, s.misc->blk[b0 + nbi].nrows - nt * R);
-        if (ok) ok = tile_wait(k);
-        if (ok) cn = col_words<CPS>(sh, ph, gi, tpr, nrows);
-        slot_advance();
-      }
-      if (ok) {
-        const float *sv = svals + s.misc->blk[b0 + bi].lrow0 + t * R;
+      // the block is complete: add its groups into the accumulator
+      float *dst = acc + b.out_off;
+      if (sh.nseg == 1) {
+        if (ok) {
 #pragma unroll
-        for (int q = 0; q < 8 / CPS; ++q) {
-          const int r = ph + q * sh.nseg;
-          const float xv = r < rows ? sv[r] : 0.f;
-          const float2 xx = make_float2(xv, xv);
-#pragma unroll
-          for (int j = 0; j < CPS; ++j) {
-            acc2[j][0] = __ffma2_rn(Store<T>::pair(cw.w[q][j].x), xx, acc2[j][0]);
-            acc2[j][1] = __ffma2_rn(Store<T>::pair(cw.w[q][j].y), xx, acc2[j][1]);
-          }
+          for (int j = 0; j < CPS; ++j)
+            red_add_v4(dst + 4 * (gi + tpr * j),
+                       make_float4(acc2[j][0].x, acc2[j][0].y, acc2[j][1].x, acc2[j][1].y));
         }
-        KT(TE_TILE_MATH, acc2[0][0].x != acc2[0][0].x);
-      }
-      if (more && ok) release_slot(nslot);
-      KT(TE_TILE_DONE, 0);
-      if (nbi != bi) {
-        // the block is complete: add its groups into the accumulator
-        float *dst = acc + s.misc->blk[b0 + bi].out_off;
-        if (sh.nseg == 1) {
-          if (ok) {
-#pragma unroll
-            for (int j = 0; j < CPS; ++j)
-              red_add_v4(dst + 4 * (gi + tpr * j),
-                         make_float4(acc2[j][0].x, acc2[j][0].y, acc2[j][1].x, acc2[j][1].y));
-          }
-        } else {
-          // several row phases: add them up in shared memory first (CPS == 1)
-          float4 *scr = reinterpret_cast<float4 *>(s.vbuf);
-          scr[ph * ngrp + gi] = make_float4(acc2[0][0].x, acc2[0][0].y, acc2[0][1].x, acc2[0][1].y);
-          cbar();
-          if (tid < ngrp && !aborted()) {
-            float4 v = scr[tid];
-            for (int q = 1; q < sh.nseg; ++q) v = add4(v, scr[q * ngrp + tid]);
-            red_add_v4(dst + 4 * tid, v);
-          }
-          cbar();
+      } else {
+        // several row phases: add them up in shared memory first (CPS == 1)
+        float4 *scr = reinterpret_cast<float4 *>(s.vbuf);
+        scr[ph * ngrp + gi] = make_float4(acc2[0][0].x, acc2[0][0].y, acc2[0][1].x, acc2[0][1].y);
+        cbar();
+        if (tid < ngrp && !aborted()) {
+          float4 v = scr[tid];
+          for (int q = 1; q < sh.nseg; ++q) v = add4(v, scr[q * ngrp + tid]);
+          red_add_v4(dst + 4 * tid, v);
         }
-#pragma unroll
-        for (int j = 0; j < CPS; ++j) acc2[j][0] = acc2[j][1] = make_float2(0.f, 0.f);
+        cbar();
       }
-      if (!more) break;
-      cw = cn;
-      bi = nbi;
-      t = nt;
-      rows = nrows;
     }
     if (!ok) s.misc->abort = 1;
     Tbase += c.ntiles;
