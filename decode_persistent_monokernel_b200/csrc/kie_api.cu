@@ -98,6 +98,7 @@ struct Plan {
   std::vector<RepackJob> jobs;
   int64_t stream_bytes = 0;
   int vbuf_floats = 0, part_floats = 0, ring_slots = 0;
+  int part_atomic_off = 0;   // start of the atomic row sums inside the partials buffer
   size_t smem = 0;
   int max_split = 0;
   int64_t weight_bytes_per_step = 0;
@@ -198,6 +199,7 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
   std::vector<std::vector<Piece>> src_of_cta(n_ctas);
   P.cta_blk_begin.assign(n_ctas + 1, 0);
   int part_max = 4;
+  int max_local[ST_COUNT] = {};   // most output rows of a row stage on one CTA
   for (int c = 0; c < n_ctas; ++c) {
     P.cta_blk_begin[c] = int(P.blocks.size());
     int local_blk = 0;
@@ -268,7 +270,7 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
       int64_t bytes = 0;
       for (const Block &B : blk) bytes += int64_t(B.nrows) * sh.K * 2;
       sc.bytes = bytes;
-      if (!sh.cols) part_max = std::max(part_max, sc.nlocal * sh.nseg);
+      if (!sh.cols) max_local[k] = std::max(max_local[k], sc.nlocal);
       if (sh.cols && sc.nlocal > kMaxLocal) return "too many split-projection rows per CTA";
       if (k == ST_GU && sc.nout > kMaxLocal) return "hidden slice per CTA too large";
       for (size_t i = 0; i < blk.size(); ++i) {
@@ -328,6 +330,20 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
   for (int k : {int(ST_O), int(ST_D)})                               // column-stage phases
     vb = std::max(vb, P.shape[k].nseg * P.shape[k].K);
   P.vbuf_floats = (vb + 3) / 4 * 4;
+  // Row-stage sums: 16 per-warp partials per row (plain stores, added in a
+  // fixed order by the epilogue) when they fit kPartialFloats, else one
+  // shared-memory atomic accumulator per row.
+  // The two kinds live in disjoint regions: the atomic sums must be zero on
+  // entry (their readers clear them), the partials are overwritten each time.
+  int partial_max = 0, atomic_max = 0;
+  for (int k = 0; k < ST_COUNT; ++k) {
+    if (P.shape[k].cols) continue;
+    P.shape[k].nseg = max_local[k] * kConsumerWarps <= kPartialFloats ? kConsumerWarps : 1;
+    if (P.shape[k].nseg > 1) partial_max = std::max(partial_max, max_local[k] * kConsumerWarps);
+    else atomic_max = std::max(atomic_max, max_local[k]);
+  }
+  P.part_atomic_off = (partial_max + 3) / 4 * 4;
+  part_max = std::max(part_max, P.part_atomic_off + atomic_max);
   P.part_floats = (part_max + 3) / 4 * 4;
   const size_t fixed = monokernel_smem_bytes(0, P.vbuf_floats, P.part_floats);
   if (fixed + 3 * (kSlotBytes + 16) > smem_cap) return "shape needs more shared memory than the SM has";
@@ -640,6 +656,7 @@ static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int fi
   a.max_seq = m.max_seq;
   a.n_ctas = P.n_ctas; a.ring_slots = P.ring_slots;
   a.vbuf_floats = P.vbuf_floats; a.part_floats = P.part_floats;
+  a.part_atomic_off = P.part_atomic_off;
   for (int k = 0; k < ST_COUNT; ++k) a.shape[k] = P.shape[k];
   a.stage_cta = ctx->d_stage_cta; a.blocks = ctx->d_blocks;
   a.cta_blk_begin = ctx->d_blk_begin; a.cta_stream_off = ctx->d_stream_off;
@@ -931,6 +948,7 @@ extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t
   a.max_seq = m.max_seq;
   a.n_ctas = P.n_ctas; a.ring_slots = P.ring_slots;
   a.vbuf_floats = P.vbuf_floats; a.part_floats = P.part_floats;
+  a.part_atomic_off = P.part_atomic_off;
   for (int k = 0; k < ST_COUNT; ++k) a.shape[k] = P.shape[k];
   a.stage_cta = ctx->d_stage_cta; a.blocks = ctx->d_blocks;
   a.cta_blk_begin = ctx->d_blk_begin; a.cta_stream_off = ctx->d_stream_off;

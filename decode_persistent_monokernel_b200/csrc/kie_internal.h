@@ -84,7 +84,8 @@ constexpr int kTraceCap = 1 << 16;
 struct StageShape {
   int32_t K;       // row length (row stages: reduction length; column stages: output length)
   int32_t R;       // rows per tile (power of two)
-  int32_t nseg;    // row stages: column splits per row; column stages: row phases
+  int32_t nseg;    // row stages: partial sums kept per row (16: one per consumer warp,
+                   // 1: a shared-memory atomic sum); column stages: row phases
   int32_t rpw;     // row stages: rows per warp (1 unless R > 16)
   int32_t cps;     // row stages: 8-element chunks per (row, split);
                    // column stages: 4-element output groups per thread
@@ -128,6 +129,7 @@ constexpr int kMaxBlocksPerCta = 64;
 constexpr int kSlotBytes = 32768;  // one bulk copy per tile: >= 16 KB keeps HBM saturated
 constexpr int kConsumerWarps = 16;
 constexpr int kMaxLocal = 256;     // scalars a column stage holds per CTA
+constexpr int kPartialFloats = 4096;  // shared-memory budget of per-warp row partials
 constexpr int kMaxSplit = 32;      // CTAs that share one KV head's positions (others only merge)
 
 struct KernelArgs {
@@ -139,6 +141,7 @@ struct KernelArgs {
   int32_t max_seq;
   // plan
   int32_t n_ctas, ring_slots, vbuf_floats, part_floats;
+  int32_t part_atomic_off;      // row sums kept as shared atomics start here in `part`
   StageShape shape[ST_COUNT];
   const StageCta *stage_cta;  // [ST_COUNT][n_ctas]
   const Block *blocks;

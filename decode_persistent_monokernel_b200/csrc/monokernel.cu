@@ -547,6 +547,63 @@ struct Consumer {
   __device__ void slot_advance() {
     if (++slot == uint32_t(a.ring_slots)) { slot = 0; phase ^= 1u; }
   }
+  // Input of a row stage: a vector already staged in shared memory (v), or,
+  // for the dense model, RMSNorm fused into the stage: x = g0 + g1 [+ g2]
+  // (global fp32 vectors) or an embedding row, times the gains; each lane
+  // loads its own 8 elements and the sum of squares goes to red_sq[warp], so
+  // the epilogue scales the row sums by rsqrt(mean(x^2) + eps) (the norm's
+  // scalar factor commutes with the dot product).
+  struct RowInput {
+    const float *v;
+    const float *g0, *g1, *g2;
+    const uint16_t *emb;
+    const float *gain;
+  };
+  __device__ __forceinline__ Inputs8 fused_inputs(const RowInput &in, int col0, int LSH) {
+    float e[8];
+    if (in.emb) {
+      const uint4 w = *reinterpret_cast<const uint4 *>(in.emb + col0);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = Store<T>::pair(ws[q]);
+        e[2 * q] = f.x;
+        e[2 * q + 1] = f.y;
+      }
+    } else {
+      const float4 *p0 = reinterpret_cast<const float4 *>(in.g0 + col0);
+      const float4 *p1 = reinterpret_cast<const float4 *>(in.g1 + col0);
+      float4 u0 = add4(__ldcg(p0), __ldcg(p1)), u1 = add4(__ldcg(p0 + 1), __ldcg(p1 + 1));
+      if (in.g2) {
+        const float4 *p2 = reinterpret_cast<const float4 *>(in.g2 + col0);
+        u0 = add4(u0, __ldcg(p2));
+        u1 = add4(u1, __ldcg(p2 + 1));
+      }
+      e[0] = u0.x; e[1] = u0.y; e[2] = u0.z; e[3] = u0.w;
+      e[4] = u1.x; e[5] = u1.y; e[6] = u1.z; e[7] = u1.w;
+    }
+    const float4 ga = *reinterpret_cast<const float4 *>(in.gain + col0);
+    const float4 gb = *reinterpret_cast<const float4 *>(in.gain + col0 + 4);
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss = fmaf(e[i], e[i], ss);
+    // the lanes of one row cover the warp's K/16 columns once
+    for (int o = (1 << LSH) >> 1; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) s.misc->red_sq[warp] = ss;
+    Inputs8 x;
+    x.v[0] = make_float2(e[0] * ga.x, e[1] * ga.y); x.v[1] = make_float2(e[2] * ga.z, e[3] * ga.w);
+    x.v[2] = make_float2(e[4] * gb.x, e[5] * gb.y); x.v[3] = make_float2(e[6] * gb.z, e[7] * gb.w);
+    return x;
+  }
+  // rsqrt(mean(x^2) + eps) of a fused stage's input, after the stage's barrier
+  __device__ float fused_scale(int n) const {
+    const float4 *q = reinterpret_cast<const float4 *>(s.misc->red_sq);
+    float4 v = q[0];
+#pragma unroll
+    for (int j = 1; j < kConsumerWarps / 4; ++j) v = add4(v, q[j]);
+    return rsqrtf(((v.x + v.y) + (v.z + v.w)) / float(n) + a.rms_eps);
+  }
+
   __device__ __forceinline__ Inputs8 row_inputs(const float *vin, int in_off, int col0) const {
     const float4 *src = reinterpret_cast<const float4 *>(vin + in_off + col0);
     const float4 x0 = src[0], x1 = src[1];
@@ -562,7 +619,11 @@ struct Consumer {
     while (bi < nblk && s.misc->blk[b0 + bi].nrows == 0) ++bi;
   }
 
-  __device__ void gemv(int k, const float *vin) { gemv_rows(k, vin); }
+  __device__ void gemv(int k, const float *vin) {
+    RowInput in{};
+    in.v = vin;
+    gemv_rows(k, in);
+  }
 
   struct Dots4 {
     float p[4];
@@ -579,15 +640,21 @@ struct Consumer {
   // Reduces one tile's four dot products over the LPR lanes of each row and
   // adds them into the rows' shared-memory sums (`rows` < R only for the last
   // tile of a block).
-  __device__ __forceinline__ void row_tile_reduce(const Dots4 &d4, float *prow, int lrow, int rows,
-                                                  bool full, int LSH) {
+  // prow: this lane's first row of the tile in the partial sums; rstride 16
+  // (per-warp partials: prow already includes + warp) or 1 (atomic sums).
+  __device__ __forceinline__ void row_put(float *pr, float v, int rstride) {
+    if (rstride == 1) sred_add(pr, v);
+    else *pr = v;
+  }
+  __device__ __forceinline__ void row_tile_reduce(const Dots4 &d4, float *prow, int rstride, int lrow,
+                                                  int rows, bool full, int LSH) {
     const int LPR = 1 << LSH, RPL = 32 >> LSH;
     const float *p = d4.p;
     KT(TE_TILE_MATH, p[0] != p[0]);
     if (LSH == 0) {
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        if (full || lrow + q * RPL < rows) sred_add(prow + q * RPL, p[q]);
+        if (full || lrow + q * RPL < rows) row_put(prow + q * RPL * rstride, p[q], rstride);
     } else {
       const int H = LPR >> 1;
       const bool hi = lane & H;
@@ -597,8 +664,8 @@ struct Consumer {
       const float a1 = (hi ? p[3] : p[1]) + s1;   // value 3 if hi else 1
       const int v0 = hi ? 2 : 0;
       if (LSH == 1) {
-        if (full || lrow + v0 * RPL < rows) sred_add(prow + v0 * RPL, a0);
-        if (full || lrow + (v0 + 1) * RPL < rows) sred_add(prow + (v0 + 1) * RPL, a1);
+        if (full || lrow + v0 * RPL < rows) row_put(prow + v0 * RPL * rstride, a0, rstride);
+        if (full || lrow + (v0 + 1) * RPL < rows) row_put(prow + (v0 + 1) * RPL * rstride, a1, rstride);
       } else {
         const int H2 = LPR >> 2;
         const bool hi2 = lane & H2;
@@ -606,8 +673,43 @@ struct Consumer {
         float v = (hi2 ? a1 : a0) + s2;           // value v0 + hi2
         for (int o = LPR >> 3; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         const int vi = v0 + (hi2 ? 1 : 0);
-        if ((lane & (H2 - 1)) == 0 && (full || lrow + vi * RPL < rows)) sred_add(prow + vi * RPL, v);
+        if ((lane & (H2 - 1)) == 0 && (full || lrow + vi * RPL < rows))
+          row_put(prow + vi * RPL * rstride, v, rstride);
       }
+    }
+  }
+
+  // Two tiles' dot products (da: tile at prow_a, db: the next tile at
+  // prow_b), reduced together over the LPR >= 8 lanes of each row: a
+  // transposed butterfly halves the values per lane at each of the first
+  // three steps (8 shuffles for 8 values with LPR = 16), then plain steps.
+  __device__ __forceinline__ void row_pair_reduce(const Dots4 &da, const Dots4 &db, float *prow_a,
+                                                  float *prow_b, int rstride, int lrow, int rows_a,
+                                                  int rows_b, int LSH) {
+    const int LPR = 1 << LSH, RPL = 32 >> LSH;
+    const int H = LPR >> 1, H2 = LPR >> 2, H3 = LPR >> 3;
+    const bool hi = lane & H, hi2 = lane & H2, hi3 = lane & H3;
+    float a4[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float keep = hi ? db.p[j] : da.p[j];        // values 4..7 if hi else 0..3
+      const float give = hi ? da.p[j] : db.p[j];
+      a4[j] = keep + __shfl_xor_sync(0xffffffffu, give, H);
+    }
+    float b2[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float keep = hi2 ? a4[2 + j] : a4[j];
+      const float give = hi2 ? a4[j] : a4[2 + j];
+      b2[j] = keep + __shfl_xor_sync(0xffffffffu, give, H2);
+    }
+    float v = (hi3 ? b2[1] : b2[0]) + __shfl_xor_sync(0xffffffffu, hi3 ? b2[0] : b2[1], H3);
+    for (int o = H3 >> 1; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int vi = (hi ? 4 : 0) + (hi2 ? 2 : 0) + (hi3 ? 1 : 0);
+    const int q = vi & 3, r = lrow + q * RPL;
+    if ((lane & (H3 - 1)) == 0) {
+      if (vi < 4) { if (r < rows_a) row_put(prow_a + q * RPL * rstride, v, rstride); }
+      else if (r < rows_b) row_put(prow_b + q * RPL * rstride, v, rstride);
     }
   }
 
@@ -630,7 +732,7 @@ struct Consumer {
   // Row stage (K/128 lanes per row).  Tiles of a block are processed in pairs
   // with two register sets (no copies): the next tile is fetched before the
   // current one's arithmetic and its slot handed back right after it.
-  __device__ void gemv_rows(int k, const float *vin) {
+  __device__ void gemv_rows(int k, const RowInput &in) {
     KP_BEGIN(t_gemv);
     KT(TE_STAGE_BEGIN, k);
     const StageCta &c = s.misc->sc[k];
@@ -641,13 +743,17 @@ struct Consumer {
     const int col0 = warp * (K >> 4) + ((lane & (LPR - 1)) << 3);
     const uint32_t off0 = uint32_t(lrow * K + col0) * 2u;   // + q * 8192 bytes
     bool ok = !aborted();
+    Inputs8 xf{};
+    if (!in.v) xf = fused_inputs(in, col0, LSH);   // every block reads the whole vector
     for (int bi = 0; bi < c.nblk && ok; ++bi) {
       const Block b = s.misc->blk[c.blk_begin + bi];
       if (b.nrows == 0) continue;
-      const Inputs8 x = row_inputs(vin, b.in_off, col0);
+      const Inputs8 x = in.v ? row_inputs(in.v, b.in_off, col0) : xf;
       const int n = (b.nrows + R - 1) / R;     // tiles of the block; the last may be partial
       const int last_rows = b.nrows - (n - 1) * R;
-      float *prow0 = s.part + b.lrow0 + lrow;
+      const int rstride = a.shape[k].nseg;      // 16 (per-warp partials) or 1 (atomic sums)
+      float *prow0 = rstride > 1 ? s.part + (b.lrow0 + lrow) * rstride + warp
+                                 : s.part + a.part_atomic_off + b.lrow0 + lrow;
       uint32_t sa = 0, sb = 0;
       Words4 wa = row_fetch(k, off0, lrow, n == 1 ? last_rows : R, n > 1, sa, ok, RPL);
       if (ok) release_slot(sa);
@@ -655,23 +761,31 @@ struct Consumer {
         // tile t in wa (released), tile t + 1 into wb
         const bool has_b = t + 1 < n;
         const bool b_full = t + 1 < n - 1;
+        const int rows_a = t < n - 1 ? R : last_rows, rows_b = b_full ? R : last_rows;
         Words4 wb{};
-        if (has_b) wb = row_fetch(k, off0, lrow, b_full ? R : last_rows, b_full, sb, ok, RPL);
-        const bool a_full = t < n - 1;
-        // the slot goes back before the shared atomics, whose completion the
-        // arrive's release semantics would otherwise wait for
+        if (has_b) wb = row_fetch(k, off0, lrow, rows_b, b_full, sb, ok, RPL);
+        // slots go back before the row sums are written (shared atomics in one
+        // mode), whose completion the arrive's release semantics would wait for
         const Dots4 da = row_tile_dots(wa, x);
         if (has_b && ok) release_slot(sb);
-        row_tile_reduce(da, prow0 + t * R, lrow, a_full ? R : last_rows, a_full, LSH);
-        KT(TE_TILE_DONE, 0);
-        if (!has_b || !ok) break;
+        if (!has_b || !ok) {
+          row_tile_reduce(da, prow0 + t * R * rstride, rstride, lrow, rows_a, rows_a == R, LSH);
+          KT(TE_TILE_DONE, 0);
+          break;
+        }
         // tile t + 1 in wb (released), tile t + 2 into wa
         const bool has_a = t + 2 < n;
         const bool a2_full = t + 2 < n - 1;
         if (has_a) wa = row_fetch(k, off0, lrow, a2_full ? R : last_rows, a2_full, sa, ok, RPL);
         const Dots4 db = row_tile_dots(wb, x);
         if (has_a && ok) release_slot(sa);
-        row_tile_reduce(db, prow0 + (t + 1) * R, lrow, b_full ? R : last_rows, b_full, LSH);
+        if (LSH >= 3) {
+          row_pair_reduce(da, db, prow0 + t * R * rstride, prow0 + (t + 1) * R * rstride, rstride, lrow,
+                          rows_a, rows_b, LSH);
+        } else {
+          row_tile_reduce(da, prow0 + t * R * rstride, rstride, lrow, rows_a, rows_a == R, LSH);
+          row_tile_reduce(db, prow0 + (t + 1) * R * rstride, rstride, lrow, rows_b, b_full, LSH);
+        }
         KT(TE_TILE_DONE, 0);
       }
     }
@@ -685,10 +799,18 @@ struct Consumer {
 
   // Sum of row i of the last row stage (its shared-memory accumulator), which
   // is cleared for the next stage.  Each row is read by exactly one thread.
-  __device__ float rowsum(int i) const {
-    const float v = s.part[i];
-    s.part[i] = 0.f;
-    return v;
+  __device__ float rowsum(int k, int i) const {
+    if (a.shape[k].nseg == 1) {
+      float *p = s.part + a.part_atomic_off + i;
+      const float v = *p;
+      *p = 0.f;
+      return v;
+    }
+    const float4 *q = reinterpret_cast<const float4 *>(s.part + i * kConsumerWarps);
+    float4 v = q[0];
+#pragma unroll
+    for (int j = 1; j < kConsumerWarps / 4; ++j) v = add4(v, q[j]);
+    return (v.x + v.y) + (v.z + v.w);
   }
 
   // ---- attention over the cache for one KV head group (split-KV)
@@ -1074,14 +1196,14 @@ struct Consumer {
   }
 
   // ---- LM head epilogue: logits and the CTA's share of the argmax
-  __device__ void lm_epilogue() {
+  __device__ void lm_epilogue(float sc) {
     const StageCta &c = s.misc->sc[ST_LM];
     // bidx starts at a row of this CTA so that the key always names a valid
     // token; a NaN logit never wins a comparison and raises DE_NONFINITE.
     float best = -INFINITY;
     int bidx = c.row0;
     for (int i = tid; i < c.nout; i += kNC) {
-      const float v = rowsum(i);
+      const float v = sc * rowsum(ST_LM, i);
       const int row = c.row0 + i;
       if (a.logits_out) a.logits_out[size_t(step) * a.vocab + row] = v;
       if (v != v) raise_error(a, DE_NONFINITE | (uint32_t(step & 0xffff) << 8));
@@ -1144,15 +1266,34 @@ struct Consumer {
         // ---------------- RMSNorm + q/k/v rows of the group
         // (every CTA's down contribution to the previous layer is in)
         if (gl > 0 && !gate(SY_S2, gl * nc, 0x10, 1)) goto done;
-        stage_norm([=](int j) { return xin4(j); }, a.gain_attn + size_t(l) * d, d, a.lane_width,
-                   a.xres + size_t(cur) * d, own_lo, own_hi);
-        gemv(ST_QKV, s.vbuf);
+        if (lanes) {
+          stage_norm([=](int j) { return xin4(j); }, a.gain_attn + size_t(l) * d, d, a.lane_width,
+                     a.xres + size_t(cur) * d, own_lo, own_hi);
+          gemv(ST_QKV, s.vbuf);
+        } else {
+          // the residual entering the layer: its owners keep their rows of it
+          RowInput in{};
+          if (l == 0) {
+            in.emb = a.embed + size_t(tok) * d;
+          } else {
+            in.g0 = a.xres + size_t(prev) * d;
+            in.g1 = a.acc_o + size_t(prev) * d;
+            in.g2 = a.acc_d + size_t(prev) * d;
+          }
+          in.gain = a.gain_attn + size_t(l) * d;
+          for (int r = own_lo + tid; r < own_hi; r += kNC)
+            a.xres[size_t(cur) * d + r] =
+                l == 0 ? Store<T>::to_f(in.emb[r])
+                       : __ldcg(in.g0 + r) + __ldcg(in.g1 + r) + __ldcg(in.g2 + r);
+          gemv_rows(ST_QKV, in);
+        }
         if (aborted()) goto done;
         {
           const StageCta &c = s.misc->sc[ST_QKV];
+          const float sc = lanes ? 1.f : fused_scale(d);
           for (int bi = 0; bi < c.nblk; ++bi) {
             const Block b = s.misc->blk[c.blk_begin + bi];
-            for (int i = tid; i < b.nrows; i += kNC) a.qkv[b.out_off + i] = rowsum(b.lrow0 + i);
+            for (int i = tid; i < b.nrows; i += kNC) a.qkv[b.out_off + i] = sc * rowsum(ST_QKV, b.lrow0 + i);
           }
         }
         if (!(a.skip_signal_cta == cta && step == 0 && l == 0)) signal(SY_QG0 + g);
@@ -1166,7 +1307,7 @@ struct Consumer {
           if (aborted()) goto done;
           const StageCta &c = s.misc->sc[ST_MIX];
           float *dst = a.dsum + size_t((l - 1) % delta) * d;
-          for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(i);
+          for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(ST_MIX, i);
         }
         // ---------------- attention of the group, merged in every group CTA
         if (!gate(SY_QG0 + g, (gl + 1) * ng, 0x20, 4)) goto done;
@@ -1185,18 +1326,25 @@ struct Consumer {
             a.acc_o[size_t(prev) * d + r] = 0.f;
             a.acc_d[size_t(prev) * d + r] = 0.f;
           }
-        {
+        if (lanes) {
           const float4 *xr = vec4(a.xres, cur), *ao = vec4(a.acc_o, cur);
           stage_norm([=](int j) { return add4(__ldcg(xr + j), __ldcg(ao + j)); },
                      a.gain_ffn + size_t(l) * d, d, a.lane_width);
+          gemv(ST_GU, s.vbuf);
+        } else {
+          RowInput in{};
+          in.g0 = a.xres + size_t(cur) * d;
+          in.g1 = a.acc_o + size_t(cur) * d;
+          in.gain = a.gain_ffn + size_t(l) * d;
+          gemv_rows(ST_GU, in);
         }
-        gemv(ST_GU, s.vbuf);
         if (aborted()) goto done;
         {
           const StageCta &c = s.misc->sc[ST_GU];
+          const float sc = lanes ? 1.f : fused_scale(d);
           float *h = s.svec + kSvecO;
           for (int i = tid; i < c.nout; i += kNC) {
-            const float gt = rowsum(i), up = rowsum(c.nout + i);
+            const float gt = sc * rowsum(ST_GU, i), up = sc * rowsum(ST_GU, c.nout + i);
             h[i] = gt / (1.f + expf(-gt)) * up;
           }
           cbar();
@@ -1221,25 +1369,31 @@ struct Consumer {
           if (aborted()) goto done;
           const StageCta &c = s.misc->sc[ST_MIX];
           float *dst = a.dsum + size_t((L - 1) % delta) * d;
-          for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(i);
+          for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(ST_MIX, i);
           signal(SY_MIXF);
           if (!gate(SY_MIXF, lm_count * nc, 0x70, 2)) goto done;
         }
-        {
+        if (lanes) {
           const float4 *xr = vec4(a.xres, last), *ao = vec4(a.acc_o, last), *ad = vec4(a.acc_d, last);
           stage_norm(
               [=](int j) {
                 float4 v = add4(add4(__ldcg(xr + j), __ldcg(ao + j)), __ldcg(ad + j));
-                if (lanes)
-                  for (int li = (L > delta ? L - delta : 0); li < L; ++li)
-                    v = add4(v, __ldcg(reinterpret_cast<const float4 *>(a.dsum + size_t(li % delta) * d) + j));
+                for (int li = (L > delta ? L - delta : 0); li < L; ++li)
+                  v = add4(v, __ldcg(reinterpret_cast<const float4 *>(a.dsum + size_t(li % delta) * d) + j));
                 return v;
               },
               a.gain_final, d, d);
+          gemv(ST_LM, s.vbuf);
+        } else {
+          RowInput in{};
+          in.g0 = a.xres + size_t(last) * d;
+          in.g1 = a.acc_o + size_t(last) * d;
+          in.g2 = a.acc_d + size_t(last) * d;
+          in.gain = a.gain_final;
+          gemv_rows(ST_LM, in);
         }
-        gemv(ST_LM, s.vbuf);
         if (aborted()) goto done;
-        lm_epilogue();
+        lm_epilogue(lanes ? 1.f : fused_scale(d));
         signal(SY_TOK);
         if (!gate(SY_TOK, lm_count * nc, 0x80, 3)) goto done;
         const unsigned long long key = __ldcg(a.keys + step);

@@ -96,8 +96,10 @@ def test_tiny_free_run_teacher_forced_and_cache():
 
 
 def test_tiny_is_repeatable():
-    """Two launches agree to float rounding.  The split projections are summed
-    with atomics, so the summation order (and the last bits) may differ."""
+    """Two launches agree to float rounding.  The O and down projections are
+    summed over SMs with fp32 atomics, so the summation order (and the last
+    bits) differ from run to run; the bound, 5e-5 relative, is a twentieth of
+    the logits tolerance against the oracle."""
     w = synth.WORKLOADS[0]
     m = w.model
     bits = synth.generate_weights(m, w.weight_seed)
@@ -111,7 +113,7 @@ def test_tiny_is_repeatable():
         dec.kie_destroy()
     a, b = runs[0].astype(np.float64), runs[1].astype(np.float64)
     rel = np.linalg.norm(a - b, axis=1) / np.linalg.norm(a, axis=1)
-    assert rel.max() < 1e-5, rel.max()
+    assert rel.max() < 5e-5, rel.max()
 
 
 @pytest.mark.parametrize("shape", ["tiny", "lanes2_d2"])
