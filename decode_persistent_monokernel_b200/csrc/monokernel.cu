@@ -1281,10 +1281,6 @@ struct Consumer {
             in.g2 = a.acc_d + size_t(prev) * d;
           }
           in.gain = a.gain_attn + size_t(l) * d;
-          for (int r = own_lo + tid; r < own_hi; r += kNC)
-            a.xres[size_t(cur) * d + r] =
-                l == 0 ? Store<T>::to_f(in.emb[r])
-                       : __ldcg(in.g0 + r) + __ldcg(in.g1 + r) + __ldcg(in.g2 + r);
           gemv_rows(ST_QKV, in);
         }
         if (aborted()) goto done;
@@ -1309,6 +1305,16 @@ struct Consumer {
           float *dst = a.dsum + size_t((l - 1) % delta) * d;
           for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(ST_MIX, i);
         }
+        // the residual entering the layer: its owners keep their rows of it (read
+        // by every SM only after the grid-wide wait that follows O); warp 1 does
+        // it while thread 0 waits for the group's q/k/v
+        if (!lanes && warp == 1)
+          for (int r = own_lo + lane; r < own_hi; r += 32) {
+            const size_t pr = size_t(prev) * d + r;
+            a.xres[size_t(cur) * d + r] =
+                l == 0 ? Store<T>::to_f(a.embed[size_t(tok) * d + r])
+                       : __ldcg(a.xres + pr) + __ldcg(a.acc_o + pr) + __ldcg(a.acc_d + pr);
+          }
         // ---------------- attention of the group, merged in every group CTA
         if (!gate(SY_QG0 + g, (gl + 1) * ng, 0x20, 4)) goto done;
         attention();
