@@ -57,8 +57,10 @@ typedef enum { KIE_F16 = 0, KIE_BF16 = 1 } kie_dtype;
  * Lane models: every per-lane size is the total divided by n_lanes
  * (lane width d_model/n_lanes, n_heads/n_lanes query heads, n_kv_heads/n_lanes
  * KV heads, ffn_dim/n_lanes hidden units), lane_delay >= 2.
- * Requirements: n_heads % n_kv_heads == 0; head_dim in {64, 128};
- * d_model, ffn_dim (per lane) multiples of 8. */
+ * Requirements: n_heads % n_kv_heads == 0 with at most 4 query heads per KV
+ * head; head_dim in {64, 128}; d_model <= 4096; lane width a multiple of
+ * 128; ffn_dim per lane a multiple of 8.  kie_create returns KIE_ERR_INVALID
+ * (reason via kie_strerror) for any other shape. */
 typedef struct {
   int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, ffn_dim, vocab;
   float rms_eps, rope_theta;
