@@ -318,3 +318,31 @@ def test_nonfinite_logits_stop_the_kernel():
         dec.kie_decode(1)
     assert e.value.code == kie.KIE_ERR_POISONED
     dec.kie_destroy()
+
+
+def test_watchdog_reports_a_missing_signal():
+    """Failure detection without a fault: one SM skips its q/k/v signal in the
+    first step of a launch, so its KV group's waits run out after the short
+    watchdog; the kernel returns KIE_ERR_DEVICE_TIMEOUT (every SM leaves its
+    bounded waits, producers drain their copies), the context is poisoned, and
+    the device stays usable for a new context."""
+    import decode_persistent_monokernel_b200 as kie
+    w = synth.WORKLOADS[0]
+    m = w.model
+    bits = synth.generate_weights(m, w.weight_seed)
+    prompt = synth.prompt(w)
+    dec = make_decoder(m, bits, 64)
+    dec.kie_prefill(prompt)
+    dec.kie_debug_set(200, 5)        # 200 ms limit; SM 5 never signals its group
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_decode(4)
+    assert e.value.code == kie.KIE_ERR_DEVICE_TIMEOUT
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_decode(1)
+    assert e.value.code == kie.KIE_ERR_POISONED
+    dec.kie_destroy()
+    dec = make_decoder(m, bits, 64)
+    t0 = dec.kie_prefill(prompt)
+    toks = dec.kie_decode(4)
+    assert 0 <= t0 < m.vocab and all(0 <= t < m.vocab for t in toks)
+    dec.kie_destroy()
