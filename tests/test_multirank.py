@@ -1,0 +1,63 @@
+"""The replica path of bench.py on CPU: two gloo ranks reduce their timings to
+the max over ranks, whole-job throughput counts every rank's tokens, and the
+reference arm runs on rank 0 only."""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_q):
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        ms, e2e, kms = bench.reduce_max_over_ranks([1.0 + rank, 10.0 * rank, 3.0], world, "cpu")
+        out_q.put((rank, ms, e2e, kms))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_max():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.SimpleQueue()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get() for _ in range(world))
+    for rank, ms, e2e, kms in got:
+        assert (ms, e2e, kms) == (2.0, 10.0, 3.0), rank
+
+
+def test_job_throughput_counts_every_replica():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.reduce_max_over_ranks([1.5, 2.5], 1, "cpu") == [1.5, 2.5]
+    assert bench.job_tokens_per_s(1, 512, 1000.0) == pytest.approx(512.0)
+    assert bench.job_tokens_per_s(4, 512, 1000.0) == pytest.approx(2048.0)
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, RANK="1", LOCAL_RANK="1", WORLD_SIZE="2")
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "3"], env=env, capture_output=True,
+                         text=True, timeout=600)
+    assert res.returncode == 0 and res.stdout.strip() == ""
