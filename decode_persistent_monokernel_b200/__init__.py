@@ -62,11 +62,19 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int32
 
 
-def load(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load libkie.so (built by ``build.py``); raises if it is not there."""
-    global _lib
+_lib_path = None
+
+
+def load(path: str = None) -> ctypes.CDLL:
+    """Load libkie.so (built by ``build.py``), or ``path`` (e.g. the profiling
+    build libkie_prof.so); raises if it is not there.  One library per process:
+    asking for a different one after the first load raises."""
+    global _lib, _lib_path
     if _lib is not None:
+        if path is not None and os.path.abspath(path) != _lib_path:
+            raise RuntimeError(f"{_lib_path} is already loaded; cannot switch to {path}")
         return _lib
+    path = LIB_PATH if path is None else path
     if not os.path.exists(path):
         raise RuntimeError(f"libkie.so not built: {path} is missing (run "
                            "decode_persistent_monokernel_b200/build.py)")
@@ -92,6 +100,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         f.argtypes = args
         f.restype = res
     _lib = L
+    _lib_path = os.path.abspath(path)
     return L
 
 
