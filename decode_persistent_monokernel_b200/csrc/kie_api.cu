@@ -267,6 +267,20 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
       sc.nlocal = (k == ST_GU) ? 2 * sc.nout : sc.nout;
       sc.ntiles = tile;
       sc.nblk = int(blk.size());
+      // a row stage whose blocks read one input slice and fill consecutive
+      // local rows is tiled as one run (fewer partial tiles and restarts)
+      if (!sh.cols && blk.size() > 1) {
+        bool m = true;
+        int n = 0;
+        for (const Block &B : blk) {
+          m = m && B.in_off == blk[0].in_off && B.lrow0 == blk[0].lrow0 + n;
+          n += B.nrows;
+        }
+        if (m && n == sc.nlocal && blk[0].lrow0 == 0) {
+          sc.merged = 1;
+          sc.ntiles = (n + sh.R - 1) / sh.R;
+        }
+      }
       int64_t bytes = 0;
       for (const Block &B : blk) bytes += int64_t(B.nrows) * sh.K * 2;
       sc.bytes = bytes;

@@ -75,9 +75,11 @@ constexpr int kTraceCap = 1 << 16;
 
 // Per-stage constants shared by every CTA.  A tile is R whole rows (at most
 // kSlotBytes).
-//  Row stages (QKV, GU, MIX, LM): out[row] = sum_k W[row][k] in[k].  All
-//    consumer warps share every tile: warp w takes row group w / nseg (rpw
-//    rows) and column split w % nseg (cps 8-element chunks of each row).
+//  Row stages (QKV, GU, MIX, LM): out[row] = sum_k W[row][k] in[k], R =
+//    16384 / K rows per tile.  All consumer warps share every tile: warp w
+//    takes columns [w K/16, (w+1) K/16) of every row, each lane 8 of them in
+//    four rows; nseg = 16 keeps one partial sum per (row, warp), nseg = 1 one
+//    shared-memory atomic sum per row.
 //  Column stages (O, D): out[:] += sum_row s[row] W[row][:], where a row is
 //    a column of the canonical matrix.  Thread t takes row phase t / ngrp
 //    and 4-element output groups t % ngrp + ngrp * j (j < cps); nseg phases.
@@ -86,9 +88,8 @@ struct StageShape {
   int32_t R;       // rows per tile (power of two)
   int32_t nseg;    // row stages: partial sums kept per row (16: one per consumer warp,
                    // 1: a shared-memory atomic sum); column stages: row phases
-  int32_t rpw;     // row stages: rows per warp (1 unless R > 16)
-  int32_t cps;     // row stages: 8-element chunks per (row, split);
-                   // column stages: 4-element output groups per thread
+  int32_t rpw;     // 1 (kept for the plan checker)
+  int32_t cps;     // column stages: 4-element output groups per thread (row stages: 1)
   int32_t in_len;  // length of the stage input vector
   int32_t out_len; // length of the stage output vector
   int32_t cols;    // 1 for column stages
@@ -102,6 +103,9 @@ struct StageCta {
   int32_t blk_begin;  // first block, counted from the CTA's own first block
   int32_t nblk;
   int64_t bytes;      // stream bytes of one instance of this stage
+  int32_t merged;     // 1: a row stage whose blocks share one input slice and fill
+                      // local rows 0..nlocal-1 in order, tiled as one run of nlocal rows
+  int32_t pad;
 };
 
 // A run of rows of one CTA's stage with one input slice and one output place.

@@ -299,8 +299,8 @@ struct Producer {
     const int R = a.shape[k].R;
     const uint32_t rowb = uint32_t(a.shape[k].K) * 2u;
     const uint32_t NS = a.ring_slots;
-    for (int bi = 0; bi < nblk; ++bi) {
-      const int nrows = s.misc->blk[b0 + bi].nrows;
+    for (int bi = 0; bi < (c.merged ? 1 : nblk); ++bi) {
+      const int nrows = c.merged ? c.nlocal : s.misc->blk[b0 + bi].nrows;
       for (int r0 = 0; r0 < nrows; r0 += R) {
         if (T >= NS) {
 #ifdef KIE_PROFILE
@@ -745,8 +745,9 @@ struct Consumer {
     bool ok = !aborted();
     Inputs8 xf{};
     if (!in.v) xf = fused_inputs(in, col0, LSH);   // every block reads the whole vector
-    for (int bi = 0; bi < c.nblk && ok; ++bi) {
-      const Block b = s.misc->blk[c.blk_begin + bi];
+    for (int bi = 0; bi < (c.merged ? 1 : c.nblk) && ok; ++bi) {
+      Block b = s.misc->blk[c.blk_begin + bi];
+      if (c.merged) b.nrows = c.nlocal;        // one run over all the stage's rows
       if (b.nrows == 0) continue;
       const Inputs8 x = in.v ? row_inputs(in.v, b.in_off, col0) : xf;
       const int n = (b.nrows + R - 1) / R;     // tiles of the block; the last may be partial

@@ -21,6 +21,11 @@ static void check(kie_model_desc m, int n_ctas, const char *name) {
   printf("%s: ctas %d slots %d smem %zu vbuf %d part %d stream %.3f GB jobs %zu blocks %zu\n", name, n_ctas,
          P.ring_slots, P.smem, P.vbuf_floats, P.part_floats, P.stream_bytes / 1e9, P.jobs.size(), P.blocks.size());
   REQ(P.smem <= 232448, "smem");
+  {
+    int merged = 0;
+    for (const StageCta &sc : P.stage_cta) merged += sc.merged;
+    printf("  merged row-stage instances: %d\n", merged);
+  }
   for (int k = 0; k < ST_COUNT; ++k)
     printf("  stage %d: K %d R %d nseg %d rpw %d cps %d cols %d\n", k, P.shape[k].K, P.shape[k].R,
            P.shape[k].nseg, P.shape[k].rpw, P.shape[k].cps, P.shape[k].cols);
@@ -74,8 +79,26 @@ static void check(kie_model_desc m, int n_ctas, const char *name) {
         const StageShape &sh = P.shape[k];
         std::vector<int64_t> tstart;
         int t = 0;
-        for (int bi = 0; bi < sc.nblk; ++bi) {
-          const Block &b = P.blocks[P.cta_blk_begin[c] + sc.blk_begin + bi];
+        // the runs the producer and the consumers tile: one per block, or one
+        // over all the stage's rows when the plan merged them
+        std::vector<Block> runs;
+        if (sc.merged) {
+          REQ(!sh.cols && sc.nblk > 1, "merged stage");
+          int n = 0;
+          for (int bi = 0; bi < sc.nblk; ++bi) {
+            const Block &b = P.blocks[P.cta_blk_begin[c] + sc.blk_begin + bi];
+            REQ(b.lrow0 == n && b.in_off == P.blocks[P.cta_blk_begin[c] + sc.blk_begin].in_off, "merge");
+            n += b.nrows;
+          }
+          REQ(n == sc.nlocal, "merged rows");
+          Block run = P.blocks[P.cta_blk_begin[c] + sc.blk_begin];
+          run.nrows = n;
+          run.tile0 = 0;
+          runs.push_back(run);
+        } else {
+          for (int bi = 0; bi < sc.nblk; ++bi) runs.push_back(P.blocks[P.cta_blk_begin[c] + sc.blk_begin + bi]);
+        }
+        for (const Block &b : runs) {
           REQ(b.tile0 == t, "tile0");
           for (int r0 = 0; r0 < b.nrows; r0 += sh.R) {
             const int rows = std::min(sh.R, b.nrows - r0);
@@ -97,8 +120,7 @@ static void check(kie_model_desc m, int n_ctas, const char *name) {
           // partial sum of every (local row, warp); every (row, column chunk) read once
           std::vector<double> rowpart(size_t(std::max(1, sc.nlocal)) * kConsumerWarps, 0.0);
           std::vector<int> chunk_hit(size_t(std::max(1, sc.nlocal)) * (sh.K / 8), 0);
-          for (int bi = 0; bi < sc.nblk; ++bi) {
-            const Block &b = P.blocks[P.cta_blk_begin[c] + sc.blk_begin + bi];
+          for (const Block &b : runs) {
             const int ntile = (b.nrows + sh.R - 1) / sh.R;
             for (int t = 0; t < ntile; ++t) {
               const int rows = std::min(sh.R, b.nrows - t * sh.R);
