@@ -97,3 +97,12 @@ def test_null_context_calls_rejected(lib):
     assert "watchdog" in kie.strerror(kie.KIE_ERR_DEVICE_TIMEOUT)
     assert "non-finite" in kie.strerror(kie.KIE_ERR_NONFINITE)
     assert lib.kie_set_sync_mode(None, kie.KIE_SYNC_GRID) == kie.KIE_ERR_INVALID
+
+
+def test_binding_loads_one_library_per_process(lib):
+    # the library is already loaded by the fixture: asking again returns it,
+    # asking for another one raises instead of silently reusing the first
+    assert kie.load() is lib
+    assert kie.load(kie.LIB_PATH) is lib
+    with pytest.raises(RuntimeError):
+        kie.load(kie.PROF_LIB_PATH)
