@@ -219,36 +219,63 @@ def test_long_context_two_layers(dense_2b):
     print(f"long-2L: rel-L2 {rel:.3g} max-abs {mab:.3g} near ties {near}")
 
 
-def test_long_context_full_model_properties(dense_2b):
-    """The full long-context workload: 8192-token prefill then 256 greedy steps.
-    Layer 0's cached K/V depend only on each token and its position, so the
-    oracle checks them at every position; the rest must be finite and the
-    cache must be written exactly up to the current position."""
-    w = synth.WORKLOADS[3]
-    m = w.model
-    prompt = synth.prompt(w)
-    P, N = w.prompt_len, w.decode_len
-    max_seq = P + N + 16
-    dec = make_decoder(m, dense_2b, max_seq)
-    t0 = dec.kie_prefill(prompt)
-    toks = dec.kie_decode(N)
-    assert 0 <= t0 < m.vocab and ((toks >= 0) & (toks < m.vocab)).all()
-    seq = np.concatenate([prompt, [t0], toks[:-1]])
-    m1, b1 = _first_layers(m, dense_2b, 1)
+def _check_layer0_kv_and_bounds(dec, m, bits, seq, max_seq):
+    """Layer 0's cached K/V depend only on each token and its position, so the
+    oracle (the model cut to its first layer) checks them at every position of
+    ``seq``; at every layer the cache is written exactly up to len(seq) and
+    finite there."""
+    L = len(seq)
+    m1, b1 = _first_layers(m, bits, 1)
     orc = Oracle(m1, b1, max_seq)
     orc.forward(list(seq), logits="none")
     for g in range(m.n_kv_heads):
         k, v = dec.kie_copy_kv(0, g, 0, max_seq)
         kf, vf = storage_to_f64(k, m.dtype), storage_to_f64(v, m.dtype)
-        L = P + N
         assert np.isnan(kf[L:]).all() and np.isnan(vf[L:]).all()
         for got, want in ((kf[:L], orc.K[0, g, :L]), (vf[:L], orc.V[0, g, :L])):
-            assert np.abs(got - want).max() <= 4e-3 * np.abs(want).max()
+            assert np.abs(got - want).max() <= 4e-3 * np.abs(want).max(), g
     for l in (1, m.n_layers // 2, m.n_layers - 1):
-        k, v = dec.kie_copy_kv(l, 3, 0, max_seq)
-        assert np.isfinite(storage_to_f64(k[:P + N], m.dtype)).all()
-        assert np.isnan(storage_to_f64(k[P + N:], m.dtype)).all()
+        for g in (0, m.n_kv_heads - 1):
+            k, v = dec.kie_copy_kv(l, g, 0, max_seq)
+            for c in (storage_to_f64(k, m.dtype), storage_to_f64(v, m.dtype)):
+                assert np.isfinite(c[:L]).all() and np.isnan(c[L:]).all(), (l, g)
+
+
+def _greedy_full_model(m, bits, w):
+    """Prefill the workload's prompt, then its greedy decode steps in one
+    launch with the logits kept.  Every fed-back token must be the lowest index
+    of the largest logit the kernel wrote for its step (bit-exact: the same
+    fp32 values decide both), and the cache must hold the oracle's layer-0 K/V
+    for the prompt followed by exactly the tokens the kernel reported."""
+    prompt = synth.prompt(w)
+    P, N = w.prompt_len, w.decode_len
+    max_seq = P + N + 16
+    dec = make_decoder(m, bits, max_seq)
+    t0 = dec.kie_prefill(prompt)
+    toks, z = _gpu_logits(dec, N, m.vocab, None)
+    assert 0 <= t0 < m.vocab and ((toks >= 0) & (toks < m.vocab)).all()
+    assert np.isfinite(z).all()
+    assert (toks == np.argmax(z, axis=1)).all()
+    seq = np.concatenate([prompt, [t0], toks[:-1]])
+    _check_layer0_kv_and_bounds(dec, m, bits, seq, max_seq)
     dec.kie_destroy()
+
+
+def test_long_context_full_model_properties(dense_2b):
+    """The full long-context workload: 8192-token prefill then 256 greedy steps
+    in one launch, checked through the properties that hold at any size."""
+    w = synth.WORKLOADS[3]
+    _greedy_full_model(w.model, dense_2b, w)
+
+
+def test_8b_class_full_model_properties():
+    """The full 8B-class workload as it is benchmarked (bf16, 32 layers,
+    V 128256; 1024-token prefill then 256 greedy steps in one launch), checked
+    through the same properties; its logits are compared with the oracle's on
+    the first two layers by the test above."""
+    w = synth.WORKLOADS[4]
+    bits = synth.generate_weights(w.model, w.weight_seed)
+    _greedy_full_model(w.model, bits, w)
 
 
 def test_8b_class_two_layers():
