@@ -98,16 +98,20 @@ def kernel_sources_digest(files):
     return h.hexdigest()
 
 
-def dram_traffic(algorithmic_bytes):
+def dram_traffic(algorithmic_bytes, workload):
     """DRAM bytes of the timed launch, from the last hardware-counter capture of
     the decode kernel: that capture's DRAM bytes / algorithmic bytes, times this
     launch's algorithmic bytes (the traffic scales with the bytes streamed).
-    None when there is no capture or the kernel sources changed since."""
+    None when there is no capture, the capture ran another workload's model
+    (other stage shapes, another K/V share), or the kernel sources changed
+    since."""
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
         if kernel_sources_digest(rec["files"]) != rec["kernel_sources_sha256"]:
             return None, "kernel changed since the last counter capture"
+        if int(rec["workload"]) != workload:
+            return None, f"the counter capture covers workload {rec['workload']}'s layer shapes only"
         return rec["ratio"] * algorithmic_bytes, rec["capture"]
     except (OSError, KeyError, ValueError):
         return None, "no counter capture recorded"
@@ -315,7 +319,7 @@ def main():
 
     total_bytes = workload_bytes(m, P, K, st.weight_bytes_per_step, st.kv_bytes_per_position)
     peak, peak_kind = peak_hbm()
-    traffic, traffic_src = dram_traffic(total_bytes)
+    traffic, traffic_src = dram_traffic(total_bytes, args.workload)
     achieved = total_bytes / (kernel_ms * 1e-3) / 1e9
     value = job_tokens_per_s(world, K, ms)
     line = {

@@ -56,6 +56,7 @@ def record_traffic(report, args):
     data = {"files": KERNEL_FILES, "kernel_sources_sha256": bench.kernel_sources_digest(KERNEL_FILES),
             "capture": f"ncu --set full of profile_case --workload {args.workload} --layers "
                        f"{args.layers} --steps {args.steps}; traffic scaled by algorithmic bytes",
+            "workload": args.workload,
             "dram_bytes": dram, "algorithmic_bytes": alg, "ratio": dram / alg,
             "gpu_time_ns": float(rec["gpu__time_duration.sum"])}
     with open(os.path.join(root, "profiles", "monokernel_traffic.json"), "w") as f:

@@ -61,3 +61,20 @@ def test_reference_arm_runs_on_rank_zero_only():
                           "--steps", "1", "--warmup", "3"], env=env, capture_output=True,
                          text=True, timeout=600)
     assert res.returncode == 0 and res.stdout.strip() == ""
+
+
+def test_traffic_is_scaled_only_for_the_captured_kernel_and_workload():
+    sys.path.insert(0, ROOT)
+    import bench
+    import json
+    with open(bench.TRAFFIC_FILE) as f:
+        rec = json.load(f)
+    current = bench.kernel_sources_digest(rec["files"]) == rec["kernel_sources_sha256"]
+    t, src = bench.dram_traffic(1e9, int(rec["workload"]))
+    if current:
+        assert t == pytest.approx(rec["ratio"] * 1e9) and src == rec["capture"]
+    else:
+        assert t is None and "kernel changed" in src
+    other = (int(rec["workload"]) + 1) % 5
+    t, src = bench.dram_traffic(1e9, other)
+    assert t is None
