@@ -89,13 +89,17 @@ int kie_create(const kie_model_desc *desc, const void *weights, void *stream, ki
 /* Process a prompt from position 0 (the KV cache is reset and its unused
  * slots filled with NaN) and return the greedy next token, the argmax of the
  * logits at position n-1.
- *   tokens: HOST array of n ids in [0, vocab); next_token: HOST out. */
+ *   tokens: HOST array of n ids in [0, vocab); next_token: HOST out.
+ *   n < 1 or an id outside [0, vocab) returns KIE_ERR_INVALID before any
+ *   device work (the cache and position are left as they were). */
 int kie_prefill(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_token);
 
 /* Greedy decode: step k feeds the pending token at position pos+k, appends
  * its K/V, and the argmax of its logits becomes out_tokens[k] and the next
  * pending token.  The first pending token is kie_prefill's next_token.
- *   out_tokens: HOST array of n_steps. */
+ *   out_tokens: HOST array of n_steps.
+ *   n_steps < 1, or no pending token (no kie_prefill yet), returns
+ *   KIE_ERR_INVALID before any device work. */
 int kie_decode(kie_ctx *ctx, int32_t n_steps, int32_t *out_tokens);
 
 /* kie_decode with options:

@@ -316,8 +316,14 @@ def test_errors_and_capacity():
     with pytest.raises(kie.KieError) as e:
         dec.kie_prefill(np.zeros(21, dtype=np.int32))
     assert e.value.code == kie.KIE_ERR_CAPACITY
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_prefill(np.zeros(0, dtype=np.int32))   # empty prompt
+    assert e.value.code == kie.KIE_ERR_INVALID
     dec.kie_prefill(np.arange(15, dtype=np.int32))
-    dec.kie_decode(5)
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_decode(0)                          # no steps
+    assert e.value.code == kie.KIE_ERR_INVALID
+    dec.kie_decode(5)                              # fills the cache to max_seq exactly
     with pytest.raises(kie.KieError) as e:
         dec.kie_decode(1)
     assert e.value.code == kie.KIE_ERR_CAPACITY
