@@ -114,7 +114,9 @@ const char *make_shape(int K, int in_len, int out_len, StageShape &s) {
   // lane 8 of those, so K/128 lanes share a row: one 16-byte load per lane
   // covers 4096/K rows, and four of them cover R = 16384/K rows, one 32 KB
   // tile.
-  if (K % 128 || K < 128 || K > 4096) return "row length must be a multiple of 128, at most 4096";
+  // (K / 128 lanes share a row, so it must be a power of two)
+  if (K % 128 || K < 128 || K > 4096 || ((K >> 7) & ((K >> 7) - 1)))
+    return "row length must be 128 times a power of two, at most 4096";
   s.R = 16384 / K;
   s.nseg = 1;    // one (shared-memory atomic) sum per row
   s.rpw = 1;
@@ -436,6 +438,11 @@ static const char *validate(const kie_model_desc *m) {
   if ((m->d_model / nl) % 8 || (m->ffn_dim / nl) % 8) return "lane width and lane ffn must be multiples of 8";
   if ((m->d_model / nl) % 128) return "lane width (d_model / n_lanes) must be a multiple of 128";
   if (m->d_model > 4096) return "d_model above 4096 is not supported";
+  // rows of d_model (lane mix, LM head) and of the lane width are split over
+  // K / 128 lanes of a warp, a power of two
+  const int w128 = m->d_model / nl / 128, d128 = m->d_model / 128;
+  if ((w128 & (w128 - 1)) || (d128 & (d128 - 1)))
+    return "lane width and d_model must be 128 times a power of two";
   if (nl > 1 && m->lane_delay < 2) return "lane_delay must be >= 2";
   if (nl > 64) return "at most 64 lanes";
   if (!(m->rms_eps >= 0.f) || !(m->rope_theta > 0.f)) return "bad rms_eps or rope_theta";

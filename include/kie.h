@@ -58,8 +58,9 @@ typedef enum { KIE_F16 = 0, KIE_BF16 = 1 } kie_dtype;
  * (lane width d_model/n_lanes, n_heads/n_lanes query heads, n_kv_heads/n_lanes
  * KV heads, ffn_dim/n_lanes hidden units), lane_delay >= 2.
  * Requirements: n_heads % n_kv_heads == 0 with at most 4 query heads per KV
- * head; head_dim in {64, 128}; d_model <= 4096; lane width a multiple of
- * 128; ffn_dim per lane a multiple of 8.  kie_create returns KIE_ERR_INVALID
+ * head; head_dim in {64, 128}; d_model <= 4096; lane width and d_model
+ * 128 times a power of two (so n_lanes is a power of two); ffn_dim per lane
+ * a multiple of 8.  kie_create returns KIE_ERR_INVALID
  * (reason via kie_strerror) for any other shape. */
 typedef struct {
   int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, ffn_dim, vocab;

@@ -72,6 +72,10 @@ def _desc(**kw):
     dict(ffn_dim=700),                   # not a multiple of 8
     dict(max_seq=0),
     dict(n_heads=8, n_kv_heads=1, d_model=512),  # more than 4 q heads per kv head
+    # rows shared by K/128 lanes of a warp: 128 x a power of two only
+    dict(n_heads=6, n_kv_heads=6, head_dim=128, d_model=768),
+    dict(n_heads=24, n_kv_heads=8, head_dim=128, d_model=3072, ffn_dim=8192),
+    dict(n_lanes=3, lane_delay=2, n_heads=6, n_kv_heads=3, d_model=384, ffn_dim=768),
 ])
 def test_invalid_descriptors_rejected(lib, bad):
     h = ctypes.c_void_p()
