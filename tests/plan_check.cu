@@ -313,6 +313,20 @@ int main() {
     printf("%s: %s slots %d smem %zu stream %.3f GB wbytes %lld\n", nm, why ? why : "ok", P.ring_slots, P.smem,
            P.stream_bytes / 1e9, (long long)P.weight_bytes_per_step);
   }
+  // row lengths: K / 128 lanes share a row, so only 128 x a power of two
+  for (int K = 128; K <= 4096; K += 128) {
+    StageShape sh;
+    const bool pow2 = ((K >> 7) & ((K >> 7) - 1)) == 0;
+    REQ((make_shape(K, K, K, sh) == nullptr) == pow2, "make_shape K=%d", K);
+    if (pow2) REQ(sh.R * K == 16384, "tile rows K=%d", K);
+  }
+  {
+    // a 3-lane model with 128-wide lanes: its d_model rows (mix, LM head)
+    // have K = 384, which the plan must refuse
+    Plan P;
+    kie_model_desc m3{2, 384, 6, 3, 64, 768, 4096, 1e-5f, 1e4f, 0, 3, 2, 64};
+    REQ(build_plan(m3, 148, 232448, P) != nullptr, "3-lane d_model 384 accepted");
+  }
   printf(fails ? "FAILED (%d)\n" : "ALL OK\n", fails);
   return fails != 0;
 }
