@@ -91,6 +91,7 @@ def load(path: str = None) -> ctypes.CDLL:
         "kie_copy_kv": ([_P, _I, _I, _I, _I, _P, _P], _I),
         "kie_debug_set": ([_P, _I, _I], _I),
         "kie_set_sync_mode": ([_P, _I], _I),
+        "kie_set_max_steps_per_launch": ([_P, _I], _I),
         "kie_trace_request": ([_P, _I, _I], _I),
         "kie_get_trace": ([_P, _P, _I], _I),
         "kie_get_profile": ([_P, _P, _I], _I),
@@ -215,6 +216,9 @@ class Decoder:
 
     def kie_set_sync_mode(self, mode: int) -> None:
         _check(load().kie_set_sync_mode(self._h, mode))
+
+    def kie_set_max_steps_per_launch(self, n: int) -> None:
+        _check(load().kie_set_max_steps_per_launch(self._h, n))
 
     def kie_destroy(self) -> None:
         if self._h:

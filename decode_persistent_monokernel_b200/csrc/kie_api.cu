@@ -393,6 +393,7 @@ struct kie_ctx {
   uint64_t watchdog_ns = 2000000000ull;
   int skip_signal_cta = -1;
   int grid_sync = 0;
+  int max_launch_steps = 0;   // 0: the counters' own limit (steps_per_launch)
   float last_ms = 0.f;
   int last_steps = 0;
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
@@ -661,6 +662,68 @@ static int device_error(kie_ctx *ctx, uint32_t status) {
   return rc;
 }
 
+// The epoch counters are 32-bit, and every CTA adds to them at most 4 L + 2
+// times per step: the q/k/v, attention, O and down signals of each layer, and
+// the lane-mix flush and token of each step.  One launch therefore runs at
+// most this many steps, so that no counter passes 2^31; a longer call runs as
+// several launches back to back.
+static int steps_per_launch(const kie_ctx *ctx) {
+  const int64_t per_step = (4 * int64_t(ctx->m.n_layers) + 2) * ctx->plan.n_ctas;
+  int64_t n = ((int64_t(1) << 31) - 1) / per_step;
+  if (ctx->max_launch_steps > 0 && ctx->max_launch_steps < n) n = ctx->max_launch_steps;
+  return int(std::max<int64_t>(n, 1));
+}
+
+// Runs the n steps described by `a` (forced tokens, output tokens, argmax
+// keys and logits of the whole call) as one or more launches.  Each launch
+// takes the next run of steps and starts from the previous launch's last
+// token.  The counters, both layer accumulators and the launch's keys are
+// cleared before each launch.  The output tokens end in host_out.  The
+// context's device time spans from the first launch's start to the last
+// one's end.
+static int launch_steps(kie_ctx *ctx, const KernelArgs &a, size_t sync_bytes, int n,
+                        int32_t *host_out) {
+  cudaStream_t st = ctx->stream;
+  const int cap = steps_per_launch(ctx);
+  int32_t tok = a.first_token;
+  uint32_t status = 0;
+  for (int s0 = 0; s0 < n; s0 += cap) {
+    const int c = std::min(cap, n - s0);
+    KernelArgs b = a;
+    b.pos0 = a.pos0 + s0;
+    b.n_steps = c;
+    b.first_token = tok;
+    b.forced = a.forced ? a.forced + s0 : nullptr;
+    b.out_tokens = a.out_tokens + s0;
+    b.keys = a.keys + s0;
+    b.logits_out = a.logits_out ? a.logits_out + size_t(s0) * ctx->m.vocab : nullptr;
+    b.skip_signal_cta = s0 == 0 ? a.skip_signal_cta : -1;
+    if (a.trace && a.trace_step >= s0 && a.trace_step < s0 + c) b.trace_step = a.trace_step - s0;
+    else b.trace = nullptr;
+    CK(cudaMemsetAsync(a.sync, 0, sync_bytes, st));
+    CK(cudaMemsetAsync(a.acc_o, 0, size_t(4) * ctx->m.d_model * 4, st));   // both accumulators, both parities
+    CK(cudaMemsetAsync(b.keys, 0, size_t(c) * 8, st));
+    if (s0 == 0) CK(cudaEventRecord(ctx->ev0, st));
+    void *args[] = {&b};
+    CK(cudaLaunchCooperativeKernel(monokernel_fn(ctx->m.dtype), dim3(ctx->plan.n_ctas),
+                                   dim3(monokernel_threads()), args, ctx->plan.smem, st));
+    if (s0 + c < n) {   // the next launch needs this one's last token
+      CK(cudaMemcpyAsync(&status, a.sync + SY_STATUS * kSyncStride, 4, cudaMemcpyDeviceToHost, st));
+      CK(cudaMemcpyAsync(&tok, b.out_tokens + c - 1, 4, cudaMemcpyDeviceToHost, st));
+      CK(cudaStreamSynchronize(st));
+      if (status != 0) return device_error(ctx, status);
+    }
+  }
+  CK(cudaEventRecord(ctx->ev1, st));
+  CK(cudaMemcpyAsync(&status, a.sync + SY_STATUS * kSyncStride, 4, cudaMemcpyDeviceToHost, st));
+  CK(cudaMemcpyAsync(host_out, a.out_tokens, size_t(n) * 4, cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  CK(cudaEventElapsedTime(&ctx->last_ms, ctx->ev0, ctx->ev1));
+  ctx->last_steps = n;
+  if (status != 0) return device_error(ctx, status);
+  return KIE_OK;
+}
+
 static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int first_token,
                bool logits_every_step, float *logits_out, int32_t *out_host) {
   const kie_model_desc &m = ctx->m;
@@ -707,25 +770,11 @@ static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int fi
     CK(cudaMemsetAsync(ctx->trace, 0, 8, st));
   }
 
-  const size_t sync_words = size_t(SY_QG0 + 2 * m.n_kv_heads) * kSyncStride;
+  const size_t sync_bytes = size_t(SY_QG0 + 2 * m.n_kv_heads) * kSyncStride * 4;
   if (forced_host)
     CK(cudaMemcpyAsync(ctx->tokens_in, forced_host, size_t(n) * 4, cudaMemcpyHostToDevice, st));
-  CK(cudaMemsetAsync(ctx->sync, 0, sync_words * 4, st));
-  CK(cudaMemsetAsync(a.acc_o, 0, size_t(4) * m.d_model * 4, st));   // both accumulators, both parities
-  CK(cudaMemsetAsync(ctx->keys, 0, size_t(n) * 8, st));
-  void *args[] = {&a};
-  CK(cudaEventRecord(ctx->ev0, st));
-  CK(cudaLaunchCooperativeKernel(monokernel_fn(m.dtype), dim3(P.n_ctas), dim3(monokernel_threads()),
-                                 args, P.smem, st));
-  CK(cudaEventRecord(ctx->ev1, st));
-  uint32_t status = 0;
-  CK(cudaMemcpyAsync(&status, ctx->sync + SY_STATUS * kSyncStride, 4, cudaMemcpyDeviceToHost, st));
   ctx->host_tokens.resize(n);
-  CK(cudaMemcpyAsync(ctx->host_tokens.data(), ctx->tokens_out, size_t(n) * 4, cudaMemcpyDeviceToHost, st));
-  CK(cudaStreamSynchronize(st));
-  CK(cudaEventElapsedTime(&ctx->last_ms, ctx->ev0, ctx->ev1));
-  ctx->last_steps = n;
-  if (status != 0) return device_error(ctx, status);
+  if (int rc = launch_steps(ctx, a, sync_bytes, n, ctx->host_tokens.data())) return rc;
   if (out_host) memcpy(out_host, ctx->host_tokens.data(), size_t(n) * 4);
   return KIE_OK;
 }
@@ -874,6 +923,12 @@ extern "C" int kie_debug_set(kie_ctx *ctx, int32_t watchdog_ms, int32_t skip_sig
   return KIE_OK;
 }
 
+extern "C" int kie_set_max_steps_per_launch(kie_ctx *ctx, int32_t n) {
+  if (!ctx || n < 0) return KIE_ERR_INVALID;
+  ctx->max_launch_steps = n;
+  return KIE_OK;
+}
+
 extern "C" int kie_set_sync_mode(kie_ctx *ctx, int32_t mode) {
   if (!ctx || (mode != KIE_SYNC_DEPENDENCY && mode != KIE_SYNC_GRID)) return KIE_ERR_INVALID;
   ctx->grid_sync = mode == KIE_SYNC_GRID ? 1 : 0;
@@ -992,24 +1047,10 @@ extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t
   a.skip_signal_cta = -1;
   a.grid_sync = ctx->grid_sync;
 
-  cudaStream_t st = ctx->stream;
-  // the counters and the argmax keys must start at zero on every call
   if (forced_tokens)
-    CK(cudaMemcpyAsync(s + o_tin, forced_tokens, size_t(n_steps) * 4, cudaMemcpyHostToDevice, st));
-  CK(cudaMemsetAsync(s, 0, o_tin, st));
-  CK(cudaMemsetAsync(a.acc_o, 0, size_t(4) * m.d_model * 4, st));   // both accumulators
-  void *args[] = {&a};
-  CK(cudaEventRecord(ctx->ev0, st));
-  CK(cudaLaunchCooperativeKernel(monokernel_fn(m.dtype), dim3(P.n_ctas), dim3(monokernel_threads()),
-                                 args, P.smem, st));
-  CK(cudaEventRecord(ctx->ev1, st));
-  uint32_t status = 0;
-  CK(cudaMemcpyAsync(&status, s + SY_STATUS * kSyncStride * 4, 4, cudaMemcpyDeviceToHost, st));
-  CK(cudaMemcpyAsync(out_tokens, s + o_tout, size_t(n_steps) * 4, cudaMemcpyDeviceToHost, st));
-  CK(cudaStreamSynchronize(st));
-  CK(cudaEventElapsedTime(&ctx->last_ms, ctx->ev0, ctx->ev1));
-  ctx->last_steps = n_steps;
-  if (status != 0) return device_error(ctx, status);
+    CK(cudaMemcpyAsync(s + o_tin, forced_tokens, size_t(n_steps) * 4, cudaMemcpyHostToDevice,
+                       ctx->stream));
+  if (int rc = launch_steps(ctx, a, sync_bytes, n_steps, out_tokens)) return rc;
   ctx->pos += n_steps;
   ctx->pending = out_tokens[n_steps - 1];
   return KIE_OK;

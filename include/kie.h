@@ -149,8 +149,9 @@ typedef struct {
   int32_t pos;                /* next position to be written */
   int64_t weight_bytes_per_step; /* weights one decode step streams (incl. LM head) */
   int64_t kv_bytes_per_position; /* K+V bytes per cached position, all layers */
-  float last_kernel_ms;       /* device time of the most recent launch (CUDA events) */
-  int32_t last_launch_steps;  /* steps run by that launch */
+  float last_kernel_ms;       /* device time of the most recent call's launches, from the
+                                 first one's start to the last one's end (CUDA events) */
+  int32_t last_launch_steps;  /* steps run by that call */
   int32_t pending_token;
 } kie_stats;
 
@@ -208,6 +209,16 @@ int kie_debug_set(kie_ctx *ctx, int32_t watchdog_ms, int32_t skip_signal_cta);
  * Returns KIE_ERR_INVALID for any other mode. */
 enum { KIE_SYNC_DEPENDENCY = 0, KIE_SYNC_GRID = 1 };
 int kie_set_sync_mode(kie_ctx *ctx, int32_t mode);
+
+/* Most decode steps one kernel launch runs (applies to later calls of this
+ * context).  A call with more steps runs as several launches back to back,
+ * each starting at the position and token where the previous one stopped;
+ * the results are those of one launch.  The kernel's epoch counters are
+ * 32-bit, so a launch never runs more than (2^31 - 1) / ((4 n_layers + 2) *
+ * SMs) steps whatever is set here (about 105,000 steps for 34 layers on 148
+ * SMs).  n = 0 restores that limit; n > 0 lowers it (to bound how long one
+ * launch holds the GPU).  Returns KIE_ERR_INVALID for n < 0. */
+int kie_set_max_steps_per_launch(kie_ctx *ctx, int32_t n);
 
 #ifdef __cplusplus
 }

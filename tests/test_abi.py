@@ -101,6 +101,7 @@ def test_null_context_calls_rejected(lib):
     assert "watchdog" in kie.strerror(kie.KIE_ERR_DEVICE_TIMEOUT)
     assert "non-finite" in kie.strerror(kie.KIE_ERR_NONFINITE)
     assert lib.kie_set_sync_mode(None, kie.KIE_SYNC_GRID) == kie.KIE_ERR_INVALID
+    assert lib.kie_set_max_steps_per_launch(None, 5) == kie.KIE_ERR_INVALID
 
 
 def test_binding_loads_one_library_per_process(lib):

@@ -95,6 +95,45 @@ def test_tiny_free_run_teacher_forced_and_cache():
     dec.kie_destroy()
 
 
+@pytest.mark.parametrize("cap", [1, 5])
+def test_calls_split_into_several_launches(cap):
+    """A call longer than the per-launch step limit runs as several launches,
+    each starting where the previous one stopped: the prompt (16 tokens) and
+    32 decode steps with at most `cap` steps per launch give the oracle's
+    logits, greedy tokens and cache, as one launch does."""
+    w = synth.WORKLOADS[0]
+    m = w.model
+    bits = synth.generate_weights(m, w.weight_seed)
+    prompt = synth.prompt(w)
+    P, N = w.prompt_len, w.decode_len
+    max_seq = P + N + 8
+    orc = Oracle(m, bits, max_seq)
+    t0, z0 = orc.prefill(prompt)
+    toks, zs = orc.decode(N)
+    dec = make_decoder(m, bits, max_seq)
+    dec.kie_set_max_steps_per_launch(cap)
+    g0 = dec.kie_prefill(prompt)
+    check_argmax([g0], z0, f"prefill, {cap} steps per launch")
+    gt = dec.kie_decode(N)
+    free_run_prefix(np.concatenate([[g0], gt]), np.concatenate([[t0], toks]),
+                    np.vstack([z0, zs]), f"free run, {cap} steps per launch")
+    st = dec.kie_get_stats()
+    assert st.pos == P + N and st.pending_token == gt[-1] and st.last_launch_steps == N
+    forced = np.concatenate([[t0], toks[:-1]]).astype(np.int32)
+    dec.kie_prefill(prompt)
+    gt2, z = _gpu_logits(dec, N, m.vocab, forced)
+    check_logits(z, zs, f"teacher-forced, {cap} steps per launch")
+    check_argmax(gt2, zs, f"teacher-forced, {cap} steps per launch")
+    orc2 = Oracle(m, bits, max_seq)
+    orc2.teacher_forced_logits(prompt, forced)
+    _check_kv(dec, orc2, m, P + N, max_seq)
+    import decode_persistent_monokernel_b200 as kie
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_set_max_steps_per_launch(-1)
+    assert e.value.code == kie.KIE_ERR_INVALID
+    dec.kie_destroy()
+
+
 def test_tiny_is_repeatable():
     """Two launches agree to float rounding.  The O and down projections are
     summed over SMs with fp32 atomics, so the summation order (and the last
