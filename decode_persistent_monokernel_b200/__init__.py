@@ -81,6 +81,7 @@ def load(path: str = None) -> ctypes.CDLL:
     L = ctypes.CDLL(path)
     sig = {
         "kie_create": ([ctypes.POINTER(kie_model_desc), _P, _P, ctypes.POINTER(_P)], _I),
+        "kie_weights_bytes": ([ctypes.POINTER(kie_model_desc), ctypes.POINTER(ctypes.c_int64)], _I),
         "kie_prefill": ([_P, _P, _I, ctypes.POINTER(_I)], _I),
         "kie_decode": ([_P, _I, _P], _I),
         "kie_decode_ex": ([_P, _I, _P, _P, _P], _I),
@@ -129,6 +130,13 @@ def make_desc(shape, max_seq: int) -> kie_model_desc:
                           shape.n_lanes, shape.lane_delay if shape.n_lanes > 1 else 0, max_seq)
 
 
+def weights_bytes(desc: kie_model_desc) -> int:
+    """Bytes of the canonical weights kie_create reads for `desc`."""
+    n = ctypes.c_int64()
+    _check(load().kie_weights_bytes(ctypes.byref(desc), ctypes.byref(n)))
+    return n.value
+
+
 def _ptr(buf):
     """Address of a torch tensor or a numpy array (host buffers must be contiguous)."""
     if buf is None:
@@ -144,6 +152,13 @@ class Decoder:
     def __init__(self, desc: kie_model_desc, weights_dev, stream=None):
         L = load()
         self._h = _P()
+        if hasattr(weights_dev, "data_ptr"):
+            # the library reads exactly weights_bytes(desc) from the pointer
+            need = weights_bytes(desc)
+            if not (weights_dev.is_cuda and weights_dev.is_contiguous()
+                    and weights_dev.numel() * weights_dev.element_size() == need):
+                raise ValueError(f"weights must be a contiguous CUDA tensor of {need} bytes "
+                                 f"(the canonical layout of this model)")
         st = None if stream is None else (stream.cuda_stream if hasattr(stream, "cuda_stream")
                                           else stream)
         _check(L.kie_create(ctypes.byref(desc), _ptr(weights_dev), st, ctypes.byref(self._h)))

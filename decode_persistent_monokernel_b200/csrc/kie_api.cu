@@ -485,6 +485,16 @@ static int alloc(kie_ctx *ctx, void **p, size_t bytes, const char *what) {
   return KIE_OK;
 }
 
+extern "C" int kie_weights_bytes(const kie_model_desc *desc, int64_t *out) {
+  if (!out) return KIE_ERR_INVALID;
+  if (const char *why = validate(desc)) {
+    g_last_error = why;
+    return KIE_ERR_INVALID;
+  }
+  *out = make_layout(*desc).total * 2;
+  return KIE_OK;
+}
+
 extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void *stream,
                           kie_ctx **out) {
   if (!out) return KIE_ERR_INVALID;

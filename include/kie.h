@@ -25,8 +25,11 @@
  *   - calls are synchronous: they return after the work queued on the
  *     context's stream has finished;
  *   - after KIE_ERR_DEVICE_TIMEOUT, KIE_ERR_NONFINITE or KIE_ERR_CUDA the
- *     context is poisoned:
- *     every later call except kie_destroy returns KIE_ERR_POISONED.
+ *     context is poisoned: every later kie_prefill and kie_decode* call
+ *     returns KIE_ERR_POISONED.  kie_destroy and the calls that only read
+ *     state back (kie_get_stats, kie_copy_kv, kie_get_profile,
+ *     kie_get_trace) still work, so a failed launch can be inspected; the
+ *     settings calls still take effect but nothing runs again.
  *   - a context is not thread-safe; use one per host thread.
  */
 #ifndef KIE_H
@@ -81,11 +84,18 @@ typedef struct kie_ctx kie_ctx;
  *         wv[Hkvl*dh,dl], wo[dl,Hql*dh], ffn_norm[dl], w_gate[Fl,dl],
  *         w_up[Fl,dl], w_down[dl,Fl];  lane models then mix[d,d];
  *       final_norm[d], lm_head[V,d].
+ *     The buffer must hold kie_weights_bytes(desc) bytes; the library reads
+ *     exactly those and cannot check a raw pointer's extent itself.
  *     Borrowed for this call only: the library copies the weights into its
  *     own per-SM streaming layout, so the caller may free them on return.
  *   stream: cudaStream_t to run on (NULL = legacy default stream).
  *   out: receives the context (owner: caller, release with kie_destroy). */
 int kie_create(const kie_model_desc *desc, const void *weights, void *stream, kie_ctx **out);
+
+/* Size in bytes of the canonical weights of `desc` (what kie_create reads).
+ * Host-only, no device work; KIE_ERR_INVALID (reason via kie_strerror) for a
+ * descriptor kie_create would refuse, or a null out. */
+int kie_weights_bytes(const kie_model_desc *desc, int64_t *out);
 
 /* Process a prompt from position 0 (the KV cache is reset and its unused
  * slots filled with NaN) and return the greedy next token, the argmax of the

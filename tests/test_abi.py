@@ -7,6 +7,8 @@ import subprocess
 
 import pytest
 
+import synth
+
 import decode_persistent_monokernel_b200 as kie
 from decode_persistent_monokernel_b200 import build as kbuild
 
@@ -82,6 +84,24 @@ def test_invalid_descriptors_rejected(lib, bad):
     rc = lib.kie_create(ctypes.byref(_desc(**bad)), ctypes.c_void_p(16), None, ctypes.byref(h))
     assert rc == kie.KIE_ERR_INVALID
     assert not h.value
+
+
+def test_weights_bytes_matches_the_canonical_layout(lib):
+    # the library's layout size against the generator's own tensor table
+    for w in synth.WORKLOADS.values():
+        desc = kie.make_desc(w.model, 64)
+        assert kie.weights_bytes(desc) == 2 * synth.total_elements(w.model), w.model
+    n = ctypes.c_int64()
+    assert lib.kie_weights_bytes(ctypes.byref(_desc(n_kv_heads=3)), ctypes.byref(n)) == \
+        kie.KIE_ERR_INVALID
+    assert lib.kie_weights_bytes(ctypes.byref(_desc()), None) == kie.KIE_ERR_INVALID
+
+
+def test_binding_checks_the_weights_tensor_before_the_library(lib):
+    import torch
+    desc = _desc()
+    with pytest.raises(ValueError):      # a host tensor
+        kie.Decoder(desc, torch.zeros(kie.weights_bytes(desc) // 2, dtype=torch.int16))
 
 
 def test_null_and_misaligned_weights_rejected(lib):

@@ -412,6 +412,13 @@ def test_watchdog_reports_a_missing_signal():
     with pytest.raises(kie.KieError) as e:
         dec.kie_decode(1)
     assert e.value.code == kie.KIE_ERR_POISONED
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_prefill(prompt)
+    assert e.value.code == kie.KIE_ERR_POISONED
+    # the read-back calls still work, so the failed launch can be inspected
+    assert dec.kie_get_stats().pos == len(prompt)
+    k, _ = dec.kie_copy_kv(0, 0, 0, len(prompt))
+    assert np.isfinite(storage_to_f64(k, m.dtype)).all()
     dec.kie_destroy()
     dec = make_decoder(m, bits, 64)
     t0 = dec.kie_prefill(prompt)
