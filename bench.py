@@ -209,6 +209,15 @@ def oracle_decode_rate(w, bits, seconds, warmup=0, max_steps=None):
     return n / el, n, el, cores
 
 
+def run_config(w, P, K, world, sync, weight_bytes_per_step):
+    """The `config` object of the bench line, the same for both arms."""
+    return {"workload": w.name, "prompt": P, "decode_steps": K, "batch": 1,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "sync": sync,
+            "l2": "inputs larger than L2: %.2f GB of weights streamed per step"
+                  % (weight_bytes_per_step / 1e9)}
+
+
 def reduce_max_over_ranks(values, world, device):
     """Max over ranks of per-rank timings (a job takes as long as its slowest
     rank); identity for one rank."""
@@ -246,11 +255,11 @@ def main():
         bits = synth.generate_weights(m, w.weight_seed)
         budget = max(5.0, min(120.0, args.cpu_seconds * 4))
         rate, n, el, cores = oracle_decode_rate(w, bits, budget, warmup=min(W, 3), max_steps=K)
-        line = {"metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": 0, "steps": n,
+        line = {"metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": world, "steps": n,
                 "warmup": min(W, 3), "ms_per_step": 1e3 / rate, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "impl": "reference",
-                "config": {"workload": w.name, "prompt": P, "decode_steps": K, "batch": 1},
+                "config": run_config(w, P, K, world, args.sync, synth.streamed_weight_bytes(m)),
                 "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores,
                                  "kind": "oracle",
                                  "sample": f"{n} greedy decode steps of the float64 numpy "
@@ -327,11 +336,7 @@ def main():
         "warmup": W, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 (fp16 weights/KV)" if m.dtype == "f16"
         else "f32 (bf16 weights/KV)", "data": "synthetic (seeded weights and prompt)",
-        "config": {"workload": w.name, "prompt": P, "decode_steps": K, "batch": 1,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "sync": args.sync,
-                   "l2": "inputs larger than L2: %.2f GB of weights streamed per step"
-                         % (st.weight_bytes_per_step / 1e9)},
+        "config": run_config(w, P, K, world, args.sync, st.weight_bytes_per_step),
         "us_per_token": 1e3 * ms / K,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,

@@ -91,6 +91,10 @@ def test_weights_bytes_matches_the_canonical_layout(lib):
     for w in synth.WORKLOADS.values():
         desc = kie.make_desc(w.model, 64)
         assert kie.weights_bytes(desc) == 2 * synth.total_elements(w.model), w.model
+        # a step streams all of it but the V - 1 embedding rows it does not use
+        m = w.model
+        assert kie.weights_bytes(desc) - 2 * (m.vocab - 1) * m.d_model == \
+            synth.streamed_weight_bytes(m)
     n = ctypes.c_int64()
     assert lib.kie_weights_bytes(ctypes.byref(_desc(n_kv_heads=3)), ctypes.byref(n)) == \
         kie.KIE_ERR_INVALID

@@ -78,3 +78,34 @@ def test_traffic_is_scaled_only_for_the_captured_kernel_and_workload():
     other = (int(rec["workload"]) + 1) % 5
     t, src = bench.dram_traffic(1e9, other)
     assert t is None
+
+
+def test_reference_arm_line_keeps_the_contract():
+    """The reference arm (the oracle on the host cores) prints one JSON line
+    with the keys of the bench contract, the same metric, unit and config as
+    the GPU arm, and its own cpu_baseline and e2e objects."""
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "LOCAL_RANK", "WORLD_SIZE")}
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "2", "--warmup", "3", "--cpu-seconds", "1"], env=env,
+                         capture_output=True, text=True, timeout=900)
+    assert res.returncode == 0, res.stderr[-2000:]
+    line = json.loads(res.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "impl", "cpu_baseline", "e2e"):
+        assert key in line, key
+    w = synth.WORKLOADS[1]
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["n_gpus"] == 1 and line["warmup"] >= 3 and 1 <= line["steps"] <= 2
+    assert line["config"] == bench.run_config(w, w.prompt_len, 2, 1, "dependency",
+                                              synth.streamed_weight_bytes(w.model))
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] > 0
+    assert cb["unit"] == line["unit"] and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
