@@ -179,9 +179,10 @@ class ClockSampler:
 
 def workload_bytes(m, P, K, weight_bytes_per_step, kv_bytes_per_position):
     """Algorithmic bytes of K decode steps after a P-token prompt: every weight
-    once per step plus K and V of all positions 0..p at step p."""
+    once per step, K and V of all positions 0..p read at step p, and position
+    p's K and V written."""
     kv_positions = sum(P + k + 1 for k in range(K))
-    return K * weight_bytes_per_step + kv_positions * kv_bytes_per_position
+    return K * weight_bytes_per_step + (kv_positions + K) * kv_bytes_per_position
 
 
 def oracle_decode_rate(w, bits, seconds, warmup=0, max_steps=None):

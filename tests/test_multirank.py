@@ -109,3 +109,22 @@ def test_reference_arm_line_keeps_the_contract():
     assert cb["unit"] == line["unit"] and cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_algorithmic_bytes_agree_between_bench_and_the_counter_case():
+    """bench.py and the counter-capture case count the same bytes for the same
+    steps: every weight once per step (from the generator's tensor table), the
+    K/V of positions 0..p read and position p written."""
+    sys.path.insert(0, ROOT)
+    import dataclasses
+    import bench
+    import synth
+    from decode_persistent_monokernel_b200 import profile_case
+    for wid in (0, 1, 4):
+        w = synth.WORKLOADS[wid]
+        m = dataclasses.replace(w.model, n_layers=3)
+        P, steps = w.prompt_len, 5
+        kvpp = 2 * m.n_layers * m.n_kv_heads * m.head_dim * 2
+        # the counter case times the launch after a warm-up launch of `steps`
+        got = bench.workload_bytes(m, P + steps, steps, synth.streamed_weight_bytes(m), kvpp)
+        assert got == profile_case.algorithmic_bytes(m, P, steps), wid
