@@ -299,6 +299,10 @@ int main() {
   check(gq, 148, "cfg0-gqa2");
   check(g4, 148, "cfg0-gqa4");
   check(c0, 20, "cfg0-20cta");
+  // degenerate: fewer hidden units and vocabulary rows than SMs, so many SMs
+  // have no gate/up/down rows and no LM-head rows; one query head per KV group
+  kie_model_desc tinyv{2, 256, 4, 4, 64, 96, 100, 1e-5f, 1e4f, 0, 1, 0, 64};
+  check(tinyv, 148, "degenerate-F96-V100");
   check(l2, 148, "lanes2");
   check(l4, 148, "lanes4");
   check(d128, 148, "dh128");
