@@ -101,8 +101,10 @@ int kie_weights_bytes(const kie_model_desc *desc, int64_t *out);
  * slots filled with NaN) and return the greedy next token, the argmax of the
  * logits at position n-1.
  *   tokens: HOST array of n ids in [0, vocab); next_token: HOST out.
- *   n < 1 or an id outside [0, vocab) returns KIE_ERR_INVALID before any
- *   device work (the cache and position are left as they were). */
+ *   n < 1 or an id outside [0, vocab) returns KIE_ERR_INVALID and n > max_seq
+ *   KIE_ERR_CAPACITY, before any device work (the cache and position are left
+ *   as they were).  The prompt runs through the decode path one position per
+ *   step, in the same persistent kernel. */
 int kie_prefill(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_token);
 
 /* Greedy decode: step k feeds the pending token at position pos+k, appends
@@ -110,7 +112,9 @@ int kie_prefill(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_to
  * pending token.  The first pending token is kie_prefill's next_token.
  *   out_tokens: HOST array of n_steps.
  *   n_steps < 1, or no pending token (no kie_prefill yet), returns
- *   KIE_ERR_INVALID before any device work. */
+ *   KIE_ERR_INVALID, and pos + n_steps > max_seq KIE_ERR_CAPACITY, before any
+ *   device work.  All steps run in one kernel launch, or in several back to
+ *   back beyond the per-launch limit (kie_set_max_steps_per_launch). */
 int kie_decode(kie_ctx *ctx, int32_t n_steps, int32_t *out_tokens);
 
 /* kie_decode with options:
