@@ -177,21 +177,37 @@ class Decoder:
         _check(load().kie_decode(self._h, n_steps, out.ctypes.data))
         return out
 
+    def _decode_args(self, n_steps: int, forced, logits_out):
+        """The library reads n_steps forced tokens and writes n_steps * vocab
+        logits through raw pointers, so their buffers are checked here."""
+        import numpy as np
+        f = None
+        if forced is not None:
+            f = np.ascontiguousarray(forced, dtype=np.int32)
+            if f.ndim != 1 or f.size != n_steps:
+                raise ValueError(f"forced must hold exactly n_steps = {n_steps} token ids")
+        if logits_out is not None:
+            need = max(n_steps, 0) * self.desc.vocab
+            if not (hasattr(logits_out, "data_ptr") and logits_out.is_cuda
+                    and str(logits_out.dtype) == "torch.float32" and logits_out.is_contiguous()
+                    and logits_out.numel() >= need):
+                raise ValueError(f"logits_out must be a contiguous float32 CUDA tensor of at "
+                                 f"least n_steps * vocab = {need} elements")
+        return (None if f is None else f.ctypes.data), _ptr(logits_out), f
+
     def kie_decode_ex(self, n_steps: int, forced=None, logits_out=None):
         import numpy as np
         out = np.empty(n_steps, dtype=np.int32)
-        f = None if forced is None else np.ascontiguousarray(forced, dtype=np.int32)
-        _check(load().kie_decode_ex(self._h, n_steps, None if f is None else f.ctypes.data,
-                                    out.ctypes.data, _ptr(logits_out)))
+        fp, lp, _keep = self._decode_args(n_steps, forced, logits_out)
+        _check(load().kie_decode_ex(self._h, n_steps, fp, out.ctypes.data, lp))
         return out
 
     def kie_decode_ex_static(self, n_steps: int, forced=None, logits_out=None):
         """kie_decode_ex with the kernel scratch in the library's fixed device array."""
         import numpy as np
         out = np.empty(n_steps, dtype=np.int32)
-        f = None if forced is None else np.ascontiguousarray(forced, dtype=np.int32)
-        _check(load().kie_decode_ex_static(self._h, n_steps, None if f is None else f.ctypes.data,
-                                           out.ctypes.data, _ptr(logits_out)))
+        fp, lp, _keep = self._decode_args(n_steps, forced, logits_out)
+        _check(load().kie_decode_ex_static(self._h, n_steps, fp, out.ctypes.data, lp))
         return out
 
     def kie_get_stats(self) -> kie_stats:

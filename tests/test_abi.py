@@ -108,6 +108,24 @@ def test_binding_checks_the_weights_tensor_before_the_library(lib):
         kie.Decoder(desc, torch.zeros(kie.weights_bytes(desc) // 2, dtype=torch.int16))
 
 
+def test_binding_checks_decode_buffers_before_the_library(lib):
+    # a Decoder shell (no context: nothing may reach the library) with a model
+    # descriptor, to exercise the argument checks alone
+    import numpy as np
+    import torch
+    dec = kie.Decoder.__new__(kie.Decoder)
+    dec._h = ctypes.c_void_p()
+    dec.desc = _desc()
+    with pytest.raises(ValueError):       # fewer forced tokens than steps
+        dec.kie_decode_ex(4, forced=np.zeros(3, dtype=np.int32))
+    with pytest.raises(ValueError):       # logits into host memory
+        dec.kie_decode_ex(2, logits_out=torch.zeros(2, dec.desc.vocab))
+    with pytest.raises(ValueError):       # the static variant checks the same
+        dec.kie_decode_ex_static(4, forced=np.zeros(5, dtype=np.int32))
+    fp, lp, _ = dec._decode_args(3, np.arange(3), None)
+    assert fp is not None and lp is None
+
+
 def test_null_and_misaligned_weights_rejected(lib):
     h = ctypes.c_void_p()
     assert lib.kie_create(ctypes.byref(_desc()), None, None, ctypes.byref(h)) == kie.KIE_ERR_INVALID
