@@ -126,6 +126,43 @@ def test_binding_checks_decode_buffers_before_the_library(lib):
     assert fp is not None and lp is None
 
 
+_C_CLIENT = r"""
+#include <stdio.h>
+#include "kie.h"
+#include "kie_ubench.h"
+int main(void) {
+  kie_model_desc d = {0};
+  int64_t bytes = 0;
+  d.n_layers = 2; d.d_model = 256; d.n_heads = 4; d.n_kv_heads = 4; d.head_dim = 64;
+  d.ffn_dim = 704; d.vocab = 4096; d.rms_eps = 1e-5f; d.rope_theta = 1e4f;
+  d.dtype = KIE_F16; d.n_lanes = 1; d.lane_delay = 0; d.max_seq = 64;
+  int rc = kie_weights_bytes(&d, &bytes);
+  printf("%d %lld\n", rc, (long long)bytes);
+  d.n_kv_heads = 3;
+  const int bad = kie_weights_bytes(&d, &bytes);
+  printf("%d %s\n", bad, kie_strerror(KIE_ERR_INVALID));
+  return rc;
+}
+"""
+
+
+def test_plain_c_client_compiles_links_and_calls_the_library(lib, tmp_path):
+    """The headers are plain C (C99, pedantic, warnings as errors) and a C
+    program links against libkie.so and calls it (host-only calls here)."""
+    src = tmp_path / "client.c"
+    src.write_text(_C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(kie.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.dirname(kie.HEADER), str(src), "-o", str(exe),
+                    "-L", libdir, "-lkie", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    rc, nbytes = out[0].split()
+    assert int(rc) == 0 and int(nbytes) == 2 * synth.total_elements(synth.WORKLOADS[0].model)
+    assert out[1].startswith(f"{kie.KIE_ERR_INVALID} invalid argument")
+    assert "multiple of n_kv_heads" in out[1]
+
+
 def test_null_and_misaligned_weights_rejected(lib):
     h = ctypes.c_void_p()
     assert lib.kie_create(ctypes.byref(_desc()), None, None, ctypes.byref(h)) == kie.KIE_ERR_INVALID
