@@ -197,7 +197,9 @@ def oracle_decode_rate(w, bits, seconds, warmup=0, max_steps=None):
     import synth
     prompt = synth.prompt(w)
     orc = Oracle(m, bits, w.prompt_len + 4096, cache_f64=True)
+    t_pre = time.perf_counter()
     orc.prefill(prompt)
+    prefill_s = time.perf_counter() - t_pre
     if warmup:
         orc.decode(warmup)
     n, t0 = 0, time.perf_counter()
@@ -207,7 +209,27 @@ def oracle_decode_rate(w, bits, seconds, warmup=0, max_steps=None):
         el = time.perf_counter() - t0
         if el >= seconds or (max_steps and n >= max_steps):
             break
-    return n / el, n, el, cores
+    return n / el, n, el, cores, prefill_s
+
+
+def host_cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline_obj(rate, n, el, cores, prefill_s, P):
+    """The `cpu_baseline` object: the float64 oracle's greedy decode rate on
+    this host (a bounded sample), with its untimed prompt's time beside it."""
+    return {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} greedy decode steps of the float64 numpy oracle after the "
+                      f"{P}-token prompt ({el:.1f} s)",
+            "prefill_s": prefill_s, "cpu": host_cpu_model(), "host_cpus": os.cpu_count()}
 
 
 def run_config(w, P, K, world, sync, weight_bytes_per_step):
@@ -255,16 +277,14 @@ def main():
             return
         bits = synth.generate_weights(m, w.weight_seed)
         budget = max(5.0, min(120.0, args.cpu_seconds * 4))
-        rate, n, el, cores = oracle_decode_rate(w, bits, budget, warmup=min(W, 3), max_steps=K)
+        rate, n, el, cores, prefill_s = oracle_decode_rate(w, bits, budget, warmup=min(W, 3),
+                                                           max_steps=K)
         line = {"metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": world, "steps": n,
                 "warmup": min(W, 3), "ms_per_step": 1e3 / rate, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "impl": "reference",
                 "config": run_config(w, P, K, world, args.sync, synth.streamed_weight_bytes(m)),
-                "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores,
-                                 "kind": "oracle",
-                                 "sample": f"{n} greedy decode steps of the float64 numpy "
-                                           f"oracle after the {P}-token prompt ({el:.1f} s)"},
+                "cpu_baseline": cpu_baseline_obj(rate, n, el, cores, prefill_s, P),
                 "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
@@ -361,11 +381,8 @@ def main():
         line["profile_build"] = "libkie_prof.so (activity counters on): not the benchmark value"
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         dec.kie_destroy()
-        rate, n, el, cores = oracle_decode_rate(w, bits, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
-                                "kind": "oracle",
-                                "sample": f"{n} greedy decode steps of the float64 numpy oracle "
-                                          f"after the {P}-token prompt ({el:.1f} s)"}
+        rate, n, el, cores, prefill_s = oracle_decode_rate(w, bits, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline_obj(rate, n, el, cores, prefill_s, P)
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
