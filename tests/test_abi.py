@@ -181,6 +181,16 @@ def test_null_context_calls_rejected(lib):
     assert "non-finite" in kie.strerror(kie.KIE_ERR_NONFINITE)
     assert lib.kie_set_sync_mode(None, kie.KIE_SYNC_GRID) == kie.KIE_ERR_INVALID
     assert lib.kie_set_max_steps_per_launch(None, 5) == kie.KIE_ERR_INVALID
+    # every other call that takes a context refuses a null one before any device work
+    buf = (ctypes.c_uint64 * 8)()
+    assert lib.kie_decode_ex(None, 1, None, buf, None) == kie.KIE_ERR_INVALID
+    assert lib.kie_decode_ex_static(None, 1, None, buf, None) == kie.KIE_ERR_INVALID
+    assert lib.kie_copy_kv(None, 0, 0, 0, 1, buf, buf) == kie.KIE_ERR_INVALID
+    assert lib.kie_get_profile(None, buf, 8) == kie.KIE_ERR_INVALID
+    assert lib.kie_trace_request(None, 0, 0) == kie.KIE_ERR_INVALID
+    assert lib.kie_get_trace(None, buf, 8) == kie.KIE_ERR_INVALID
+    assert lib.kie_debug_set(None, 100, -1) == kie.KIE_ERR_INVALID
+    assert lib.kie_create(ctypes.byref(_desc()), ctypes.c_void_p(16), None, None) == kie.KIE_ERR_INVALID
 
 
 def test_binding_loads_one_library_per_process(lib):
