@@ -394,6 +394,9 @@ struct kie_ctx {
   int skip_signal_cta = -1;
   int grid_sync = 0;
   int max_launch_steps = 0;   // 0: the counters' own limit (steps_per_launch)
+  // L2 look-ahead of the weight producer while its ring is full (KIE_L2PF_TILES,
+  // KIE_L2PF_DELAY, KIE_L2PF_PACE): most tiles, cycles before, cycles between
+  int l2pf_tiles = 0, l2pf_delay = 2000, l2pf_pace = 600;
   float last_ms = 0.f;
   int last_steps = 0;
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
@@ -520,6 +523,10 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
     long v = atol(env);
     if (v > 0) ctx->watchdog_ns = uint64_t(v) * 1000000ull;
   }
+  // tuning overrides of the L2 look-ahead (clamped to sane ranges)
+  if (const char *env = getenv("KIE_L2PF_TILES")) ctx->l2pf_tiles = std::max(0, std::min(64, atoi(env)));
+  if (const char *env = getenv("KIE_L2PF_DELAY")) ctx->l2pf_delay = std::max(0, std::min(1 << 24, atoi(env)));
+  if (const char *env = getenv("KIE_L2PF_PACE")) ctx->l2pf_pace = std::max(0, std::min(1 << 24, atoi(env)));
   cudaError_t e = cudaGetDevice(&ctx->device);
   if (e != cudaSuccess) return fail(cuda_fail(nullptr, "cudaGetDevice", e));
   cudaPointerAttributes pa{};
@@ -734,11 +741,15 @@ static int launch_steps(kie_ctx *ctx, const KernelArgs &a, size_t sync_bytes, in
   return KIE_OK;
 }
 
-static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int first_token,
-               bool logits_every_step, float *logits_out, int32_t *out_host) {
+// Kernel arguments of one call: the model, the plan, the weights, the KV
+// cache and the context's settings.  The caller points the per-launch scratch
+// (activations, counters, keys, token buffers) somewhere and sets the run
+// fields it needs beyond pos0 / n / first token / logits.  The pending test
+// hook (skip_signal_cta) is consumed here, so it applies to exactly one call.
+static KernelArgs fill_args(kie_ctx *ctx, int pos0, int n, int first_token,
+                            bool logits_every_step, float *logits_out) {
   const kie_model_desc &m = ctx->m;
   const Plan &P = ctx->plan;
-  cudaStream_t st = ctx->stream;
   KernelArgs a{};
   a.n_layers = m.n_layers; a.d_model = m.d_model; a.n_heads = m.n_heads;
   a.n_kv_heads = m.n_kv_heads; a.head_dim = m.head_dim; a.ffn_dim = m.ffn_dim; a.vocab = m.vocab;
@@ -758,19 +769,36 @@ static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int fi
   a.gain_attn = ctx->gains; a.gain_ffn = ctx->gains + size_t(m.n_layers) * m.d_model;
   a.gain_final = ctx->gains + size_t(2 * m.n_layers) * m.d_model;
   a.rope_cs = ctx->rope; a.kcache = ctx->kcache; a.vcache = ctx->vcache;
-  a.xres = ctx->act + ctx->off_xres;
-  a.acc_o = ctx->act + ctx->off_acc; a.acc_d = a.acc_o + 2 * size_t(m.d_model);
-  a.qkv = ctx->act + ctx->off_qkv; a.dsum = ctx->act + ctx->off_dsum;
-  a.attn_part = ctx->act + ctx->off_part; a.max_split = P.max_split;
-  a.sync = ctx->sync; a.keys = ctx->keys;
+  a.max_split = P.max_split;
   a.pos0 = pos0; a.n_steps = n; a.first_token = first_token;
-  a.forced = forced_host ? ctx->tokens_in : nullptr;
   a.logits_every_step = logits_every_step ? 1 : 0;
-  a.out_tokens = ctx->tokens_out; a.logits_out = logits_out;
+  a.logits_out = logits_out;
   a.watchdog_ns = ctx->watchdog_ns;
   a.skip_signal_cta = ctx->skip_signal_cta;
   ctx->skip_signal_cta = -1;
   a.grid_sync = ctx->grid_sync;
+  a.l2pf_tiles = ctx->l2pf_tiles; a.l2pf_delay = ctx->l2pf_delay; a.l2pf_pace = ctx->l2pf_pace;
+  return a;
+}
+
+// Points the kernel's per-launch activation scratch at `act` (laid out as the
+// context's activation buffer).
+static void set_act(const kie_ctx *ctx, KernelArgs &a, float *act) {
+  a.xres = act + ctx->off_xres;
+  a.acc_o = act + ctx->off_acc; a.acc_d = a.acc_o + 2 * size_t(ctx->m.d_model);
+  a.qkv = act + ctx->off_qkv; a.dsum = act + ctx->off_dsum;
+  a.attn_part = act + ctx->off_part;
+}
+
+static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int first_token,
+               bool logits_every_step, float *logits_out, int32_t *out_host) {
+  const kie_model_desc &m = ctx->m;
+  cudaStream_t st = ctx->stream;
+  KernelArgs a = fill_args(ctx, pos0, n, first_token, logits_every_step, logits_out);
+  set_act(ctx, a, ctx->act);
+  a.sync = ctx->sync; a.keys = ctx->keys;
+  a.forced = forced_host ? ctx->tokens_in : nullptr;
+  a.out_tokens = ctx->tokens_out;
   a.prof = ctx->prof;
   if (ctx->trace && ctx->trace_step >= 0 && ctx->trace_step < n) {
     a.trace = ctx->trace;
@@ -993,7 +1021,6 @@ extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t
     for (int i = 0; i < n_steps; ++i)
       if (forced_tokens[i] < 0 || forced_tokens[i] >= ctx->m.vocab) return KIE_ERR_INVALID;
   const kie_model_desc &m = ctx->m;
-  const Plan &P = ctx->plan;
   // carve the scratch: counters | keys | forced tokens | out tokens | activations
   auto up = [](size_t b) { return (b + 255) / 256 * 256; };
   const size_t sync_bytes = size_t(SY_QG0 + 2 * m.n_kv_heads) * kSyncStride * 4;
@@ -1023,39 +1050,16 @@ extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t
   uint8_t *s = static_cast<uint8_t *>(base);
   float *act = reinterpret_cast<float *>(s + o_act);
 
-  KernelArgs a{};
-  a.n_layers = m.n_layers; a.d_model = m.d_model; a.n_heads = m.n_heads;
-  a.n_kv_heads = m.n_kv_heads; a.head_dim = m.head_dim; a.ffn_dim = m.ffn_dim; a.vocab = m.vocab;
-  a.n_lanes = m.n_lanes; a.lane_delay = m.n_lanes > 1 ? m.lane_delay : 1;
-  a.lane_width = m.d_model / m.n_lanes; a.lane_heads = m.n_heads / m.n_lanes;
-  a.lane_kv_heads = m.n_kv_heads / m.n_lanes; a.lane_ffn = m.ffn_dim / m.n_lanes;
-  a.rms_eps = m.rms_eps;
-  a.attn_scale = float(1.0 / sqrt(double(m.head_dim)));
-  a.max_seq = m.max_seq;
-  a.n_ctas = P.n_ctas; a.ring_slots = P.ring_slots;
-  a.vbuf_floats = P.vbuf_floats; a.part_floats = P.part_floats;
-  a.part_atomic_off = P.part_atomic_off;
-  for (int k = 0; k < ST_COUNT; ++k) a.shape[k] = P.shape[k];
-  a.stage_cta = ctx->d_stage_cta; a.blocks = ctx->d_blocks;
-  a.cta_blk_begin = ctx->d_blk_begin; a.cta_stream_off = ctx->d_stream_off;
-  a.wstream = ctx->wstream; a.embed = ctx->embed;
-  a.gain_attn = ctx->gains; a.gain_ffn = ctx->gains + size_t(m.n_layers) * m.d_model;
-  a.gain_final = ctx->gains + size_t(2 * m.n_layers) * m.d_model;
-  a.rope_cs = ctx->rope; a.kcache = ctx->kcache; a.vcache = ctx->vcache;
-  a.xres = act + ctx->off_xres;
-  a.acc_o = act + ctx->off_acc; a.acc_d = a.acc_o + 2 * size_t(m.d_model);
-  a.qkv = act + ctx->off_qkv; a.dsum = act + ctx->off_dsum;
-  a.attn_part = act + ctx->off_part; a.max_split = P.max_split;
+  // Same arguments as kie_decode_ex (a pending kie_debug_set hook applies to
+  // this call and is consumed by it), except that every per-launch buffer is
+  // carved from the fixed array.  The profiling build's activity counters and
+  // trace are not wired here: they live in buffers of the context.
+  KernelArgs a = fill_args(ctx, ctx->pos, n_steps, ctx->pending, true, logits_out);
+  set_act(ctx, a, act);
   a.sync = reinterpret_cast<uint32_t *>(s);
   a.keys = reinterpret_cast<unsigned long long *>(s + o_keys);
-  a.pos0 = ctx->pos; a.n_steps = n_steps; a.first_token = ctx->pending;
   a.forced = forced_tokens ? reinterpret_cast<const int32_t *>(s + o_tin) : nullptr;
-  a.logits_every_step = 1;
   a.out_tokens = reinterpret_cast<int32_t *>(s + o_tout);
-  a.logits_out = logits_out;
-  a.watchdog_ns = ctx->watchdog_ns;
-  a.skip_signal_cta = -1;
-  a.grid_sync = ctx->grid_sync;
 
   if (forced_tokens)
     CK(cudaMemcpyAsync(s + o_tin, forced_tokens, size_t(n_steps) * 4, cudaMemcpyHostToDevice,

@@ -179,6 +179,9 @@ struct KernelArgs {
   uint64_t watchdog_ns;
   int32_t skip_signal_cta;      // test hook, -1 = off
   int32_t grid_sync;            // 1: every dependency wait is a grid-wide barrier
+  int32_t l2pf_tiles;           // L2 look-ahead while the ring is full: most tiles (0 = off)
+  int32_t l2pf_delay;           //   SM cycles of waiting for a free slot before it starts
+  int32_t l2pf_pace;            //   SM cycles between two look-ahead requests
   unsigned long long *prof;     // [n_ctas][kProfSlots] (profiling build), or nullptr
   unsigned long long *trace;    // [1 + trace_cap] event trace (profiling build), or nullptr
   int32_t trace_cap, trace_cta, trace_step;

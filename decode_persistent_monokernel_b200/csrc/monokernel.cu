@@ -222,8 +222,8 @@ __device__ bool wait_counter(const KernelArgs &a, const uint32_t *ctr, uint32_t 
   const uint32_t *abortp = sync_at(a, SY_ABORT);
   for (;;) {
     if (ld_acquire(ctr) >= target) return true;
-    pump();
     const long long el = clock64() - t0;
+    pump(el);
     if (el > next_poll) {
       next_poll = el + kAbortPollCycles;
       if (ld_relaxed(abortp)) return false;
@@ -245,8 +245,8 @@ __device__ bool wait_mbar(const KernelArgs &a, uint64_t *bar, uint32_t parity, u
   const uint32_t *abortp = sync_at(a, SY_ABORT);
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    pump();
     const long long el = clock64() - t0;
+    pump(el);
     if (el > next_poll) {
       next_poll = el + kAbortPollCycles;
       if (ld_relaxed(abortp)) return false;
@@ -272,7 +272,30 @@ struct Producer {
   Smem s;
   const int cta;
   uint32_t T = 0;        // tiles issued
+  // L2 look-ahead: bytes of the stream beyond `cur` already requested into L2,
+  // and the stream's extent in the current step (it wraps to the start of the
+  // stream, the next step's first tile, at `end`).
+  uint32_t pf_ahead = 0;
+  const uint8_t *base = nullptr, *end = nullptr;
   __device__ Producer(const KernelArgs &a_, Smem s_, int cta_) : a(a_), s(s_), cta(cta_) {}
+
+  // Called while the producer waits for a free ring slot.  A wait longer than
+  // l2pf_delay cycles means the consumers are held up by a dependency (other
+  // SMs, the attention), not by weights, and HBM would idle; then the next
+  // tiles of the stream are requested into L2, one every l2pf_pace cycles, up
+  // to l2pf_tiles tiles beyond the ring, so that they land from L2 once the
+  // consumers resume.
+  __device__ __forceinline__ void l2_lookahead(long long el, uint32_t &nthis, const uint8_t *cur) {
+    if (el < a.l2pf_delay + (long long)nthis * a.l2pf_pace) return;
+    if (pf_ahead >= uint32_t(a.l2pf_tiles) * kSlotBytes) return;
+    const uint8_t *p = cur + pf_ahead;
+    if (p >= end) p = base + (p - end);
+    if (p >= end) return;
+    const uint32_t bytes = uint32_t(min((long long)kSlotBytes, (long long)(end - p)));
+    prefetch_l2(p, bytes);
+    pf_ahead += bytes;
+    ++nthis;
+  }
 
   // The cached K/V rows this CTA's attention split reads in layer l of step
   // `step` (positions before the step's own), pulled into L2 when the layer's
@@ -307,7 +330,13 @@ struct Producer {
           const long long tw = clock64();
 #endif
           // the slot's previous tile (T - NS) was released by every consumer warp
-          if (!wait_mbar(a, &s.empty[slot], phase ^ 1u, DE_TIMEOUT_EMPTY, [] {})) return false;
+          uint32_t nthis = 0;
+          const uint8_t *c0 = cur;
+          const bool pf = a.l2pf_tiles > 0;
+          if (!wait_mbar(a, &s.empty[slot], phase ^ 1u, DE_TIMEOUT_EMPTY, [&](long long el) {
+                if (pf) l2_lookahead(el, nthis, c0);
+              }))
+            return false;
 #ifdef KIE_PROFILE
           s.misc->prof[PF_PROD_EMPTY] += clock64() - tw;
 #endif
@@ -316,6 +345,7 @@ struct Producer {
         mbar_expect_tx(&s.full[slot], bytes);
         bulk_g2s(s.ring + size_t(slot) * kSlotBytes, cur, bytes, &s.full[slot], policy_evict_first());
         cur += bytes;
+        pf_ahead = pf_ahead > bytes ? pf_ahead - bytes : 0u;
         ++T;
         if (++slot == NS) { slot = 0; phase ^= 1u; }
       }
@@ -324,12 +354,21 @@ struct Producer {
   }
 
   __device__ void run() {
-    const uint8_t *base = a.wstream + a.cta_stream_off[cta];
+    base = a.wstream + a.cta_stream_off[cta];
     const bool lanes = a.n_lanes > 1;
+    // bytes of one step's stream: every layer's stages, then the final lane
+    // mix and the LM head (when the step computes logits)
+    const StageCta *sc = s.misc->sc;
+    const int64_t layer_bytes = sc[ST_QKV].bytes + sc[ST_O].bytes + sc[ST_GU].bytes + sc[ST_D].bytes;
+    const int64_t body = int64_t(a.n_layers) * layer_bytes +
+                         (lanes ? int64_t(a.n_layers - 1) * sc[ST_MIX].bytes : 0);
+    const int64_t head = (lanes ? sc[ST_MIX].bytes : 0) + sc[ST_LM].bytes;
     uint32_t slot = 0, phase = 0;   // phase: parity of the slot's current use
     bool ok = true;
     for (int step = 0; step < a.n_steps && ok; ++step) {
       const uint8_t *cur = base;
+      const bool lm = a.logits_every_step || step == a.n_steps - 1;
+      end = base + body + (lm ? head : 0);
       for (int l = 0; l < a.n_layers && ok; ++l) {
         prefetch_kv(step, l);
         ok = stage(ST_QKV, cur, slot, phase);
@@ -400,7 +439,7 @@ struct Consumer {
         target = nsig * a.n_ctas;
       }
       KT(TE_GATE_BEGIN, pkind);
-      if (!wait_counter(a, sync_at(a, slot), target, where, [] {})) s.misc->abort = 1;
+      if (!wait_counter(a, sync_at(a, slot), target, where, [](long long) {})) s.misc->abort = 1;
       KT(TE_GATE_END, pkind);
 #ifdef KIE_PROFILE
       s.misc->prof[PF_GATE] += clock64() - t0;
@@ -532,7 +571,7 @@ struct Consumer {
   __device__ __forceinline__ bool tile_wait(int k) {
     bool got = true;
     KT(TE_TILE_WAIT, 0);
-    if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [] {});
+    if (lane == 0) got = wait_mbar(a, &s.full[slot], phase, DE_TIMEOUT_FULL | (k << 8), [](long long) {});
     KT(TE_TILE_READY, 0);
     return __shfl_sync(0xffffffffu, got, 0);
   }
