@@ -77,6 +77,12 @@ typedef struct {
 typedef struct kie_ctx kie_ctx;
 
 /* Build a context on the current CUDA device.
+ * Passage: "Startup Perancis Ini Kata Perisian Sahaja Cukup..." page, stack
+ * bullets -- the monokernel bullet (the whole decode path as one persistent
+ * kernel, nothing launched between layers) and the assembly-level bullet
+ * (aim at every cycle of memory bandwidth).  What this call prepares for that
+ * kernel: the weights re-laid out once into one contiguous stream per SM in
+ * the order the SM consumes them, the KV cache, and the scratch of one call.
  *   weights: DEVICE pointer to all weights in the canonical layout (storage
  *     dtype, row-major [out, in], concatenated, no padding):
  *       embed[V,d];
@@ -100,6 +106,11 @@ int kie_weights_bytes(const kie_model_desc *desc, int64_t *out);
 /* Process a prompt from position 0 (the KV cache is reset and its unused
  * slots filled with NaN) and return the greedy next token, the argmax of the
  * logits at position n-1.
+ * Passage: "Startup Kog dosahuje 3 000 tokenu/s..." page, section "Software
+ * versus kremik": the persistent program covers prefill as well as decode
+ * and LM-head sampling.  Here the prompt is run through that same persistent
+ * kernel, one position per step, with the LM head evaluated only at the last
+ * position.
  *   tokens: HOST array of n ids in [0, vocab); next_token: HOST out.
  *   n < 1 or an id outside [0, vocab) returns KIE_ERR_INVALID and n > max_seq
  *   KIE_ERR_CAPACITY, before any device work (the cache and position are left
@@ -110,6 +121,14 @@ int kie_prefill(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_to
 /* Greedy decode: step k feeds the pending token at position pos+k, appends
  * its K/V, and the argmax of its logits becomes out_tokens[k] and the next
  * pending token.  The first pending token is kie_prefill's next_token.
+ * Passages: the monokernel bullet of the "Startup Perancis Ini Kata Perisian
+ * Sahaja Cukup..." page (every layer of the decode path inside one persistent
+ * kernel), the "Software versus kremik" section of the "Startup Kog dosahuje
+ * 3 000 tokenu/s..." page (no per-token launch cost, grid synchronisations
+ * removed, the sampled token produced inside the kernel), and the results
+ * table of the first page ("Laneformer 2B: Keputusan yang Ditunjukkan":
+ * FP16, batch 1, greedy).  One call is one launch of that kernel for all
+ * n_steps tokens; the sampled token is fed back on the device.
  *   out_tokens: HOST array of n_steps.
  *   n_steps < 1, or no pending token (no kie_prefill yet), returns
  *   KIE_ERR_INVALID, and pos + n_steps > max_seq KIE_ERR_CAPACITY, before any
@@ -117,7 +136,9 @@ int kie_prefill(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_to
  *   back beyond the per-launch limit (kie_set_max_steps_per_launch). */
 int kie_decode(kie_ctx *ctx, int32_t n_steps, int32_t *out_tokens);
 
-/* kie_decode with options:
+/* kie_decode with options (same passages as kie_decode; the two options
+ * expose the decode path for checking it: teacher forcing fixes the fed
+ * tokens, and logits_out keeps the LM-head output the greedy sampling reads):
  *   forced_tokens: HOST array of n_steps ids, or NULL.  When given, step k
  *     feeds forced_tokens[k] instead of the pending token (teacher forcing);
  *     out_tokens still receives each step's argmax.

@@ -101,13 +101,14 @@ def test_reference_arm_line_keeps_the_contract():
     w = synth.WORKLOADS[1]
     assert line["impl"] == "reference" and line["metric"] == bench.METRIC
     assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
-    assert line["n_gpus"] == 1 and line["warmup"] >= 3 and 1 <= line["steps"] <= 2
+    assert line["n_gpus"] == 1 and line["warmup"] == 3 and 1 <= line["steps"] <= 2
     assert line["config"] == bench.run_config(w, w.prompt_len, 2, 1, "dependency",
                                               synth.streamed_weight_bytes(w.model))
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] > 0
     assert cb["unit"] == line["unit"] and cb["sample"]
-    assert cb["prefill_s"] > 0 and cb["cpu"] and cb["host_cpus"] >= 1 and cb["cores"] >= 1
+    assert cb["prefill_s"] > 0 and cb["cpu"] and cb["host_cpus"] >= 1
+    assert cb["cores"] == 1     # single-threaded, as the CPU baseline is planned
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
