@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--sync", choices=["dependency", "grid"], default="dependency",
                     help="how SMs wait for one another: per-dependency counters (default) or "
                          "a grid-wide barrier at every dependency point (ablation)")
+    ap.add_argument("--sum", choices=["fp32_atomic", "exact"], default=None,
+                    help="how the O / down projections are added over SMs (default: the "
+                         "library's default mode)")
     ap.add_argument("--profile", action="store_true",
                     help="run the profiling build (libkie_prof.so) and report where each "
                          "SM's time goes; its timings are not the benchmark value")
@@ -322,6 +325,9 @@ def main():
     dec = kie.Decoder(kie.make_desc(m, max_seq), wdev, stream=stream)
     if args.sync == "grid":
         dec.kie_set_sync_mode(kie.KIE_SYNC_GRID)
+    if args.sum is not None:
+        dec.kie_set_sum_mode(kie.KIE_SUM_EXACT if args.sum == "exact"
+                             else kie.KIE_SUM_FP32_ATOMIC)
     del wdev
     torch.cuda.empty_cache()
     st = dec.kie_get_stats()
@@ -357,10 +363,10 @@ def main():
     toks2 = dec.kie_decode(K)
     e2e_s = time.perf_counter() - t0
     barrier()
-    # The O/down sums (and the 8B-class LM head's) add fp32 contributions from
-    # many SMs atomically, so the last bits of the logits vary between runs
-    # and a free-running greedy decode may take a different token at a near
-    # tie; report how long the two runs agree instead of requiring equality.
+    # With fp32 atomic O/down sums the last bits of the logits vary between
+    # runs, so a free-running greedy decode may take a different token at a
+    # near tie; with exact sums the two runs are identical.  Report how
+    # long they agree.
     diff = np.nonzero(toks != toks2)[0]
     repro_prefix = int(diff[0]) if diff.size else int(K)
 
@@ -391,6 +397,7 @@ def main():
         "clocks": clk.summary(),
         "gpu_launches": 1,
         "repeat_agreement": {"tokens_equal_prefix": repro_prefix, "of": K},
+        "sum_mode": args.sum or "library default",
         "e2e": {"value": job_tokens_per_s(world, K, e2e_s * 1e3), "unit": "tokens/s",
                 "what": "decode tokens / wall time of one kie_decode(K) call into a host "
                         "array (launch, K steps, token and status copies, synchronisation)",

@@ -27,6 +27,8 @@ KIE_ERR_POISONED = -7
 KIE_ERR_NONFINITE = -8
 KIE_SYNC_DEPENDENCY = 0
 KIE_SYNC_GRID = 1
+KIE_SUM_FP32_ATOMIC = 0
+KIE_SUM_EXACT = 1
 KIE_F16 = 0
 KIE_BF16 = 1
 
@@ -92,6 +94,7 @@ def load(path: str = None) -> ctypes.CDLL:
         "kie_copy_kv": ([_P, _I, _I, _I, _I, _P, _P], _I),
         "kie_debug_set": ([_P, _I, _I], _I),
         "kie_set_sync_mode": ([_P, _I], _I),
+        "kie_set_sum_mode": ([_P, _I], _I),
         "kie_set_max_steps_per_launch": ([_P, _I], _I),
         "kie_trace_request": ([_P, _I, _I], _I),
         "kie_get_trace": ([_P, _P, _I], _I),
@@ -247,6 +250,9 @@ class Decoder:
 
     def kie_set_sync_mode(self, mode: int) -> None:
         _check(load().kie_set_sync_mode(self._h, mode))
+
+    def kie_set_sum_mode(self, mode: int) -> None:
+        _check(load().kie_set_sum_mode(self._h, mode))
 
     def kie_set_max_steps_per_launch(self, n: int) -> None:
         _check(load().kie_set_max_steps_per_launch(self._h, n))

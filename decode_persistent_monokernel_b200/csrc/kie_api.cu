@@ -98,30 +98,38 @@ struct Plan {
   std::vector<RepackJob> jobs;
   int64_t stream_bytes = 0;
   int vbuf_floats = 0, part_floats = 0, ring_slots = 0;
-  int part_atomic_off = 0;   // start of the atomic row sums inside the partials buffer
+  int rsum_off = 0;          // start of the row sums inside the partials buffer
   size_t smem = 0;
   int max_split = 0;
   int64_t weight_bytes_per_step = 0;
 };
 
-// Tile shape of a row stage whose rows have K elements (see StageShape).
-const char *make_shape(int K, int in_len, int out_len, StageShape &s) {
+// Row stage whose rows have K elements (see StageShape); the chunk width cps
+// and the row-block size R are set once the plan knows the stage's runs.
+const char *make_shape(int K, int in_len, int out_len, int norm, StageShape &s) {
   s = StageShape{};
   s.K = K;
   s.in_len = in_len;
   s.out_len = out_len;
-  // Each of the 16 consumer warps owns K/16 columns of every row and each
-  // lane 8 of those, so K/128 lanes share a row: one 16-byte load per lane
-  // covers 4096/K rows, and four of them cover R = 16384/K rows, one 32 KB
-  // tile.
-  // (K / 128 lanes share a row, so it must be a power of two)
+  s.norm = norm;
+  // a tile spans 128 cps columns (16 warps x cps 16-byte chunks), so K must
+  // be a multiple of 128; K / 128 a power of two keeps every cps choice exact
   if (K % 128 || K < 128 || K > 4096 || ((K >> 7) & ((K >> 7) - 1)))
     return "row length must be 128 times a power of two, at most 4096";
-  s.R = 16384 / K;
-  s.nseg = 1;    // one (shared-memory atomic) sum per row
-  s.rpw = 1;
+  s.nseg = 1;
   s.cps = 1;
+  s.R = kMaxRowBlock;
   return nullptr;
+}
+
+// Chunk width of a row stage whose longest run of rows with one input slice
+// (on any CTA) has `run` rows: the widest tile (most columns) whose row blocks
+// still hold such a run whole, within 4 chunks per lane and K.
+void set_row_tiling(StageShape &s, int run) {
+  int c = run <= 32 ? 4 : run <= 64 ? 2 : 1;
+  while (c > 1 && 128 * c > s.K) c >>= 1;
+  s.cps = c;
+  s.R = kMaxRowBlock / c;
 }
 
 // Tile shape of a column stage whose rows (canonical columns) have n_out
@@ -149,7 +157,6 @@ const char *make_cshape(int n_out, int in_len, StageShape &s) {
   while (R * 2 * 2 * n_out <= kSlotBytes && R < 64) R *= 2;
   s.R = R;
   if ((R + s.nseg - 1) / s.nseg > 8) return "split projection tile has more than 8 rows per thread";
-  s.rpw = 1;
   return nullptr;
 }
 
@@ -168,7 +175,7 @@ void cut_blocks(const std::vector<Piece> &pieces, int r0, int r1, bool up, int l
       B.in_off = pc.in_off;
       B.tile0 = tile;
       B.out_off = pc.trans ? pc.out_off : pc.out_off + (a - base);
-      tile += (B.nrows + sh.R - 1) / sh.R;
+      if (sh.cols) tile += (B.nrows + sh.R - 1) / sh.R;
       blk.push_back(B);
       Piece one = pc;
       one.rows = b - a;
@@ -180,6 +187,23 @@ void cut_blocks(const std::vector<Piece> &pieces, int r0, int r1, bool up, int l
   }
 }
 
+// Runs of consecutive output blocks with one input slice (a row stage's local
+// rows are in block order).
+std::vector<std::pair<int, int>> input_runs(const std::vector<Block> &blk) {
+  std::vector<std::pair<int, int>> runs;   // (first local row, rows)
+  for (size_t i = 0; i < blk.size();) {
+    size_t j = i + 1;
+    int n = blk[i].nrows;
+    while (j < blk.size() && blk[j].in_off == blk[i].in_off && blk[j].lrow0 == blk[i].lrow0 + n) {
+      n += blk[j].nrows;
+      ++j;
+    }
+    runs.push_back({blk[i].lrow0, n});
+    i = j;
+  }
+  return runs;
+}
+
 const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Plan &P) {
   const Layout Ly = make_layout(m);
   const int nl = m.n_lanes, d = m.d_model, dh = m.head_dim;
@@ -188,28 +212,26 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
   const bool lanes = nl > 1;
   P.n_ctas = n_ctas;
   const char *err = nullptr;
-  if ((err = make_shape(dl, d, (m.n_heads + 2 * Hkv) * dh, P.shape[ST_QKV])) ||
+  if ((err = make_shape(dl, d, (m.n_heads + 2 * Hkv) * dh, dl, P.shape[ST_QKV])) ||
       (err = make_cshape(dl, m.n_heads * dh, P.shape[ST_O])) ||
-      (err = make_shape(dl, d, m.ffn_dim, P.shape[ST_GU])) ||
+      (err = make_shape(dl, d, m.ffn_dim, dl, P.shape[ST_GU])) ||
       (err = make_cshape(dl, m.ffn_dim, P.shape[ST_D])) ||
-      (err = make_shape(d, d, d, P.shape[ST_MIX])) ||
-      (err = make_shape(d, d, m.vocab, P.shape[ST_LM])))
+      (err = make_shape(d, d, d, 0, P.shape[ST_MIX])) ||
+      (err = make_shape(d, d, m.vocab, d, P.shape[ST_LM])))
     return err;
   auto lane0 = [&](int ln) { return Ly.layer0 + int64_t(ln) * Ly.lane_stride; };
 
+  // ---- pass 1: each CTA's rows of each stage, as output blocks
   P.stage_cta.assign(size_t(ST_COUNT) * n_ctas, StageCta{});
-  std::vector<std::vector<Piece>> src_of_cta(n_ctas);
-  P.cta_blk_begin.assign(n_ctas + 1, 0);
-  int part_max = 4;
-  int max_local[ST_COUNT] = {};   // most output rows of a row stage on one CTA
+  std::vector<std::vector<Block>> oblk(size_t(ST_COUNT) * n_ctas);
+  std::vector<std::vector<Piece>> osrc(size_t(ST_COUNT) * n_ctas);
+  int longest_run[ST_COUNT] = {};
   for (int c = 0; c < n_ctas; ++c) {
-    P.cta_blk_begin[c] = int(P.blocks.size());
-    int local_blk = 0;
     const int g = c % Hkv, sidx = c / Hkv, ng = (n_ctas - 1 - g) / Hkv + 1;
     const int ln_g = g / hkv;   // lane of KV head g (0 for dense models)
     for (int k = 0; k < ST_COUNT; ++k) {
-      StageCta &sc = P.stage_cta[size_t(k) * n_ctas + c];
       if (k == ST_MIX && !lanes) continue;
+      StageCta &sc = P.stage_cta[size_t(k) * n_ctas + c];
       const StageShape &sh = P.shape[k];
       std::vector<Piece> pieces;
       int r0 = 0, r1 = 0;
@@ -260,64 +282,110 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
       }
       sc.row0 = r0;
       sc.nout = r1 - r0;
-      sc.blk_begin = local_blk;
       int tile = 0;
-      std::vector<Block> blk;
-      std::vector<Piece> src;
+      std::vector<Block> &blk = oblk[size_t(k) * n_ctas + c];
+      std::vector<Piece> &src = osrc[size_t(k) * n_ctas + c];
       cut_blocks(pieces, r0, r1, false, 0, sh, tile, blk, src);
       if (k == ST_GU) cut_blocks(pieces, r0, r1, true, sc.nout, sh, tile, blk, src);
       sc.nlocal = (k == ST_GU) ? 2 * sc.nout : sc.nout;
-      sc.ntiles = tile;
-      sc.nblk = int(blk.size());
-      // a row stage whose blocks read one input slice and fill consecutive
-      // local rows is tiled as one run (fewer partial tiles and restarts)
-      if (!sh.cols && blk.size() > 1) {
-        bool m = true;
-        int n = 0;
-        for (const Block &B : blk) {
-          m = m && B.in_off == blk[0].in_off && B.lrow0 == blk[0].lrow0 + n;
-          n += B.nrows;
-        }
-        if (m && n == sc.nlocal && blk[0].lrow0 == 0) {
-          sc.merged = 1;
-          sc.ntiles = (n + sh.R - 1) / sh.R;
-        }
+      if (sh.cols) {
+        sc.ntiles = tile;
+        if (sc.nlocal > kMaxLocal) return "too many split-projection rows per CTA";
+      } else {
+        for (auto &r : input_runs(blk)) longest_run[k] = std::max(longest_run[k], r.second);
+        if (k != ST_LM && sc.nlocal > kMaxRowSums) return "too many rows of a row stage per CTA";
       }
+      if (k == ST_GU && sc.nout > kMaxLocal) return "hidden slice per CTA too large";
       int64_t bytes = 0;
       for (const Block &B : blk) bytes += int64_t(B.nrows) * sh.K * 2;
       sc.bytes = bytes;
-      if (!sh.cols) max_local[k] = std::max(max_local[k], sc.nlocal);
-      if (sh.cols && sc.nlocal > kMaxLocal) return "too many split-projection rows per CTA";
-      if (k == ST_GU && sc.nout > kMaxLocal) return "hidden slice per CTA too large";
-      for (size_t i = 0; i < blk.size(); ++i) {
-        P.blocks.push_back(blk[i]);
-        src_of_cta[c].push_back(src[i]);
-      }
-      local_blk += int(blk.size());
     }
-    if (local_blk > kMaxBlocksPerCta) return "too many row blocks per CTA for this shape";
   }
-  P.cta_blk_begin[n_ctas] = int(P.blocks.size());
+  for (int k = 0; k < ST_COUNT; ++k)
+    if (!P.shape[k].cols) set_row_tiling(P.shape[k], longest_run[k]);
 
-  // per-CTA streams in consumption order, and the repack jobs that fill them
+  // ---- pass 2: per CTA, its output blocks and row blocks; the streams in
+  // consumption order and the repack jobs that fill them
+  P.cta_blk_begin.assign(n_ctas + 1, 0);
+  int rsum_max = 4;
   int64_t off = 0;
   for (int c = 0; c < n_ctas; ++c) {
+    P.cta_blk_begin[c] = int(P.blocks.size());
+    int local_blk = 0;
+    std::vector<std::vector<Block>> rblk(ST_COUNT);
+    for (int k = 0; k < ST_COUNT; ++k) {
+      StageCta &sc = P.stage_cta[size_t(k) * n_ctas + c];
+      const StageShape &sh = P.shape[k];
+      const std::vector<Block> &blk = oblk[size_t(k) * n_ctas + c];
+      sc.blk_begin = local_blk;
+      sc.nblk = int(blk.size());
+      for (const Block &B : blk) P.blocks.push_back(B);
+      local_blk += sc.nblk;
+      if (sh.cols || (k == ST_MIX && !lanes)) continue;
+      // row blocks: each run of one input slice cut into equal parts of <= R rows
+      const int kb = 128 * sh.cps, nk = sh.K / kb;
+      int tile = 0;
+      for (auto &r : input_runs(blk)) {
+        const int nb = (r.second + sh.R - 1) / sh.R;
+        for (int b = 0; b < nb; ++b) {
+          Block R{};
+          R.lrow0 = r.first + int(int64_t(r.second) * b / nb);
+          R.nrows = r.first + int(int64_t(r.second) * (b + 1) / nb) - R.lrow0;
+          R.in_off = blk[0].in_off;
+          for (const Block &B : blk)
+            if (R.lrow0 >= B.lrow0 && R.lrow0 < B.lrow0 + B.nrows) R.in_off = B.in_off;
+          R.tile0 = tile;
+          tile += nk;
+          rblk[k].push_back(R);
+        }
+      }
+      sc.rb_begin = local_blk;
+      sc.nrb = int(rblk[k].size());
+      sc.ntiles = tile;
+      for (const Block &R : rblk[k]) P.blocks.push_back(R);
+      local_blk += sc.nrb;
+      if (k != ST_LM) rsum_max = std::max(rsum_max, sc.nlocal);
+    }
+    if (local_blk > kMaxBlocksPerCta) return "too many row blocks per CTA for this shape";
+
     P.cta_stream_off.push_back(off);
     auto emit = [&](int k, int64_t layer_off) {
       const StageCta &sc = P.stage_cta[size_t(k) * n_ctas + c];
       const StageShape &sh = P.shape[k];
-      for (int b = 0; b < sc.nblk; ++b) {
-        const Block &B = P.blocks[P.cta_blk_begin[c] + sc.blk_begin + b];
-        const Piece &pc = src_of_cta[c][sc.blk_begin + b];
-        RepackJob j{};
-        j.src_elem = pc.src + layer_off;
-        j.dst_byte = off;
-        j.nrows = B.nrows;
-        j.K = sh.K;
-        j.trans = pc.trans;
-        j.src_ld = pc.ld;
-        P.jobs.push_back(j);
-        off += int64_t(B.nrows) * sh.K * 2;
+      const std::vector<Block> &blk = oblk[size_t(k) * n_ctas + c];
+      const std::vector<Piece> &src = osrc[size_t(k) * n_ctas + c];
+      if (sh.cols) {
+        for (int b = 0; b < sc.nblk; ++b) {
+          RepackJob j{};
+          j.src_elem = src[b].src + layer_off;
+          j.dst_byte = off;
+          j.nrows = blk[b].nrows;
+          j.K = sh.K;
+          j.trans = src[b].trans;
+          j.src_ld = src[b].ld;
+          P.jobs.push_back(j);
+          off += int64_t(blk[b].nrows) * sh.K * 2;
+        }
+        return;
+      }
+      // a row block's tiles, filled from the output blocks that hold its rows
+      for (const Block &R : rblk[k]) {
+        for (int b = 0; b < sc.nblk; ++b) {
+          const Block &B = blk[b];
+          const int lo = std::max(R.lrow0, B.lrow0), hi = std::min(R.lrow0 + R.nrows, B.lrow0 + B.nrows);
+          if (lo >= hi) continue;
+          RepackJob j{};
+          j.src_elem = src[b].src + layer_off + int64_t(lo - B.lrow0) * sh.K;
+          j.dst_byte = off;
+          j.nrows = hi - lo;
+          j.K = sh.K;
+          j.trans = 2;
+          j.rb = R.nrows;
+          j.rb0 = lo - R.lrow0;
+          j.kb = 128 * sh.cps;
+          P.jobs.push_back(j);
+        }
+        off += int64_t(R.nrows) * sh.K * 2;
       }
     };
     for (int l = 0; l < m.n_layers; ++l) {
@@ -332,10 +400,11 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
     emit(ST_LM, 0);
     off = (off + 255) / 256 * 256;
   }
+  P.cta_blk_begin[n_ctas] = int(P.blocks.size());
   P.stream_bytes = off;
 
   // shared memory: staging / attention scratch, partial sums, ring
-  int vb = 2 * d;   // normalised input and its gains
+  int vb = d;       // staged input of a row stage
   vb = std::max(vb, (G + 2) * dh + kConsumerWarps * G * (dh + 2));   // attention scratch
   vb = std::max(vb, G * std::min((n_ctas + Hkv - 1) / Hkv, kMaxSplit) * (dh + 2));  // group partials
   for (int g = 0; g < Hkv; ++g) {   // merge staging: (m, l) of every split + own output columns
@@ -346,21 +415,11 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
   for (int k : {int(ST_O), int(ST_D)})                               // column-stage phases
     vb = std::max(vb, P.shape[k].nseg * P.shape[k].K);
   P.vbuf_floats = (vb + 3) / 4 * 4;
-  // Row-stage sums: 16 per-warp partials per row (plain stores, added in a
-  // fixed order by the epilogue) when they fit kPartialFloats, else one
-  // shared-memory atomic accumulator per row.
-  // The two kinds live in disjoint regions: the atomic sums must be zero on
-  // entry (their readers clear them), the partials are overwritten each time.
-  int partial_max = 0, atomic_max = 0;
-  for (int k = 0; k < ST_COUNT; ++k) {
-    if (P.shape[k].cols) continue;
-    P.shape[k].nseg = max_local[k] * kConsumerWarps <= kPartialFloats ? kConsumerWarps : 1;
-    if (P.shape[k].nseg > 1) partial_max = std::max(partial_max, max_local[k] * kConsumerWarps);
-    else atomic_max = std::max(atomic_max, max_local[k]);
-  }
-  P.part_atomic_off = (partial_max + 3) / 4 * 4;
-  part_max = std::max(part_max, P.part_atomic_off + atomic_max);
-  P.part_floats = (part_max + 3) / 4 * 4;
+  // row stages: the 16 warps' partial sums of two row blocks, then the row
+  // sums of the stage (every row stage but the LM head, whose epilogue runs
+  // per row block)
+  P.rsum_off = kPartialFloats;
+  P.part_floats = (kPartialFloats + rsum_max + 3) / 4 * 4;
   const size_t fixed = monokernel_smem_bytes(0, P.vbuf_floats, P.part_floats);
   if (fixed + 3 * (kSlotBytes + 16) > smem_cap) return "shape needs more shared memory than the SM has";
   int slots = int((smem_cap - fixed) / (kSlotBytes + 16));
@@ -373,6 +432,7 @@ const char *build_plan(const kie_model_desc &m, int n_ctas, size_t smem_cap, Pla
   P.ring_slots = slots;
   P.smem = monokernel_smem_bytes(slots, P.vbuf_floats, P.part_floats);
   P.max_split = std::min((n_ctas + Hkv - 1) / Hkv, kMaxSplit);
+
 
   // weights streamed by one decode step: all matrices, norms, one embedding row
   P.weight_bytes_per_step = (Ly.total - int64_t(m.vocab) * d + d) * 2;
@@ -393,6 +453,7 @@ struct kie_ctx {
   uint64_t watchdog_ns = 2000000000ull;
   int skip_signal_cta = -1;
   int grid_sync = 0;
+  int det_sum = 0;            // KIE_SUM_EXACT: order-independent O / down sums
   int max_launch_steps = 0;   // 0: the counters' own limit (steps_per_launch)
   // L2 look-ahead of the weight producer while its ring is full (KIE_L2PF_TILES,
   // KIE_L2PF_DELAY, KIE_L2PF_PACE): most tiles, cycles before, cycles between
@@ -577,7 +638,7 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
   size_t o = 0;
   auto take = [&](size_t n) { size_t r = o; o += (n + 63) / 64 * 64; return r; };
   ctx->off_xres = take(size_t(2) * d);
-  ctx->off_acc = take(size_t(4) * d);   // acc_o[2][d] then acc_d[2][d]
+  ctx->off_acc = take(size_t(8) * d);   // acc_o[2][d] then acc_d[2][d], each with room for lo sums
   ctx->off_qkv = take(size_t(m.n_heads + 2 * m.n_kv_heads) * dh);
   ctx->off_dsum = take(size_t(std::max(1, m.lane_delay)) * d);
   ctx->off_part = take(size_t(m.n_heads) * P.max_split * (dh + 2));
@@ -718,7 +779,7 @@ static int launch_steps(kie_ctx *ctx, const KernelArgs &a, size_t sync_bytes, in
     if (a.trace && a.trace_step >= s0 && a.trace_step < s0 + c) b.trace_step = a.trace_step - s0;
     else b.trace = nullptr;
     CK(cudaMemsetAsync(a.sync, 0, sync_bytes, st));
-    CK(cudaMemsetAsync(a.acc_o, 0, size_t(4) * ctx->m.d_model * 4, st));   // both accumulators, both parities
+    CK(cudaMemsetAsync(a.acc_o, 0, size_t(8) * ctx->m.d_model * 4, st));   // both accumulators, both parities
     CK(cudaMemsetAsync(b.keys, 0, size_t(c) * 8, st));
     if (s0 == 0) CK(cudaEventRecord(ctx->ev0, st));
     void *args[] = {&b};
@@ -761,7 +822,7 @@ static KernelArgs fill_args(kie_ctx *ctx, int pos0, int n, int first_token,
   a.max_seq = m.max_seq;
   a.n_ctas = P.n_ctas; a.ring_slots = P.ring_slots;
   a.vbuf_floats = P.vbuf_floats; a.part_floats = P.part_floats;
-  a.part_atomic_off = P.part_atomic_off;
+  a.rsum_off = P.rsum_off;
   for (int k = 0; k < ST_COUNT; ++k) a.shape[k] = P.shape[k];
   a.stage_cta = ctx->d_stage_cta; a.blocks = ctx->d_blocks;
   a.cta_blk_begin = ctx->d_blk_begin; a.cta_stream_off = ctx->d_stream_off;
@@ -777,6 +838,7 @@ static KernelArgs fill_args(kie_ctx *ctx, int pos0, int n, int first_token,
   a.skip_signal_cta = ctx->skip_signal_cta;
   ctx->skip_signal_cta = -1;
   a.grid_sync = ctx->grid_sync;
+  a.det_sum = ctx->det_sum;
   a.l2pf_tiles = ctx->l2pf_tiles; a.l2pf_delay = ctx->l2pf_delay; a.l2pf_pace = ctx->l2pf_pace;
   return a;
 }
@@ -785,7 +847,8 @@ static KernelArgs fill_args(kie_ctx *ctx, int pos0, int n, int first_token,
 // context's activation buffer).
 static void set_act(const kie_ctx *ctx, KernelArgs &a, float *act) {
   a.xres = act + ctx->off_xres;
-  a.acc_o = act + ctx->off_acc; a.acc_d = a.acc_o + 2 * size_t(ctx->m.d_model);
+  // fp32 sums take [2][d] floats per accumulator, deterministic sums [2][d] hi + [2][d] lo
+  a.acc_o = act + ctx->off_acc; a.acc_d = a.acc_o + (ctx->det_sum ? 4 : 2) * size_t(ctx->m.d_model);
   a.qkv = act + ctx->off_qkv; a.dsum = act + ctx->off_dsum;
   a.attn_part = act + ctx->off_part;
 }
@@ -964,6 +1027,12 @@ extern "C" int kie_debug_set(kie_ctx *ctx, int32_t watchdog_ms, int32_t skip_sig
 extern "C" int kie_set_max_steps_per_launch(kie_ctx *ctx, int32_t n) {
   if (!ctx || n < 0) return KIE_ERR_INVALID;
   ctx->max_launch_steps = n;
+  return KIE_OK;
+}
+
+extern "C" int kie_set_sum_mode(kie_ctx *ctx, int32_t mode) {
+  if (!ctx || (mode != KIE_SUM_FP32_ATOMIC && mode != KIE_SUM_EXACT)) return KIE_ERR_INVALID;
+  ctx->det_sum = mode == KIE_SUM_EXACT ? 1 : 0;
   return KIE_OK;
 }
 

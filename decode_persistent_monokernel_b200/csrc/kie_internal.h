@@ -73,23 +73,28 @@ enum TraceEvent : int {
 };
 constexpr int kTraceCap = 1 << 16;
 
-// Per-stage constants shared by every CTA.  A tile is R whole rows (at most
-// kSlotBytes).
-//  Row stages (QKV, GU, MIX, LM): out[row] = sum_k W[row][k] in[k], R =
-//    16384 / K rows per tile.  All consumer warps share every tile: warp w
-//    takes columns [w K/16, (w+1) K/16) of every row, each lane 8 of them in
-//    four rows; nseg = 16 keeps one partial sum per (row, warp), nseg = 1 one
-//    shared-memory atomic sum per row.
+// Per-stage constants shared by every CTA.
+//  Row stages (QKV, GU, MIX, LM): out[row] = sum_k W[row][k] in[k].  A CTA's
+//    rows of the stage are cut into row blocks of at most R = 128 / cps rows
+//    that share one input slice; a row block streams as K / (128 cps) tiles,
+//    tile t holding columns [t 128 cps, (t+1) 128 cps) of every row of the
+//    block (rows * 256 cps bytes, at most kSlotBytes), row-major, with the
+//    16-byte chunk c of row r stored at chunk position c ^ (r & 7).  Lane l
+//    of every consumer warp owns rows l, l + 32, ... of the block; warp w
+//    owns chunks [w cps, (w+1) cps) of each tile, so it accumulates its
+//    rows' partial dot products in registers over the block's tiles, and the
+//    16 warps' partials are added in a fixed order once per row block.
 //  Column stages (O, D): out[:] += sum_row s[row] W[row][:], where a row is
-//    a column of the canonical matrix.  Thread t takes row phase t / ngrp
-//    and 4-element output groups t % ngrp + ngrp * j (j < cps); nseg phases.
+//    a column of the canonical matrix; a tile is R whole rows.  Thread t takes
+//    row phase t / ngrp and 4-element output groups t % ngrp + ngrp * j
+//    (j < cps); nseg phases.
 struct StageShape {
   int32_t K;       // row length (row stages: reduction length; column stages: output length)
-  int32_t R;       // rows per tile (power of two)
-  int32_t nseg;    // row stages: partial sums kept per row (16: one per consumer warp,
-                   // 1: a shared-memory atomic sum); column stages: row phases
-  int32_t rpw;     // 1 (kept for the plan checker)
-  int32_t cps;     // column stages: 4-element output groups per thread (row stages: 1)
+  int32_t R;       // row stages: most rows of a row block; column stages: rows per tile
+  int32_t nseg;    // column stages: row phases (row stages: 1)
+  int32_t norm;    // row stages: width of the RMSNorm slices of the input (0: no norm)
+  int32_t cps;     // row stages: 16-byte chunks per lane per row of a tile (1, 2, 4);
+                   // column stages: 4-element output groups per thread
   int32_t in_len;  // length of the stage input vector
   int32_t out_len; // length of the stage output vector
   int32_t cols;    // 1 for column stages
@@ -98,42 +103,51 @@ struct StageShape {
 // One CTA's share of a stage.
 struct StageCta {
   int32_t row0, nout; // GU: hidden slice [row0, row0 + nout); MIX, LM: output rows
-  int32_t nlocal;     // local rows (partial sums of row stages, scalars of column stages)
+  int32_t nlocal;     // local rows (row sums of row stages, scalars of column stages)
   int32_t ntiles;
-  int32_t blk_begin;  // first block, counted from the CTA's own first block
+  int32_t blk_begin;  // first output block, counted from the CTA's own first block
   int32_t nblk;
   int64_t bytes;      // stream bytes of one instance of this stage
-  int32_t merged;     // 1: a row stage whose blocks share one input slice and fill
-                      // local rows 0..nlocal-1 in order, tiled as one run of nlocal rows
-  int32_t pad;
+  int32_t rb_begin;   // row stages: first row block (same numbering as blk_begin)
+  int32_t nrb;        // row stages: row blocks
 };
 
-// A run of rows of one CTA's stage with one input slice and one output place.
+// A run of rows of one CTA's stage.  Output blocks (blk_begin): rows with one
+// output place (and, for row stages, one input slice).  Row blocks of row
+// stages (rb_begin): the units the GEMV tiles, at most StageShape::R rows of
+// one input slice.
 struct Block {
   int32_t lrow0;   // first local row
   int32_t nrows;
   int32_t in_off;  // row stages: offset of the rows' input in the stage input vector
   int32_t tile0;   // index of the block's first tile within the stage
-  int32_t out_off; // row stages: output index of the first row; column stages:
-                   // offset of the block's output slice in the d-vector
+  int32_t out_off; // output blocks of row stages: output index of the first row; column
+                   // stages: offset of the block's output slice in the d-vector
   int32_t pad;
 };
 
 // Copy job of the weight repack: one block of one stage instance.
 //  trans == 0: nrows canonical rows of K elements, copied as they are;
 //  trans == 1: nrows columns of a row-major matrix with K rows and row stride
-//              src_ld, each written as one row of K elements.
+//              src_ld, each written as one row of K elements;
+//  trans == 2: nrows canonical rows of K elements (consecutive rows of one
+//              matrix), rows rb0 .. rb0 + nrows - 1 of a row block of rb rows
+//              whose tiles of kb columns start at dst_byte; chunk c (8
+//              elements) of tile row r goes to chunk position c ^ (r & 7).
 struct RepackJob {
   int64_t src_elem;  // canonical element offset of the first row (or first column's top)
   int64_t dst_byte;  // byte offset in the streaming buffer
   int32_t nrows, K, trans, src_ld;
+  int32_t rb, rb0, kb, pad;
 };
 
 constexpr int kMaxBlocksPerCta = 64;
 constexpr int kSlotBytes = 32768;  // one bulk copy per tile: >= 16 KB keeps HBM saturated
 constexpr int kConsumerWarps = 16;
 constexpr int kMaxLocal = 256;     // scalars a column stage holds per CTA
-constexpr int kPartialFloats = 4096;  // shared-memory budget of per-warp row partials
+constexpr int kMaxRowBlock = 128;  // rows of a row block (lane l: rows l + 32 j, j < 4)
+constexpr int kPartialFloats = 2 * kConsumerWarps * kMaxRowBlock;  // double-buffered warp partials
+constexpr int kMaxRowSums = 1024;  // row sums a non-LM row stage keeps per CTA
 constexpr int kMaxSplit = 32;      // CTAs that share one KV head's positions (others only merge)
 
 struct KernelArgs {
@@ -145,7 +159,7 @@ struct KernelArgs {
   int32_t max_seq;
   // plan
   int32_t n_ctas, ring_slots, vbuf_floats, part_floats;
-  int32_t part_atomic_off;      // row sums kept as shared atomics start here in `part`
+  int32_t rsum_off;             // row sums of the last row stage start here in `part`
   StageShape shape[ST_COUNT];
   const StageCta *stage_cta;  // [ST_COUNT][n_ctas]
   const Block *blocks;
@@ -161,8 +175,9 @@ struct KernelArgs {
   // state
   uint16_t *kcache, *vcache; // [L, Hkv, max_seq, dh]
   float *xres;   // [2, d] residual entering global layer G, in xres[G % 2] (row owners write it)
-  float *acc_o;  // [2, d] attention sublayer output of layer G (atomic sums; zero when reused)
-  float *acc_d;  // [2, d] MLP sublayer output of layer G
+  float *acc_o;  // [2, d] attention sublayer output of layer G (atomic sums; zero when reused);
+                 // in deterministic mode followed by [2, d] sums of the lo parts
+  float *acc_d;  // [2, d] MLP sublayer output of layer G (same storage as acc_o)
   float *qkv;    // [(Hq + 2 Hkv) dh]
   float *dsum;   // [delta, d] delayed cross-lane sums
   float *attn_part;  // [Hq, max_split, dh + 2] per-split attention partials
@@ -179,6 +194,7 @@ struct KernelArgs {
   uint64_t watchdog_ns;
   int32_t skip_signal_cta;      // test hook, -1 = off
   int32_t grid_sync;            // 1: every dependency wait is a grid-wide barrier
+  int32_t det_sum;              // 1: O / down sums split into exact hi / lo fp32 sums (order-independent)
   int32_t l2pf_tiles;           // L2 look-ahead while the ring is full: most tiles (0 = off)
   int32_t l2pf_delay;           //   SM cycles of waiting for a free slot before it starts
   int32_t l2pf_pace;            //   SM cycles between two look-ahead requests

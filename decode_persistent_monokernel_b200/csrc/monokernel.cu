@@ -115,6 +115,23 @@ __device__ __forceinline__ void red_add_v4(float *p, float4 v) {
                "f"(v.z), "f"(v.w)
                : "memory");
 }
+// Order-independent fp32 sums (deterministic mode).  A contribution v is
+// split into hi = v rounded to a multiple of 2^-8 and lo = (v - hi) rounded
+// to a multiple of 2^-25 (|lo| <= 2^-9), each added with ordinary fp32 vector
+// atomics into its own accumulator.  With fewer than 256 contributors of
+// magnitude below 256, every partial sum of the hi parts is a multiple of
+// 2^-8 below 2^16 and every partial sum of the lo parts a multiple of 2^-25
+// below 2^-1: both fit fp32's 24-bit significand, so every addition is exact
+// and the sums do not depend on the order in which SMs add.  The value read
+// back is hi_sum + lo_sum; the rounding of lo costs at most 2^-26 absolute
+// per contribution.
+constexpr float kHiQ = 256.0f, kHiInvQ = 0.00390625f;                  // 2^8, 2^-8
+constexpr float kLoQ = 33554432.0f, kLoInvQ = 2.9802322387695312e-08f;  // 2^25, 2^-25
+__device__ __forceinline__ void split_hi_lo(float v, float &hi, float &lo) {
+  hi = rintf(v * kHiQ) * kHiInvQ;
+  lo = rintf((v - hi) * kLoQ) * kLoInvQ;
+}
+
 // Named barrier over the consumer warps only (the producer never joins).
 __device__ __forceinline__ void cbar() {
   __syncwarp();
@@ -314,17 +331,22 @@ struct Producer {
     prefetch_l2(a.vcache + row, bytes);
   }
 
-  // Issues every tile of stage k (its blocks in order); false once a wait
-  // for a free slot gave up.
+  // Issues every tile of stage k in the order the consumers take them: for a
+  // row stage, the column tiles of each row block (rows * 256 cps bytes
+  // each); for a column stage, R whole rows of each block at a time.  False
+  // once a wait for a free slot gave up.
   __device__ bool stage(int k, const uint8_t *&cur, uint32_t &slot, uint32_t &phase) {
     const StageCta &c = s.misc->sc[k];
-    const int nblk = c.nblk, b0 = c.blk_begin;
-    const int R = a.shape[k].R;
-    const uint32_t rowb = uint32_t(a.shape[k].K) * 2u;
+    const StageShape &sh = a.shape[k];
+    const bool rows = !sh.cols;
+    const int nb = rows ? c.nrb : c.nblk, b0 = rows ? c.rb_begin : c.blk_begin;
+    const uint32_t rowb = uint32_t(sh.K) * 2u;
     const uint32_t NS = a.ring_slots;
-    for (int bi = 0; bi < (c.merged ? 1 : nblk); ++bi) {
-      const int nrows = c.merged ? c.nlocal : s.misc->blk[b0 + bi].nrows;
-      for (int r0 = 0; r0 < nrows; r0 += R) {
+    const int nk = rows ? sh.K / (128 * sh.cps) : 0;
+    for (int bi = 0; bi < nb; ++bi) {
+      const int nrows = s.misc->blk[b0 + bi].nrows;
+      const int ntile = rows ? (nrows > 0 ? nk : 0) : (nrows + sh.R - 1) / sh.R;
+      for (int t = 0; t < ntile; ++t) {
         if (T >= NS) {
 #ifdef KIE_PROFILE
           const long long tw = clock64();
@@ -341,7 +363,8 @@ struct Producer {
           s.misc->prof[PF_PROD_EMPTY] += clock64() - tw;
 #endif
         }
-        const uint32_t bytes = uint32_t(min(R, nrows - r0)) * rowb;
+        const uint32_t bytes = rows ? uint32_t(nrows) * 256u * uint32_t(sh.cps)
+                                    : uint32_t(min(sh.R, nrows - t * sh.R)) * rowb;
         mbar_expect_tx(&s.full[slot], bytes);
         bulk_g2s(s.ring + size_t(slot) * kSlotBytes, cur, bytes, &s.full[slot], policy_evict_first());
         cur += bytes;
@@ -410,6 +433,7 @@ struct Consumer {
   uint32_t gl = 0;        // global layer index step * n_layers + l (parity of the buffers)
   uint32_t lm_count = 0;
   uint32_t nsig = 0;      // signals this CTA has made (grid-barrier mode)
+  uint32_t ag_rounds = 0; // split-KV attention rounds (partials exchanged in the group)
   bool tracing = false;   // profiling build: this SM records the current step
 #ifdef KIE_PROFILE
   __device__ void trace_put(int type, int arg) {
@@ -468,7 +492,30 @@ struct Consumer {
   __device__ const float4 *vec4(const float *base, uint32_t parity) const {
     return reinterpret_cast<const float4 *>(base + size_t(parity & 1u) * a.d_model);
   }
-
+  // Elements 4j..4j+3 of a layer accumulator (acc_o or acc_d) of the given
+  // parity: the fp32 sums, or in deterministic mode the hi sums plus the lo
+  // sums (stored 2 d floats further on).
+  __device__ float4 acc4(const float *base, uint32_t parity, int j) const {
+    const float4 h = __ldcg(vec4(base, parity) + j);
+    if (!a.det_sum) return h;
+    const float4 l = __ldcg(vec4(base + 2 * size_t(a.d_model), parity) + j);
+    return make_float4(h.x + l.x, h.y + l.y, h.z + l.z, h.w + l.w);
+  }
+  // Adds outputs e .. e+3 into a layer accumulator of the given parity.
+  __device__ __forceinline__ void acc_add4(float *base, uint32_t parity, int e, float4 v) const {
+    float *p = base + size_t(parity & 1u) * a.d_model + e;
+    if (!a.det_sum) {
+      red_add_v4(p, v);
+      return;
+    }
+    float4 hi, lo;
+    split_hi_lo(v.x, hi.x, lo.x);
+    split_hi_lo(v.y, hi.y, lo.y);
+    split_hi_lo(v.z, hi.z, lo.z);
+    split_hi_lo(v.w, hi.w, lo.w);
+    red_add_v4(p, hi);
+    red_add_v4(p + 2 * size_t(a.d_model), lo);
+  }
   // elements 4j..4j+3 of the residual entering the current layer (the
   // embedding row at layer 0), plus the delayed cross-lane sum landing here
   __device__ float4 xin4(int j) const {
@@ -479,8 +526,7 @@ struct Consumer {
       v = make_float4(lo.x, lo.y, hi.x, hi.y);
     } else {
       const uint32_t q = gl - 1;
-      v = add4(add4(__ldcg(vec4(a.xres, q) + j), __ldcg(vec4(a.acc_o, q) + j)),
-               __ldcg(vec4(a.acc_d, q) + j));
+      v = add4(add4(__ldcg(vec4(a.xres, q) + j), acc4(a.acc_o, q, j)), acc4(a.acc_d, q, j));
     }
     if (a.n_lanes > 1 && l >= a.lane_delay)
       v = add4(v, __ldcg(reinterpret_cast<const float4 *>(
@@ -488,20 +534,21 @@ struct Consumer {
     return v;
   }
 
-  // vbuf[0..n) = RMSNorm(src) * gain, per lane slice of width seg (a
-  // multiple of 128).  src(i4) returns elements 4*i4 .. 4*i4+3.  Each thread
-  // holds up to 4 float4 groups; warp partial sums of squares go through
-  // shared memory and every thread adds up the ones of its own slice.
-  // If own is not null, this CTA's rows [own_lo, own_hi) of the raw input are
-  // also written to own (the residual of the layer, kept by its row owners).
+  // Staging of a row stage's input: vbuf[0..n) = src(i) * gain[i] (gain may
+  // be null: no gain), and red_sq[i] = the sum of src^2 over elements
+  // [128 i, 128 i + 128), so that the mean square of any lane slice (a
+  // multiple of 128 elements) is a sum of red_sq entries.  The RMSNorm's
+  // scalar factor rsqrt(mean(x^2) + eps) commutes with the dot products and
+  // is applied to the row sums (norm_scale).  src(j) returns elements
+  // 4j .. 4j+3.  If own is not null, this CTA's rows [own_lo, own_hi) of the
+  // raw input are also written to own (the residual kept by its row owners).
   template <typename Src>
-  __device__ void stage_norm(Src src, const float *gain, int n, int seg, float *own = nullptr,
-                             int own_lo = 0, int own_hi = 0) {
+  __device__ void stage_input(Src src, const float *gain, int n, float *own = nullptr,
+                              int own_lo = 0, int own_hi = 0) {
     KP_BEGIN(t_norm);
     KT(TE_NORM_BEGIN, 0);
     const int ng = n >> 2;
     float4 *vb = reinterpret_cast<float4 *>(s.vbuf);
-    float4 *gb = vb + ng;   // the gains, staged beside the input
     for (int q = 0; q * kNC < ng; ++q) {
       const int j = tid + q * kNC;
       float ss = 0.f;
@@ -513,59 +560,27 @@ struct Consumer {
           for (int u = 0; u < 4; ++u)
             if (4 * j + u >= own_lo && 4 * j + u < own_hi) own[4 * j + u] = e[u];
         }
-        gb[j] = *reinterpret_cast<const float4 *>(gain + 4 * j);
-        vb[j] = v;
+        const float4 g = gain ? __ldg(reinterpret_cast<const float4 *>(gain) + j)
+                              : make_float4(1.f, 1.f, 1.f, 1.f);
+        vb[j] = make_float4(v.x * g.x, v.y * g.y, v.z * g.z, v.w * g.w);
         ss = v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
       }
       for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       if (lane == 0) s.misc->red_sq[q * kConsumerWarps + warp] = ss;
     }
     cbar();
-    for (int q = 0; q * kNC < ng; ++q) {
-      const int j = tid + q * kNC;
-      if (j < ng) {
-        // the slice holding element 4j covers the warps' 128-element ranges
-        // e0 / 128 .. (e0 + seg) / 128 - 1 of red_sq, which are contiguous
-        const int e0 = (4 * j) / seg * seg;
-        const int i0 = e0 >> 7, n = seg >> 7;
-        float tot = 0.f;
-        if ((n & 3) == 0) {
-          const float4 *rq = reinterpret_cast<const float4 *>(s.misc->red_sq + i0);
-          for (int i = 0; i < (n >> 2); ++i) {
-            const float4 r4 = rq[i];
-            tot += (r4.x + r4.y) + (r4.z + r4.w);
-          }
-        } else {
-          for (int i = 0; i < n; ++i) tot += s.misc->red_sq[i0 + i];
-        }
-        const float r = rsqrtf(tot / float(seg) + a.rms_eps);
-        const float4 g = gb[j];
-        const float4 v = vb[j];
-        vb[j] = make_float4(v.x * r * g.x, v.y * r * g.y, v.z * r * g.z, v.w * r * g.w);
-      }
-    }
-    cbar();
     KT(TE_NORM_END, 0);
     KP_END(t_norm, PF_STAGE);
   }
 
-  // ---- row stages: part[row] = W[row, :] . vin over the stage's tiles
-  // Warp w owns columns [w*K/16, (w+1)*K/16) of every row; lane l covers the
-  // 8 columns col0 = w*K/16 + (l % lpr)*8 (lpr = K/128 lanes per row) of rows
-  // l / lpr + q * (32 / lpr), q = 0..3, of each tile: one 16-byte shared load
-  // per q, 8 fp32 inputs in registers.  The tile after the current one is
-  // waited for and loaded before the current one's arithmetic (one-tile
-  // software pipeline, across block boundaries too); a tile's slot is
-  // released once its words have been used.  Each row's partial sums are
-  // reduced across its lpr lanes (transposed butterfly) and added into
-  // part[row] with shared-memory atomics: part must be zero on entry
-  // (rowsum_clear leaves it so).
-  struct Words4 {
-    uint4 q[4];
-  };
-  struct Inputs8 {
-    float2 v[4];
-  };
+  // rsqrt(mean(x^2) + eps) over the norm slice [in_off, in_off + seg) of the
+  // staged input (seg = 0: no norm, factor 1).
+  __device__ float norm_scale(int in_off, int seg) const {
+    if (seg == 0) return 1.f;
+    float tot = 0.f;
+    for (int i = in_off >> 7; i < (in_off + seg) >> 7; ++i) tot += s.misc->red_sq[i];
+    return rsqrtf(tot / float(seg) + a.rms_eps);
+  }
 
   // Waits (warp-wide outcome) for the weight tile in the current ring slot.
   __device__ __forceinline__ bool tile_wait(int k) {
@@ -586,272 +601,114 @@ struct Consumer {
   __device__ void slot_advance() {
     if (++slot == uint32_t(a.ring_slots)) { slot = 0; phase ^= 1u; }
   }
-  // Input of a row stage: a vector already staged in shared memory (v), or,
-  // for the dense model, RMSNorm fused into the stage: x = g0 + g1 [+ g2]
-  // (global fp32 vectors) or an embedding row, times the gains; each lane
-  // loads its own 8 elements and the sum of squares goes to red_sq[warp], so
-  // the epilogue scales the row sums by rsqrt(mean(x^2) + eps) (the norm's
-  // scalar factor commutes with the dot product).
-  struct RowInput {
-    const float *v;
-    const float *g0, *g1, *g2;
-    const uint16_t *emb;
-    const float *gain;
+
+  // ---- row stages: out(local row, (W[row, :] . vin) * norm factor)
+  // For each row block (at most 128 / C rows with one input slice): lane l
+  // takes rows l + 32 j; warp w takes the 16-byte chunks w C .. w C + C - 1 of
+  // every tile (8 C columns), found at chunk position ^ (row & 7).  A warp
+  // loads its words of a tile, hands the slot back, then does the tile's
+  // arithmetic; its rows' partial dot products stay in registers across the
+  // block's tiles (no reduction per tile, so the 16 warps working on a tile
+  // keep its short load latency covered).  At the end of the block each warp
+  // writes its partials (double-buffered by block parity), one barrier, and
+  // the block's row sums are the 16 warps' partials added in warp order
+  // (deterministic), scaled by the block's RMSNorm factor and handed to out()
+  // by thread `row`.  Ends with a barrier, so out()'s shared-memory results
+  // are visible to every consumer thread.
+  template <int C>
+  struct RowWords {
+    uint4 q[4 / C][C];
   };
-  __device__ __forceinline__ Inputs8 fused_inputs(const RowInput &in, int col0, int LSH) {
-    float e[8];
-    if (in.emb) {
-      const uint4 w = *reinterpret_cast<const uint4 *>(in.emb + col0);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = Store<T>::pair(ws[q]);
-        e[2 * q] = f.x;
-        e[2 * q + 1] = f.y;
-      }
-    } else {
-      const float4 *p0 = reinterpret_cast<const float4 *>(in.g0 + col0);
-      const float4 *p1 = reinterpret_cast<const float4 *>(in.g1 + col0);
-      float4 u0 = add4(__ldcg(p0), __ldcg(p1)), u1 = add4(__ldcg(p0 + 1), __ldcg(p1 + 1));
-      if (in.g2) {
-        const float4 *p2 = reinterpret_cast<const float4 *>(in.g2 + col0);
-        u0 = add4(u0, __ldcg(p2));
-        u1 = add4(u1, __ldcg(p2 + 1));
-      }
-      e[0] = u0.x; e[1] = u0.y; e[2] = u0.z; e[3] = u0.w;
-      e[4] = u1.x; e[5] = u1.y; e[6] = u1.z; e[7] = u1.w;
-    }
-    const float4 ga = *reinterpret_cast<const float4 *>(in.gain + col0);
-    const float4 gb = *reinterpret_cast<const float4 *>(in.gain + col0 + 4);
-    float ss = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) ss = fmaf(e[i], e[i], ss);
-    // the lanes of one row cover the warp's K/16 columns once
-    for (int o = (1 << LSH) >> 1; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) s.misc->red_sq[warp] = ss;
-    Inputs8 x;
-    x.v[0] = make_float2(e[0] * ga.x, e[1] * ga.y); x.v[1] = make_float2(e[2] * ga.z, e[3] * ga.w);
-    x.v[2] = make_float2(e[4] * gb.x, e[5] * gb.y); x.v[3] = make_float2(e[6] * gb.z, e[7] * gb.w);
-    return x;
-  }
-  // rsqrt(mean(x^2) + eps) of a fused stage's input, after the stage's barrier
-  __device__ float fused_scale(int n) const {
-    const float4 *q = reinterpret_cast<const float4 *>(s.misc->red_sq);
-    float4 v = q[0];
-#pragma unroll
-    for (int j = 1; j < kConsumerWarps / 4; ++j) v = add4(v, q[j]);
-    return rsqrtf(((v.x + v.y) + (v.z + v.w)) / float(n) + a.rms_eps);
-  }
 
-  __device__ __forceinline__ Inputs8 row_inputs(const float *vin, int in_off, int col0) const {
-    const float4 *src = reinterpret_cast<const float4 *>(vin + in_off + col0);
-    const float4 x0 = src[0], x1 = src[1];
-    Inputs8 x;
-    x.v[0] = make_float2(x0.x, x0.y); x.v[1] = make_float2(x0.z, x0.w);
-    x.v[2] = make_float2(x1.x, x1.y); x.v[3] = make_float2(x1.z, x1.w);
-    return x;
-  }
-  // The tile after (bi, t) of the stage's blocks, skipping empty blocks.
-  __device__ void next_tile(int b0, int nblk, int R, int &bi, int &t) const {
-    ++t;
-    if (t * R >= s.misc->blk[b0 + bi].nrows) { ++bi; t = 0; }
-    while (bi < nblk && s.misc->blk[b0 + bi].nrows == 0) ++bi;
-  }
-
-  __device__ void gemv(int k, const float *vin) {
-    RowInput in{};
-    in.v = vin;
-    gemv_rows(k, in);
-  }
-
-  struct Dots4 {
-    float p[4];
-  };
-  __device__ __forceinline__ Dots4 row_tile_dots(const Words4 &w, const Inputs8 &x) const {
-    Dots4 d4;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 d = dot8x2<T>(w.q[q], x.v, make_float2(0.f, 0.f));
-      d4.p[q] = d.x + d.y;
-    }
-    return d4;
-  }
-  // Reduces one tile's four dot products over the LPR lanes of each row and
-  // adds them into the rows' shared-memory sums (`rows` < R only for the last
-  // tile of a block).
-  // prow: this lane's first row of the tile in the partial sums; rstride 16
-  // (per-warp partials: prow already includes + warp) or 1 (atomic sums).
-  __device__ __forceinline__ void row_put(float *pr, float v, int rstride) {
-    if (rstride == 1) sred_add(pr, v);
-    else *pr = v;
-  }
-  __device__ __forceinline__ void row_tile_reduce(const Dots4 &d4, float *prow, int rstride, int lrow,
-                                                  int rows, bool full, int LSH) {
-    const int LPR = 1 << LSH, RPL = 32 >> LSH;
-    const float *p = d4.p;
-    KT(TE_TILE_MATH, p[0] != p[0]);
-    if (LSH == 0) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        if (full || lrow + q * RPL < rows) row_put(prow + q * RPL * rstride, p[q], rstride);
-    } else {
-      const int H = LPR >> 1;
-      const bool hi = lane & H;
-      const float s0 = __shfl_xor_sync(0xffffffffu, hi ? p[0] : p[2], H);
-      const float s1 = __shfl_xor_sync(0xffffffffu, hi ? p[1] : p[3], H);
-      const float a0 = (hi ? p[2] : p[0]) + s0;   // value 2 if hi else 0
-      const float a1 = (hi ? p[3] : p[1]) + s1;   // value 3 if hi else 1
-      const int v0 = hi ? 2 : 0;
-      if (LSH == 1) {
-        if (full || lrow + v0 * RPL < rows) row_put(prow + v0 * RPL * rstride, a0, rstride);
-        if (full || lrow + (v0 + 1) * RPL < rows) row_put(prow + (v0 + 1) * RPL * rstride, a1, rstride);
-      } else {
-        const int H2 = LPR >> 2;
-        const bool hi2 = lane & H2;
-        const float s2 = __shfl_xor_sync(0xffffffffu, hi2 ? a0 : a1, H2);
-        float v = (hi2 ? a1 : a0) + s2;           // value v0 + hi2
-        for (int o = LPR >> 3; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        const int vi = v0 + (hi2 ? 1 : 0);
-        if ((lane & (H2 - 1)) == 0 && (full || lrow + vi * RPL < rows))
-          row_put(prow + vi * RPL * rstride, v, rstride);
-      }
-    }
-  }
-
-  // Two tiles' dot products (da: tile at prow_a, db: the next tile at
-  // prow_b), reduced together over the LPR >= 8 lanes of each row: a
-  // transposed butterfly halves the values per lane at each of the first
-  // three steps (8 shuffles for 8 values with LPR = 16), then plain steps.
-  __device__ __forceinline__ void row_pair_reduce(const Dots4 &da, const Dots4 &db, float *prow_a,
-                                                  float *prow_b, int rstride, int lrow, int rows_a,
-                                                  int rows_b, int LSH) {
-    const int LPR = 1 << LSH, RPL = 32 >> LSH;
-    const int H = LPR >> 1, H2 = LPR >> 2, H3 = LPR >> 3;
-    const bool hi = lane & H, hi2 = lane & H2, hi3 = lane & H3;
-    float a4[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float keep = hi ? db.p[j] : da.p[j];        // values 4..7 if hi else 0..3
-      const float give = hi ? da.p[j] : db.p[j];
-      a4[j] = keep + __shfl_xor_sync(0xffffffffu, give, H);
-    }
-    float b2[2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const float keep = hi2 ? a4[2 + j] : a4[j];
-      const float give = hi2 ? a4[j] : a4[2 + j];
-      b2[j] = keep + __shfl_xor_sync(0xffffffffu, give, H2);
-    }
-    float v = (hi3 ? b2[1] : b2[0]) + __shfl_xor_sync(0xffffffffu, hi3 ? b2[0] : b2[1], H3);
-    for (int o = H3 >> 1; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    const int vi = (hi ? 4 : 0) + (hi2 ? 2 : 0) + (hi3 ? 1 : 0);
-    const int q = vi & 3, r = lrow + q * RPL;
-    if ((lane & (H3 - 1)) == 0) {
-      if (vi < 4) { if (r < rows_a) row_put(prow_a + q * RPL * rstride, v, rstride); }
-      else if (r < rows_b) row_put(prow_b + q * RPL * rstride, v, rstride);
-    }
-  }
-
-  // This lane's words of the tile in the current ring slot; the slot index
-  // is returned in `sl` and the ring position advanced.
-  __device__ __forceinline__ Words4 row_fetch(int k, uint32_t off0, int lrow, int rows, bool full,
-                                              uint32_t &sl, bool &ok, int RPL) {
-    Words4 w;
+  template <int C>
+  __device__ __forceinline__ RowWords<C> row_fetch(int k, int nrows, uint32_t &sl, bool &ok) {
+    constexpr int JM = 4 / C;
+    constexpr int KB2 = 256 * C;   // bytes of one tile row
+    RowWords<C> w;
     sl = slot;
     ok = ok && tile_wait(k);
-    const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes + off0;
+    const uint8_t *tile = s.ring + size_t(slot) * kSlotBytes;
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      w.q[q] = (ok && (full || lrow + q * RPL < rows)) ? *reinterpret_cast<const uint4 *>(tile + q * 8192)
-                                                      : make_uint4(0u, 0u, 0u, 0u);
+    for (int j = 0; j < JM; ++j) {
+      const int r = lane + 32 * j;
+      const bool in = ok && r < nrows;
+#pragma unroll
+      for (int cc = 0; cc < C; ++cc)
+        w.q[j][cc] = in ? *reinterpret_cast<const uint4 *>(tile + r * KB2 + (((warp * C + cc) ^ (r & 7)) << 4))
+                        : make_uint4(0u, 0u, 0u, 0u);
+    }
     slot_advance();
     return w;
   }
 
-  // Row stage (K/128 lanes per row).  Tiles of a block are processed in pairs
-  // with two register sets (no copies): the next tile is fetched before the
-  // current one's arithmetic and its slot handed back right after it.
-  __device__ void gemv_rows(int k, const RowInput &in) {
-    KP_BEGIN(t_gemv);
-    KT(TE_STAGE_BEGIN, k);
+  template <int C>
+  __device__ __forceinline__ void row_math(const RowWords<C> &w, const float *xin, float2 (&acc)[4 / C]) const {
+    constexpr int JM = 4 / C;
+#pragma unroll
+    for (int cc = 0; cc < C; ++cc) {
+      const float4 x0 = *reinterpret_cast<const float4 *>(xin + 8 * cc);
+      const float4 x1 = *reinterpret_cast<const float4 *>(xin + 8 * cc + 4);
+      const float2 xv[4] = {make_float2(x0.x, x0.y), make_float2(x0.z, x0.w),
+                            make_float2(x1.x, x1.y), make_float2(x1.z, x1.w)};
+#pragma unroll
+      for (int j = 0; j < JM; ++j) acc[j] = dot8x2<T>(w.q[j][cc], xv, acc[j]);
+    }
+  }
+
+  template <int C, typename OutF>
+  __device__ void gemv_rows_c(int k, const float *vin, OutF &out) {
+    constexpr int JM = 4 / C;
+    constexpr int KB = 128 * C;
     const StageCta &c = s.misc->sc[k];
-    const int K = a.shape[k].K, R = a.shape[k].R;
-    const int LSH = __ffs(K >> 7) - 1;         // log2 of the lanes that share a row
-    const int LPR = 1 << LSH, RPL = 32 >> LSH;
-    const int lrow = lane >> LSH;               // this lane's row within a load
-    const int col0 = warp * (K >> 4) + ((lane & (LPR - 1)) << 3);
-    const uint32_t off0 = uint32_t(lrow * K + col0) * 2u;   // + q * 8192 bytes
+    const int nk = a.shape[k].K / KB, seg = a.shape[k].norm;
     bool ok = !aborted();
-    Inputs8 xf{};
-    if (!in.v) xf = fused_inputs(in, col0, LSH);   // every block reads the whole vector
-    for (int bi = 0; bi < (c.merged ? 1 : c.nblk) && ok; ++bi) {
-      Block b = s.misc->blk[c.blk_begin + bi];
-      if (c.merged) b.nrows = c.nlocal;        // one run over all the stage's rows
-      if (b.nrows == 0) continue;
-      const Inputs8 x = in.v ? row_inputs(in.v, b.in_off, col0) : xf;
-      const int n = (b.nrows + R - 1) / R;     // tiles of the block; the last may be partial
-      const int last_rows = b.nrows - (n - 1) * R;
-      const int rstride = a.shape[k].nseg;      // 16 (per-warp partials) or 1 (atomic sums)
-      float *prow0 = rstride > 1 ? s.part + (b.lrow0 + lrow) * rstride + warp
-                                 : s.part + a.part_atomic_off + b.lrow0 + lrow;
-      uint32_t sa = 0, sb = 0;
-      Words4 wa = row_fetch(k, off0, lrow, n == 1 ? last_rows : R, n > 1, sa, ok, RPL);
-      if (ok) release_slot(sa);
-      for (int t = 0; t < n && ok; t += 2) {
-        // tile t in wa (released), tile t + 1 into wb
-        const bool has_b = t + 1 < n;
-        const bool b_full = t + 1 < n - 1;
-        const int rows_a = t < n - 1 ? R : last_rows, rows_b = b_full ? R : last_rows;
-        Words4 wb{};
-        if (has_b) wb = row_fetch(k, off0, lrow, rows_b, b_full, sb, ok, RPL);
-        // slots go back before the row sums are written (shared atomics in one
-        // mode), whose completion the arrive's release semantics would wait for
-        const Dots4 da = row_tile_dots(wa, x);
-        if (has_b && ok) release_slot(sb);
-        if (!has_b || !ok) {
-          row_tile_reduce(da, prow0 + t * R * rstride, rstride, lrow, rows_a, rows_a == R, LSH);
-          KT(TE_TILE_DONE, 0);
-          break;
-        }
-        // tile t + 1 in wb (released), tile t + 2 into wa
-        const bool has_a = t + 2 < n;
-        const bool a2_full = t + 2 < n - 1;
-        if (has_a) wa = row_fetch(k, off0, lrow, a2_full ? R : last_rows, a2_full, sa, ok, RPL);
-        const Dots4 db = row_tile_dots(wb, x);
-        if (has_a && ok) release_slot(sa);
-        if (LSH >= 3) {
-          row_pair_reduce(da, db, prow0 + t * R * rstride, prow0 + (t + 1) * R * rstride, rstride, lrow,
-                          rows_a, rows_b, LSH);
-        } else {
-          row_tile_reduce(da, prow0 + t * R * rstride, rstride, lrow, rows_a, rows_a == R, LSH);
-          row_tile_reduce(db, prow0 + (t + 1) * R * rstride, rstride, lrow, rows_b, b_full, LSH);
-        }
+    for (int rb = 0; rb < c.nrb; ++rb) {
+      const Block b = s.misc->blk[c.rb_begin + rb];
+      const float *xw = vin + b.in_off + warp * 8 * C;   // this warp's columns of tile 0
+      float2 acc[JM];
+#pragma unroll
+      for (int j = 0; j < JM; ++j) acc[j] = make_float2(0.f, 0.f);
+      for (int t = 0; t < nk && ok; ++t) {
+        uint32_t sl = 0;
+        const RowWords<C> w = row_fetch<C>(k, b.nrows, sl, ok);
+        if (!ok) break;
+        release_slot(sl);
+        row_math<C>(w, xw + t * KB, acc);
         KT(TE_TILE_DONE, 0);
+      }
+      float *pb = s.part + (rb & 1) * (kConsumerWarps * kMaxRowBlock);
+#pragma unroll
+      for (int j = 0; j < JM; ++j)
+        if (lane + 32 * j < b.nrows) pb[warp * kMaxRowBlock + lane + 32 * j] = acc[j].x + acc[j].y;
+      cbar();
+      if (tid < b.nrows) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) v += pb[w * kMaxRowBlock + tid];
+        out(b.lrow0 + tid, v * norm_scale(b.in_off, seg));
       }
     }
     if (!ok) s.misc->abort = 1;
-    Tbase += c.ntiles;
     cbar();
+  }
+
+  template <typename OutF>
+  __device__ void gemv_rows(int k, const float *vin, OutF &&out) {
+    KP_BEGIN(t_gemv);
+    KT(TE_STAGE_BEGIN, k);
+    switch (a.shape[k].cps) {
+      case 4: gemv_rows_c<4>(k, vin, out); break;
+      case 2: gemv_rows_c<2>(k, vin, out); break;
+      default: gemv_rows_c<1>(k, vin, out); break;
+    }
+    Tbase += s.misc->sc[k].ntiles;
     KT(TE_STAGE_END, k);
     KP_END(t_gemv, k == ST_LM ? PF_LM : PF_GEMV);
     KP_END(t_gemv, PF_GEMV_K + k);
   }
 
-  // Sum of row i of the last row stage (its shared-memory accumulator), which
-  // is cleared for the next stage.  Each row is read by exactly one thread.
-  __device__ float rowsum(int k, int i) const {
-    if (a.shape[k].nseg == 1) {
-      float *p = s.part + a.part_atomic_off + i;
-      const float v = *p;
-      *p = 0.f;
-      return v;
-    }
-    const float4 *q = reinterpret_cast<const float4 *>(s.part + i * kConsumerWarps);
-    float4 v = q[0];
-#pragma unroll
-    for (int j = 1; j < kConsumerWarps / 4; ++j) v = add4(v, q[j]);
-    return (v.x + v.y) + (v.z + v.w);
-  }
+  // Row sums of the last non-LM row stage, kept in shared memory.
+  __device__ float *rsum() const { return s.part + a.rsum_off; }
 
   // ---- attention over the cache for one KV head group (split-KV)
   // Positions of this CTA's split: [j0, j1) of 0..p.  Each warp folds
@@ -899,23 +756,18 @@ struct Consumer {
     KP_END(t_attn, PF_ATTN);
   }
 
-  __device__ void attention_body() {
+  // RoPE of this step's q (scaled by 1/sqrt(dh)) and k, k and v rounded to
+  // the cache type (the current token uses the rounded values too), into
+  // shared memory: qs [G][dh], kcur [dh], vcur [dh] at the start of vbuf.
+  // The writer also stores position p's K/V in the cache.  Ends with a
+  // barrier.
+  __device__ void attn_prologue(bool writer) {
     const int dh = a.head_dim, half = dh >> 1;
     const int Hkv = a.n_kv_heads, G = a.n_heads / a.n_kv_heads;
     const int g = cta % Hkv;
-    const int ngroup = (a.n_ctas - 1 - g) / Hkv + 1;      // CTAs of this KV group
-    int j0, j1, split, nsplit;
-    kv_range(j0, j1, split, nsplit);
-    // the first cached rows (already pulled into L2 by the producer) are
-    // requested together with this step's q/k/v
-    KvWords kw;
-    kv_load(kw, j0 + warp, j1);
-    const bool active = split < nsplit;
-    const bool writer = (split == nsplit - 1);  // its range holds position p
-    float *qs = s.vbuf;              // [G][dh] roped, scaled queries
-    float *kcur = qs + G * dh;       // [dh] roped, rounded key of position p
-    float *vcur = kcur + dh;         // [dh] rounded value of position p
-    float *wst = vcur + dh;          // [W][G][dh + 2] per-warp softmax states
+    float *qs = s.vbuf;
+    float *kcur = qs + G * dh;
+    float *vcur = kcur + dh;
     const float *qkv = a.qkv;
     const float2 *cs = a.rope_cs + size_t(p) * half;
     const size_t cache_row = ((size_t(l) * Hkv + g) * a.max_seq + p) * dh;
@@ -943,6 +795,26 @@ struct Consumer {
       }
     }
     cbar();
+  }
+
+  __device__ void attention_body() {
+    const int dh = a.head_dim, half = dh >> 1;
+    const int Hkv = a.n_kv_heads, G = a.n_heads / a.n_kv_heads;
+    const int g = cta % Hkv;
+    const int ngroup = (a.n_ctas - 1 - g) / Hkv + 1;      // CTAs of this KV group
+    int j0, j1, split, nsplit;
+    kv_range(j0, j1, split, nsplit);
+    // the first cached rows (already pulled into L2 by the producer) are
+    // requested together with this step's q/k/v
+    KvWords kw;
+    kv_load(kw, j0 + warp, j1);
+    const bool active = split < nsplit;
+    const bool writer = (split == nsplit - 1);  // its range holds position p
+    float *qs = s.vbuf;              // [G][dh] roped, scaled queries
+    float *kcur = qs + G * dh;       // [dh] roped, rounded key of position p
+    float *vcur = kcur + dh;         // [dh] rounded value of position p
+    float *wst = vcur + dh;          // [W][G][dh + 2] per-warp softmax states
+    attn_prologue(writer);
     // Online softmax, kU positions per iteration: their score reductions are
     // independent and one rescale covers them.  The next iteration's rows are
     // requested before this one's arithmetic.
@@ -1057,8 +929,9 @@ struct Consumer {
     // group loads all of them into shared memory (one coalesced pass) and
     // merges them (log-sum-exp) into the group's attention output
     KT(TE_ATTN, 2);
+    ++ag_rounds;
     signal(SY_QG0 + Hkv + g);
-    if (!gate(SY_QG0 + Hkv + g, (gl + 1) * uint32_t(ngroup), 0x28, 5)) return;
+    if (!gate(SY_QG0 + Hkv + g, ag_rounds * uint32_t(ngroup), 0x28, 5)) return;
     // This SM's O projection reads only the merged outputs [r0, r0 + nr) of
     // the group's G*dh: stage every split's (m, l) and those output columns.
     const int r0 = s.misc->sc[ST_O].row0, nr = s.misc->sc[ST_O].nout;
@@ -1131,9 +1004,10 @@ struct Consumer {
     return cw;
   }
 
-  __device__ void gemv_cols(int k, const float *svals, float *acc) {
-    if (a.shape[k].cps == 1) gemv_cols_impl<1>(k, svals, acc);
-    else gemv_cols_impl<2>(k, svals, acc);
+  // acc: the accumulator (acc_o or acc_d); parity: the layer's half of it
+  __device__ void gemv_cols(int k, const float *svals, float *acc, uint32_t parity) {
+    if (a.shape[k].cps == 1) gemv_cols_impl<1>(k, svals, acc, parity);
+    else gemv_cols_impl<2>(k, svals, acc, parity);
   }
 
   // Accumulates one tile (its rows ph, ph + nseg, ...) into acc2.
@@ -1165,7 +1039,7 @@ struct Consumer {
   }
 
   template <int CPS>
-  __device__ void gemv_cols_impl(int k, const float *svals, float *acc) {
+  __device__ void gemv_cols_impl(int k, const float *svals, float *acc, uint32_t parity) {
     KP_BEGIN(t_gemv);
     KT(TE_STAGE_BEGIN, k);
     const StageShape sh = a.shape[k];
@@ -1206,13 +1080,12 @@ struct Consumer {
         KT(TE_TILE_DONE, 0);
       }
       // the block is complete: add its groups into the accumulator
-      float *dst = acc + b.out_off;
       if (sh.nseg == 1) {
         if (ok) {
 #pragma unroll
           for (int j = 0; j < CPS; ++j)
-            red_add_v4(dst + 4 * (gi + tpr * j),
-                       make_float4(acc2[j][0].x, acc2[j][0].y, acc2[j][1].x, acc2[j][1].y));
+            acc_add4(acc, parity, b.out_off + 4 * (gi + tpr * j),
+                     make_float4(acc2[j][0].x, acc2[j][0].y, acc2[j][1].x, acc2[j][1].y));
         }
       } else {
         // several row phases: add them up in shared memory first (CPS == 1)
@@ -1222,7 +1095,7 @@ struct Consumer {
         if (tid < ngrp && !aborted()) {
           float4 v = scr[tid];
           for (int q = 1; q < sh.nseg; ++q) v = add4(v, scr[q * ngrp + tid]);
-          red_add_v4(dst + 4 * tid, v);
+          acc_add4(acc, parity, b.out_off + 4 * tid, v);
         }
         cbar();
       }
@@ -1236,19 +1109,19 @@ struct Consumer {
   }
 
   // ---- LM head epilogue: logits and the CTA's share of the argmax
-  __device__ void lm_epilogue(float sc) {
+  // lm_row() takes each logit as its row block is reduced (thread `row` of the
+  // block); lm_fold() then folds the threads' (value, index) pairs into one
+  // packed key per step.  bidx starts at a row of this CTA so that the key
+  // always names a valid token; a NaN logit never wins a comparison and
+  // raises DE_NONFINITE.
+  __device__ __forceinline__ void lm_row(int i, float v, float &best, int &bidx) {
+    const int row = s.misc->sc[ST_LM].row0 + i;
+    if (a.logits_out) a.logits_out[size_t(step) * a.vocab + row] = v;
+    if (v != v) raise_error(a, DE_NONFINITE | (uint32_t(step & 0xffff) << 8));
+    if (v > best || (v == best && row < bidx)) { best = v; bidx = row; }
+  }
+  __device__ void lm_fold(float best, int bidx) {
     const StageCta &c = s.misc->sc[ST_LM];
-    // bidx starts at a row of this CTA so that the key always names a valid
-    // token; a NaN logit never wins a comparison and raises DE_NONFINITE.
-    float best = -INFINITY;
-    int bidx = c.row0;
-    for (int i = tid; i < c.nout; i += kNC) {
-      const float v = sc * rowsum(ST_LM, i);
-      const int row = c.row0 + i;
-      if (a.logits_out) a.logits_out[size_t(step) * a.vocab + row] = v;
-      if (v != v) raise_error(a, DE_NONFINITE | (uint32_t(step & 0xffff) << 8));
-      if (v > best || (v == best && row < bidx)) { best = v; bidx = row; }
-    }
     for (int o = 16; o; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, best, o);
       const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
@@ -1304,63 +1177,42 @@ struct Consumer {
         KT(TE_LAYER, l & 15);
         const uint32_t cur = gl & 1u, prev = (gl - 1) & 1u;
         // ---------------- RMSNorm + q/k/v rows of the group
-        // (every CTA's down contribution to the previous layer is in)
+        // (every CTA's down contribution to the previous layer is in); the
+        // residual entering the layer is staged, its owners keep their rows
         if (gl > 0 && !gate(SY_S2, gl * nc, 0x10, 1)) goto done;
-        if (lanes) {
-          stage_norm([=](int j) { return xin4(j); }, a.gain_attn + size_t(l) * d, d, a.lane_width,
-                     a.xres + size_t(cur) * d, own_lo, own_hi);
-          gemv(ST_QKV, s.vbuf);
-        } else {
-          // the residual entering the layer: its owners keep their rows of it
-          RowInput in{};
-          if (l == 0) {
-            in.emb = a.embed + size_t(tok) * d;
-          } else {
-            in.g0 = a.xres + size_t(prev) * d;
-            in.g1 = a.acc_o + size_t(prev) * d;
-            in.g2 = a.acc_d + size_t(prev) * d;
-          }
-          in.gain = a.gain_attn + size_t(l) * d;
-          gemv_rows(ST_QKV, in);
-        }
-        if (aborted()) goto done;
+        stage_input([=](int j) { return xin4(j); }, a.gain_attn + size_t(l) * d, d,
+                    a.xres + size_t(cur) * d, own_lo, own_hi);
         {
           const StageCta &c = s.misc->sc[ST_QKV];
-          const float sc = lanes ? 1.f : fused_scale(d);
-          for (int bi = 0; bi < c.nblk; ++bi) {
-            const Block b = s.misc->blk[c.blk_begin + bi];
-            for (int i = tid; i < b.nrows; i += kNC) a.qkv[b.out_off + i] = sc * rowsum(ST_QKV, b.lrow0 + i);
-          }
+          auto to_qkv = [&](int i, float v) {
+            for (int bi = 0; bi < c.nblk; ++bi) {
+              const Block &o = s.misc->blk[c.blk_begin + bi];
+              if (unsigned(i - o.lrow0) < unsigned(o.nrows)) {
+                a.qkv[o.out_off + (i - o.lrow0)] = v;
+                break;
+              }
+            }
+          };
+          gemv_rows(ST_QKV, s.vbuf, to_qkv);
         }
+        if (aborted()) goto done;
         if (!(a.skip_signal_cta == cta && step == 0 && l == 0)) signal(SY_QG0 + g);
         // ---------------- delayed cross-lane sum of the previous layer
         if (lanes && l >= 1) {
-          const float4 *uo = vec4(a.acc_o, prev), *ud = vec4(a.acc_d, prev);
-          for (int j = tid; j < (d >> 2); j += kNC)
-            reinterpret_cast<float4 *>(s.vbuf)[j] = add4(__ldcg(uo + j), __ldcg(ud + j));
-          cbar();
-          gemv(ST_MIX, s.vbuf);
-          if (aborted()) goto done;
+          stage_input([=](int j) { return add4(acc4(a.acc_o, prev, j), acc4(a.acc_d, prev, j)); },
+                      nullptr, d);
           const StageCta &c = s.misc->sc[ST_MIX];
           float *dst = a.dsum + size_t((l - 1) % delta) * d;
-          for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(ST_MIX, i);
+          auto to_dsum = [&](int i, float v) { dst[c.row0 + i] = v; };
+          gemv_rows(ST_MIX, s.vbuf, to_dsum);
+          if (aborted()) goto done;
         }
-        // the residual entering the layer: its owners keep their rows of it (read
-        // by every SM only after the grid-wide wait that follows O); warp 1 does
-        // it while thread 0 waits for the group's q/k/v
-        if (!lanes && warp == 1)
-          for (int r = own_lo + lane; r < own_hi; r += 32) {
-            const size_t pr = size_t(prev) * d + r;
-            a.xres[size_t(cur) * d + r] =
-                l == 0 ? Store<T>::to_f(a.embed[size_t(tok) * d + r])
-                       : __ldcg(a.xres + pr) + __ldcg(a.acc_o + pr) + __ldcg(a.acc_d + pr);
-          }
         // ---------------- attention of the group, merged in every group CTA
         if (!gate(SY_QG0 + g, (gl + 1) * ng, 0x20, 4)) goto done;
         attention();
         if (aborted()) goto done;
         // ---------------- O projection over the group's attention outputs
-        gemv_cols(ST_O, s.svec + s.misc->sc[ST_O].row0, a.acc_o + size_t(cur) * d);
+        gemv_cols(ST_O, s.svec + s.misc->sc[ST_O].row0, a.acc_o, cur);
         if (aborted()) goto done;
         signal(SY_S1);
         // ---------------- RMSNorm + gate/up + SwiGLU of this CTA's hidden slice
@@ -1371,32 +1223,32 @@ struct Consumer {
           for (int r = own_lo + tid; r < own_hi; r += kNC) {
             a.acc_o[size_t(prev) * d + r] = 0.f;
             a.acc_d[size_t(prev) * d + r] = 0.f;
+            if (a.det_sum) {   // the lo sums, 2 d further on
+              a.acc_o[size_t(2 + prev) * d + r] = 0.f;
+              a.acc_d[size_t(2 + prev) * d + r] = 0.f;
+            }
           }
-        if (lanes) {
-          const float4 *xr = vec4(a.xres, cur), *ao = vec4(a.acc_o, cur);
-          stage_norm([=](int j) { return add4(__ldcg(xr + j), __ldcg(ao + j)); },
-                     a.gain_ffn + size_t(l) * d, d, a.lane_width);
-          gemv(ST_GU, s.vbuf);
-        } else {
-          RowInput in{};
-          in.g0 = a.xres + size_t(cur) * d;
-          in.g1 = a.acc_o + size_t(cur) * d;
-          in.gain = a.gain_ffn + size_t(l) * d;
-          gemv_rows(ST_GU, in);
+        {
+          const float4 *xr = vec4(a.xres, cur);
+          stage_input([=](int j) { return add4(__ldcg(xr + j), acc4(a.acc_o, cur, j)); },
+                      a.gain_ffn + size_t(l) * d, d);
+          float *rs = rsum();
+          auto to_rsum = [&](int i, float v) { rs[i] = v; };
+          gemv_rows(ST_GU, s.vbuf, to_rsum);
         }
         if (aborted()) goto done;
         {
           const StageCta &c = s.misc->sc[ST_GU];
-          const float sc = lanes ? 1.f : fused_scale(d);
+          const float *rs = rsum();
           float *h = s.svec + kSvecO;
           for (int i = tid; i < c.nout; i += kNC) {
-            const float gt = sc * rowsum(ST_GU, i), up = sc * rowsum(ST_GU, c.nout + i);
+            const float gt = rs[i], up = rs[c.nout + i];
             h[i] = gt / (1.f + expf(-gt)) * up;
           }
           cbar();
         }
         // ---------------- down projection over that slice
-        gemv_cols(ST_D, s.svec + kSvecO, a.acc_d + size_t(cur) * d);
+        gemv_cols(ST_D, s.svec + kSvecO, a.acc_d, cur);
         if (aborted()) goto done;
         signal(SY_S2);
       }
@@ -1407,39 +1259,35 @@ struct Consumer {
         if (!gate(SY_S2, (gl + 1) * nc, 0x60, 1)) goto done;
         if (lanes) {
           // the last layer's delayed sum, flushed before the final norm
-          const float4 *uo = vec4(a.acc_o, last), *ud = vec4(a.acc_d, last);
-          for (int j = tid; j < (d >> 2); j += kNC)
-            reinterpret_cast<float4 *>(s.vbuf)[j] = add4(__ldcg(uo + j), __ldcg(ud + j));
-          cbar();
-          gemv(ST_MIX, s.vbuf);
-          if (aborted()) goto done;
+          stage_input([=](int j) { return add4(acc4(a.acc_o, last, j), acc4(a.acc_d, last, j)); },
+                      nullptr, d);
           const StageCta &c = s.misc->sc[ST_MIX];
           float *dst = a.dsum + size_t((L - 1) % delta) * d;
-          for (int i = tid; i < c.nout; i += kNC) dst[c.row0 + i] = rowsum(ST_MIX, i);
+          auto to_dsum = [&](int i, float v) { dst[c.row0 + i] = v; };
+          gemv_rows(ST_MIX, s.vbuf, to_dsum);
+          if (aborted()) goto done;
           signal(SY_MIXF);
           if (!gate(SY_MIXF, lm_count * nc, 0x70, 2)) goto done;
         }
-        if (lanes) {
-          const float4 *xr = vec4(a.xres, last), *ao = vec4(a.acc_o, last), *ad = vec4(a.acc_d, last);
-          stage_norm(
+        {
+          const float4 *xr = vec4(a.xres, last);
+          const int li0 = lanes && L > delta ? L - delta : 0;
+          stage_input(
               [=](int j) {
-                float4 v = add4(add4(__ldcg(xr + j), __ldcg(ao + j)), __ldcg(ad + j));
-                for (int li = (L > delta ? L - delta : 0); li < L; ++li)
-                  v = add4(v, __ldcg(reinterpret_cast<const float4 *>(a.dsum + size_t(li % delta) * d) + j));
+                float4 v = add4(add4(__ldcg(xr + j), acc4(a.acc_o, last, j)), acc4(a.acc_d, last, j));
+                if (lanes)
+                  for (int li = li0; li < L; ++li)
+                    v = add4(v, __ldcg(reinterpret_cast<const float4 *>(a.dsum + size_t(li % delta) * d) + j));
                 return v;
               },
-              a.gain_final, d, d);
-          gemv(ST_LM, s.vbuf);
-        } else {
-          RowInput in{};
-          in.g0 = a.xres + size_t(last) * d;
-          in.g1 = a.acc_o + size_t(last) * d;
-          in.g2 = a.acc_d + size_t(last) * d;
-          in.gain = a.gain_final;
-          gemv_rows(ST_LM, in);
+              a.gain_final, d);
+          float best = -INFINITY;
+          int bidx = s.misc->sc[ST_LM].row0;
+          auto to_lm = [&](int i, float v) { lm_row(i, v, best, bidx); };
+          gemv_rows(ST_LM, s.vbuf, to_lm);
+          if (aborted()) goto done;
+          lm_fold(best, bidx);
         }
-        if (aborted()) goto done;
-        lm_epilogue(lanes ? 1.f : fused_scale(d));
         signal(SY_TOK);
         if (!gate(SY_TOK, lm_count * nc, 0x80, 3)) goto done;
         const unsigned long long key = __ldcg(a.keys + step);
@@ -1539,6 +1387,18 @@ __global__ void __launch_bounds__(256) repack_kernel(const uint16_t *__restrict_
     const RepackJob job = jobs[jb];
     uint16_t *out = reinterpret_cast<uint16_t *>(dst + job.dst_byte);
     const uint16_t *in = src + job.src_elem;
+    if (job.trans == 2) {
+      // rows of a row block's column tiles, 16-byte chunks swizzled by tile row
+      const int nchunk = job.K >> 3, cpt = job.kb >> 3;
+      const int64_t nvec = int64_t(job.nrows) * nchunk;
+      for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) {
+        const int i = int(v / nchunk), q = int(v - int64_t(i) * nchunk);
+        const int t = q / cpt, c = q - t * cpt, r = job.rb0 + i;
+        const int64_t e = (int64_t(t) * job.rb + r) * job.kb + int64_t(c ^ (r & 7)) * 8;
+        reinterpret_cast<uint4 *>(out)[e >> 3] = *reinterpret_cast<const uint4 *>(in + int64_t(i) * job.K + q * 8);
+      }
+      continue;
+    }
     if (!job.trans) {
       const int64_t nvec = int64_t(job.nrows) * job.K / 8;
       for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x)

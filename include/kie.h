@@ -245,6 +245,25 @@ int kie_debug_set(kie_ctx *ctx, int32_t watchdog_ms, int32_t skip_signal_cta);
 enum { KIE_SYNC_DEPENDENCY = 0, KIE_SYNC_GRID = 1 };
 int kie_set_sync_mode(kie_ctx *ctx, int32_t mode);
 
+/* How the persistent kernel adds up the O and down projections, whose
+ * outputs every SM contributes to (applies to later launches of this context):
+ *   KIE_SUM_FP32_ATOMIC (default): fp32 vector atomics.  The order in which
+ *     SMs add differs from run to run, so the last bits of the residual
+ *     stream, and of the logits, can differ between two identical calls.
+ *   KIE_SUM_EXACT: each contribution v is split into hi (v rounded to a
+ *     multiple of 2^-8) and lo (the rest, rounded to a multiple of 2^-25),
+ *     added with fp32 vector atomics into two accumulators whose partial sums
+ *     are then always exactly representable, so no addition rounds and the
+ *     sums do not depend on the order.  Two identical calls give
+ *     bit-identical logits and tokens as long as every contribution to an O
+ *     or down output is below 256 in magnitude (fewer than 256 SMs); larger
+ *     contributions are still added, without that guarantee.  The rounding of
+ *     lo costs at most 2^-26 absolute per contribution, and every O and down
+ *     output takes two vector atomics instead of one.
+ * Returns KIE_ERR_INVALID for any other mode. */
+enum { KIE_SUM_FP32_ATOMIC = 0, KIE_SUM_EXACT = 1 };
+int kie_set_sum_mode(kie_ctx *ctx, int32_t mode);
+
 /* Most decode steps one kernel launch runs (applies to later calls of this
  * context).  A call with more steps runs as several launches back to back,
  * each starting at the position and token where the previous one stopped;

@@ -1,12 +1,12 @@
 // Host-only check of the decode kernel's plan (no GPU calls): for each shape,
 // the repack copies every weight element into the per-SM streams exactly once;
 // the tiles the producer issues and the consumers take agree; the row-stage
-// lane mapping (each warp a column slice of every row, four 16-byte chunks per
-// lane per tile) and the column-stage thread mapping cover every weight once
-// and, emulated in double precision on the streamed bytes, reproduce the
-// canonical matrix-vector products of one layer; the attention splits
-// partition the positions; shared-memory budgets hold.  Built and run by
-// tests/test_plan.py.
+// mapping (row blocks of one input slice; in each column tile, lane l a row,
+// warp w a run of 16-byte chunks stored at a position swizzled by the row) and
+// the column-stage thread mapping cover every weight once and, emulated in
+// double precision on the streamed bytes, reproduce the canonical
+// matrix-vector products of one layer; the attention splits partition the
+// positions; shared-memory budgets hold.  Built and run by tests/test_plan.py.
 #include "../decode_persistent_monokernel_b200/csrc/kie_api.cu"
 #include <random>
 
@@ -21,14 +21,9 @@ static void check(kie_model_desc m, int n_ctas, const char *name) {
   printf("%s: ctas %d slots %d smem %zu vbuf %d part %d stream %.3f GB jobs %zu blocks %zu\n", name, n_ctas,
          P.ring_slots, P.smem, P.vbuf_floats, P.part_floats, P.stream_bytes / 1e9, P.jobs.size(), P.blocks.size());
   REQ(P.smem <= 232448, "smem");
-  {
-    int merged = 0;
-    for (const StageCta &sc : P.stage_cta) merged += sc.merged;
-    printf("  merged row-stage instances: %d\n", merged);
-  }
   for (int k = 0; k < ST_COUNT; ++k)
-    printf("  stage %d: K %d R %d nseg %d rpw %d cps %d cols %d\n", k, P.shape[k].K, P.shape[k].R,
-           P.shape[k].nseg, P.shape[k].rpw, P.shape[k].cps, P.shape[k].cols);
+    printf("  stage %d: K %d R %d nseg %d norm %d cps %d cols %d\n", k, P.shape[k].K, P.shape[k].R,
+           P.shape[k].nseg, P.shape[k].norm, P.shape[k].cps, P.shape[k].cols);
   const int nl = m.n_lanes, d = m.d_model, dh = m.head_dim, dl = d / nl, Hkv = m.n_kv_heads;
   const int hq = m.n_heads / nl, hkv = Hkv / nl, fl = m.ffn_dim / nl, G = m.n_heads / Hkv;
   const bool lanes = nl > 1;
@@ -40,14 +35,26 @@ static void check(kie_model_desc m, int n_ctas, const char *name) {
   std::vector<uint16_t> S(P.stream_bytes / 2, 0xdead);
   for (const RepackJob &j : P.jobs) {
     REQ(j.dst_byte % 16 == 0 && j.K % 4 == 0, "align");
-    REQ(j.dst_byte + int64_t(j.nrows) * j.K * 2 <= P.stream_bytes, "dst range");
+    if (j.trans == 2) {
+      REQ(j.kb % 128 == 0 && j.K % j.kb == 0 && j.rb0 + j.nrows <= j.rb && j.rb <= kMaxRowBlock, "tiled job shape");
+      REQ(j.dst_byte + int64_t(j.rb) * j.K * 2 <= P.stream_bytes, "dst range");
+      REQ(j.src_elem % 8 == 0, "tiled job alignment");
+    } else {
+      REQ(j.dst_byte + int64_t(j.nrows) * j.K * 2 <= P.stream_bytes, "dst range");
+    }
     for (int i = 0; i < j.nrows; ++i)
       for (int r = 0; r < j.K; ++r) {
-        const int64_t src = j.trans ? j.src_elem + int64_t(r) * j.src_ld + i : j.src_elem + int64_t(i) * j.K + r;
+        const int64_t src = j.trans == 1 ? j.src_elem + int64_t(r) * j.src_ld + i : j.src_elem + int64_t(i) * j.K + r;
         REQ(src >= 0 && src < Ly.total, "src range");
         if (seen[src]) { REQ(false, "copied twice %ld", (long)src); return; }
         seen[src] = 1;
-        S[j.dst_byte / 2 + int64_t(i) * j.K + r] = W[src];
+        int64_t dst = j.dst_byte / 2 + int64_t(i) * j.K + r;
+        if (j.trans == 2) {   // tile t = r / kb, chunk (r % kb) / 8 swizzled by the tile row
+          const int t = r / j.kb, c = (r % j.kb) / 8, e = r % 8, tr = j.rb0 + i;
+          dst = j.dst_byte / 2 + (int64_t(t) * j.rb + tr) * j.kb + int64_t(c ^ (tr & 7)) * 8 + e;
+        }
+        REQ(S[dst] == 0xdead, "dst written twice");
+        S[dst] = W[src];
       }
     if (!j.trans) REQ(j.src_elem % 8 == 0, "plain job alignment");
   }
@@ -79,77 +86,80 @@ static void check(kie_model_desc m, int n_ctas, const char *name) {
         const StageShape &sh = P.shape[k];
         std::vector<int64_t> tstart;
         int t = 0;
-        // the runs the producer and the consumers tile: one per block, or one
-        // over all the stage's rows when the plan merged them
-        std::vector<Block> runs;
-        if (sc.merged) {
-          REQ(!sh.cols && sc.nblk > 1, "merged stage");
-          int n = 0;
-          for (int bi = 0; bi < sc.nblk; ++bi) {
-            const Block &b = P.blocks[P.cta_blk_begin[c] + sc.blk_begin + bi];
-            REQ(b.lrow0 == n && b.in_off == P.blocks[P.cta_blk_begin[c] + sc.blk_begin].in_off, "merge");
-            n += b.nrows;
+        // the tiles the producer issues and the consumers take: every row
+        // block's column tiles (row stages), R rows of each block (column stages)
+        std::vector<Block> rbs, obs;
+        for (int bi = 0; bi < sc.nblk; ++bi) obs.push_back(P.blocks[P.cta_blk_begin[c] + sc.blk_begin + bi]);
+        if (!sh.cols)
+          for (int bi = 0; bi < sc.nrb; ++bi) rbs.push_back(P.blocks[P.cta_blk_begin[c] + sc.rb_begin + bi]);
+        if (!sh.cols) {
+          const int kb = 128 * sh.cps, nk = sh.K / kb;
+          REQ(sh.cps == 1 || sh.cps == 2 || sh.cps == 4, "cps");
+          REQ(sh.R * sh.cps == kMaxRowBlock && sh.K % kb == 0, "row tiling");
+          std::vector<int> cover(std::max(1, sc.nlocal), 0);
+          for (const Block &b : rbs) {
+            REQ(b.tile0 == t && b.nrows >= 1 && b.nrows <= sh.R, "row block");
+            REQ(int64_t(b.nrows) * kb * 2 <= kSlotBytes, "row tile fits a slot");
+            for (int i = 0; i < b.nrows; ++i) {
+              REQ(b.lrow0 + i < sc.nlocal, "row block rows");
+              cover[b.lrow0 + i]++;
+              bool found = false;   // the row's output block reads the block's input slice
+              for (const Block &o : obs)
+                if (b.lrow0 + i >= o.lrow0 && b.lrow0 + i < o.lrow0 + o.nrows) { found = true; REQ(o.in_off == b.in_off, "one input slice"); }
+              REQ(found, "row in an output block");
+            }
+            for (int q = 0; q < nk; ++q) {
+              tstart.push_back(cur);
+              cur += int64_t(b.nrows) * kb;
+              ++t;
+            }
           }
-          REQ(n == sc.nlocal, "merged rows");
-          Block run = P.blocks[P.cta_blk_begin[c] + sc.blk_begin];
-          run.nrows = n;
-          run.tile0 = 0;
-          runs.push_back(run);
+          for (int i = 0; i < sc.nlocal; ++i) REQ(cover[i] == 1, "row blocks cover local rows once");
         } else {
-          for (int bi = 0; bi < sc.nblk; ++bi) runs.push_back(P.blocks[P.cta_blk_begin[c] + sc.blk_begin + bi]);
-        }
-        for (const Block &b : runs) {
-          REQ(b.tile0 == t, "tile0");
-          for (int r0 = 0; r0 < b.nrows; r0 += sh.R) {
-            const int rows = std::min(sh.R, b.nrows - r0);
-            REQ(int64_t(rows) * sh.K * 2 <= kSlotBytes, "slot");
-            tstart.push_back(cur);
-            cur += int64_t(rows) * sh.K;
-            ++t;
+          for (const Block &b : obs) {
+            REQ(b.tile0 == t, "tile0");
+            for (int r0 = 0; r0 < b.nrows; r0 += sh.R) {
+              const int rows = std::min(sh.R, b.nrows - r0);
+              REQ(int64_t(rows) * sh.K * 2 <= kSlotBytes, "slot");
+              tstart.push_back(cur);
+              cur += int64_t(rows) * sh.K;
+              ++t;
+            }
           }
         }
         REQ(t == sc.ntiles, "ntiles");
         if (l != layer) continue;
         if (!sh.cols) {
-          // row stage: lane mapping of Consumer::gemv_rows
-          REQ(sh.K % 128 == 0 && sh.K <= 4096 && sh.R == 16384 / sh.K, "row shape");
-          REQ(sh.nseg == kConsumerWarps || sh.nseg == 1, "row sums kind");
-          int LSH = 0;
-          while ((128 << LSH) < sh.K) ++LSH;
-          const int LPR = 1 << LSH, RPL = 32 >> LSH;
-          // partial sum of every (local row, warp); every (row, column chunk) read once
+          // row stage: lane / warp mapping of Consumer::gemv_rows_c
+          const int C = sh.cps, kb = 128 * C, nk = sh.K / kb;
           std::vector<double> rowpart(size_t(std::max(1, sc.nlocal)) * kConsumerWarps, 0.0);
           std::vector<int> chunk_hit(size_t(std::max(1, sc.nlocal)) * (sh.K / 8), 0);
-          for (const Block &b : runs) {
-            const int ntile = (b.nrows + sh.R - 1) / sh.R;
-            for (int t = 0; t < ntile; ++t) {
-              const int rows = std::min(sh.R, b.nrows - t * sh.R);
+          for (const Block &b : rbs) {
+            for (int tt = 0; tt < nk; ++tt) {
+              const int64_t ts = tstart[b.tile0 + tt];
               for (int w = 0; w < kConsumerWarps; ++w)
-                for (int lane = 0; lane < 32; ++lane) {
-                  const int lrow = lane >> LSH;
-                  const int col0 = w * (sh.K >> 4) + ((lane & (LPR - 1)) << 3);
-                  const uint32_t off0 = uint32_t(lrow * sh.K + col0) * 2u;
-                  REQ(off0 < 8192 && off0 % 16 == 0, "lane offset");
-                  REQ(b.in_off + col0 + 8 <= sh.in_len, "input slice");
-                  for (int q = 0; q < 4; ++q) {
-                    const int r = lrow + q * RPL;
-                    if (r >= rows) continue;
-                    REQ(off0 + q * 8192 + 16 <= (uint32_t)kSlotBytes, "smem");
-                    REQ(off0 / 2 + q * 4096 == uint32_t(r * sh.K + col0), "chunk address");
-                    double dsum = 0;
-                    for (int e = 0; e < 8; ++e)
-                      dsum += double(S[tstart[b.tile0 + t] + int64_t(r) * sh.K + col0 + e]) * vin(b.in_off + col0 + e);
-                    const int lr = b.lrow0 + t * sh.R + r;
-                    REQ(lr < sc.nlocal, "local row");
-                    rowpart[size_t(lr) * kConsumerWarps + w] += dsum;
-                    chunk_hit[size_t(lr) * (sh.K / 8) + col0 / 8]++;
-                    // where the kernel keeps the row's sum
-                    if (sh.nseg == kConsumerWarps) REQ((lr + 1) * kConsumerWarps <= P.part_atomic_off, "partials region");
-                    else REQ(P.part_atomic_off + lr < P.part_floats, "atomic region");
+                for (int lane = 0; lane < 32; ++lane)
+                  for (int j = 0; j < 4 / C; ++j) {
+                    const int r = lane + 32 * j;
+                    if (r >= b.nrows) continue;
+                    for (int cc = 0; cc < C; ++cc) {
+                      const int pch = w * C + cc;                   // logical chunk of the tile row
+                      const int off = r * kb + ((pch ^ (r & 7)) << 3);   // element offset in the tile
+                      REQ(off % 8 == 0 && off + 8 <= b.nrows * kb, "tile offset");
+                      REQ(off * 2 + 16 <= kSlotBytes, "smem");
+                      const int col = tt * kb + pch * 8;           // canonical column
+                      REQ(b.in_off + col + 8 <= sh.in_len, "input slice");
+                      double dsum = 0;
+                      for (int e = 0; e < 8; ++e) dsum += double(S[ts + off + e]) * vin(b.in_off + col + e);
+                      const int lr = b.lrow0 + r;
+                      rowpart[size_t(lr) * kConsumerWarps + w] += dsum;
+                      chunk_hit[size_t(lr) * (sh.K / 8) + col / 8]++;
+                    }
                   }
-                }
             }
+            REQ(kConsumerWarps * kMaxRowBlock * 2 <= P.rsum_off, "partials region");
           }
+          if (k != ST_LM) REQ(P.rsum_off + sc.nlocal <= P.part_floats, "row sums region");
           for (size_t q = 0; q < size_t(sc.nlocal) * (sh.K / 8); ++q) REQ(chunk_hit[q] == 1, "stage %d chunk hit %d", k, chunk_hit[q]);
           auto rowsum = [&](int i) { double v = 0; for (int w = 0; w < kConsumerWarps; ++w) v += rowpart[size_t(i) * kConsumerWarps + w]; return v; };
           if (k == ST_QKV) {
@@ -321,8 +331,13 @@ int main() {
   for (int K = 128; K <= 4096; K += 128) {
     StageShape sh;
     const bool pow2 = ((K >> 7) & ((K >> 7) - 1)) == 0;
-    REQ((make_shape(K, K, K, sh) == nullptr) == pow2, "make_shape K=%d", K);
-    if (pow2) REQ(sh.R * K == 16384, "tile rows K=%d", K);
+    REQ((make_shape(K, K, K, K, sh) == nullptr) == pow2, "make_shape K=%d", K);
+    if (pow2)
+      for (int run = 1; run <= 300; run += 7) {   // every chunk width keeps a tile within a slot
+        set_row_tiling(sh, run);
+        REQ(128 * sh.cps <= K && K % (128 * sh.cps) == 0 && sh.R * sh.cps == kMaxRowBlock, "tiling K=%d", K);
+        REQ(sh.R * 256 * sh.cps <= kSlotBytes, "tile bytes K=%d", K);
+      }
   }
   {
     // a 3-lane model with 128-wide lanes: its d_model rows (mix, LM head)

@@ -132,25 +132,59 @@ def test_calls_split_into_several_launches(cap):
     dec.kie_destroy()
 
 
-def test_tiny_is_repeatable():
-    """Two launches agree to float rounding.  The O and down projections are
-    summed over SMs with fp32 atomics, so the summation order (and the last
-    bits) differ from run to run; the bound, 5e-5 relative, is a twentieth of
-    the logits tolerance against the oracle."""
+@pytest.mark.parametrize("mode", ["fp32_atomic", "exact"])
+def test_tiny_is_repeatable(mode):
+    """Two launches on fresh contexts.  With fp32 atomic sums the order in
+    which SMs add the O and down projections (and so the last bits) differs
+    from run to run: the bound, 5e-5 relative, is a twentieth of the logits
+    tolerance against the oracle.  With exact sums the two runs are
+    bit-identical: logits, tokens of a free run, and the cache."""
+    import decode_persistent_monokernel_b200 as kie
     w = synth.WORKLOADS[0]
     m = w.model
     bits = synth.generate_weights(m, w.weight_seed)
     prompt = synth.prompt(w)
     forced = synth.forced_tokens(w, 24)
-    runs = []
+    runs, frees, caches = [], [], []
     for _ in range(2):
         dec = make_decoder(m, bits, 64)
+        if mode == "exact":
+            dec.kie_set_sum_mode(kie.KIE_SUM_EXACT)
         dec.kie_prefill(prompt)
         runs.append(_gpu_logits(dec, 24, m.vocab, forced)[1])
+        dec.kie_prefill(prompt)
+        frees.append(dec.kie_decode(24))
+        caches.append(dec.kie_copy_kv(m.n_layers - 1, 0, 0, 64))
         dec.kie_destroy()
     a, b = runs[0].astype(np.float64), runs[1].astype(np.float64)
-    rel = np.linalg.norm(a - b, axis=1) / np.linalg.norm(a, axis=1)
-    assert rel.max() < 5e-5, rel.max()
+    if mode == "exact":
+        assert np.array_equal(runs[0].view(np.uint32), runs[1].view(np.uint32))
+        assert np.array_equal(frees[0], frees[1])
+        assert all(np.array_equal(x, y) for x, y in zip(caches[0], caches[1]))
+    else:
+        rel = np.linalg.norm(a - b, axis=1) / np.linalg.norm(a, axis=1)
+        assert rel.max() < 5e-5, rel.max()
+
+
+@pytest.mark.parametrize("shape", ["tiny", "gqa2_gains", "lanes2_d2", "bf16"])
+def test_exact_sums_match_oracle(shape):
+    """Exact (order-independent) O / down sums give oracle-parity logits and tokens."""
+    import decode_persistent_monokernel_b200 as kie
+    m = synth.WORKLOADS[0].model if shape == "tiny" else _VARIANTS[shape]
+    bits = synth.generate_weights(m, 91)
+    prompt = synth.generate_tokens(13, m.vocab, 7)
+    forced = synth.generate_tokens(30, m.vocab, 8)
+    dec = make_decoder(m, bits, 48)
+    dec.kie_set_sum_mode(kie.KIE_SUM_EXACT)
+    dec.kie_prefill(prompt)
+    toks, z = _gpu_logits(dec, 30, m.vocab, forced)
+    z_ora = Oracle(m, bits, 48).teacher_forced_logits(prompt, forced)
+    check_logits(z, z_ora, f"{shape} fixed point")
+    check_argmax(toks, z_ora, f"{shape} fixed point")
+    with pytest.raises(kie.KieError) as e:
+        dec.kie_set_sum_mode(7)
+    assert e.value.code == kie.KIE_ERR_INVALID
+    dec.kie_destroy()
 
 
 @pytest.mark.parametrize("shape", ["tiny", "lanes2_d2"])

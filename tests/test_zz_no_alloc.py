@@ -32,6 +32,42 @@ def _run(dec, fn, prompt, forced, chunks, vocab):
     return np.concatenate(toks), np.vstack(zs)
 
 
+_TINY = synth.WORKLOADS[0].model
+_SHAPES = {
+    "tiny": _TINY,
+    # a lane model: its delayed cross-lane sums also live in the fixed array
+    "lanes2_d2": _TINY.replace(n_lanes=2, lane_delay=2, n_layers=4, mix_std=0.02, gain_std=0.1),
+}
+
+
+@pytest.mark.parametrize("shape", sorted(_SHAPES))
+@pytest.mark.parametrize("cap", [0, 3])
+@pytest.mark.parametrize("teacher_forced", [True, False])
+def test_static_scratch_is_bit_exact_with_exact_sums(shape, cap, teacher_forced):
+    """With fixed-point O / down sums every launch is deterministic, so the
+    static-scratch call must give exactly the logits and tokens of
+    kie_decode_ex, call after call; also when each call is split into launches
+    of at most 3 steps (the keys and tokens of every launch come from the
+    fixed array too)."""
+    import torch
+    import decode_persistent_monokernel_b200 as kie
+    assert torch.cuda.is_available()
+    m = _SHAPES[shape]
+    bits = synth.generate_weights(m, 41)
+    prompt = synth.generate_tokens(11, m.vocab, 3)
+    forced = synth.generate_tokens(24, m.vocab, 4) if teacher_forced else None
+    dec = make_decoder(m, bits, 64)
+    dec.kie_set_sum_mode(kie.KIE_SUM_EXACT)
+    dec.kie_set_max_steps_per_launch(cap)
+    chunks = (10, 14)                       # two calls in a row
+    t_ref, z_ref = _run(dec, dec.kie_decode_ex, prompt, forced, chunks, m.vocab)
+    t_new, z_new = _run(dec, dec.kie_decode_ex_static, prompt, forced, chunks, m.vocab)
+    assert np.array_equal(t_new, t_ref)
+    assert np.array_equal(z_new.view(np.uint32), z_ref.view(np.uint32))
+    assert dec.kie_get_stats().pos == len(prompt) + sum(chunks)
+    dec.kie_destroy()
+
+
 @pytest.mark.parametrize("teacher_forced", [True, False])
 def test_static_scratch_decode_matches_decode_ex(teacher_forced):
     import torch
@@ -45,9 +81,9 @@ def test_static_scratch_decode_matches_decode_ex(teacher_forced):
     chunks = (10, 14)                       # two calls in a row
     t_ref, z_ref = _run(dec, dec.kie_decode_ex, prompt, forced, chunks, m.vocab)
     t_new, z_new = _run(dec, dec.kie_decode_ex_static, prompt, forced, chunks, m.vocab)
-    # the split projections are summed with atomics, so two launches may differ
-    # in the last bits: compare logits within the tests' tolerance and tokens by
-    # the near-tie rule; a free run may part ways only at a near tie
+    # the default fp32 atomic sums may differ between two launches in the last
+    # bits: compare logits within the tests' tolerance and tokens by the
+    # near-tie rule; a free run may part ways only at a near tie
     n = len(t_ref)
     if not teacher_forced:
         for k in range(n):
