@@ -639,12 +639,13 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
   auto take = [&](size_t n) { size_t r = o; o += (n + 63) / 64 * 64; return r; };
   ctx->off_xres = take(size_t(2) * d);
   ctx->off_acc = take(size_t(8) * d);   // acc_o[2][d] then acc_d[2][d], each with room for lo sums
-  ctx->off_qkv = take(size_t(m.n_heads + 2 * m.n_kv_heads) * dh);
+  // tagged words (8 bytes: two floats' room each)
+  ctx->off_qkv = take(size_t(2) * (m.n_heads + 2 * m.n_kv_heads) * dh);
   ctx->off_dsum = take(size_t(std::max(1, m.lane_delay)) * d);
-  ctx->off_part = take(size_t(m.n_heads) * P.max_split * (dh + 2));
+  ctx->off_part = take(size_t(2) * m.n_heads * P.max_split * (dh + 2));
   ctx->act_floats = o;
   if ((rc = alloc(ctx, (void **)&ctx->act, o * 4, "activations"))) return fail(rc);
-  const size_t sync_words = size_t(SY_QG0 + 2 * m.n_kv_heads) * kSyncStride;
+  const size_t sync_words = size_t(SY_COUNT) * kSyncStride;
   if ((rc = alloc(ctx, (void **)&ctx->sync, sync_words * 4, "sync"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->keys, size_t(m.max_seq) * 8, "keys"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->tokens_in, size_t(m.max_seq) * 4, "tokens"))) return fail(rc);
@@ -781,6 +782,10 @@ static int launch_steps(kie_ctx *ctx, const KernelArgs &a, size_t sync_bytes, in
     CK(cudaMemsetAsync(a.sync, 0, sync_bytes, st));
     CK(cudaMemsetAsync(a.acc_o, 0, size_t(8) * ctx->m.d_model * 4, st));   // both accumulators, both parities
     CK(cudaMemsetAsync(b.keys, 0, size_t(c) * 8, st));
+    // tagged q/k/v and attention partials: tags restart with every launch
+    const kie_model_desc &m = ctx->m;
+    CK(cudaMemsetAsync(a.qkv, 0, size_t(m.n_heads + 2 * m.n_kv_heads) * m.head_dim * 8, st));
+    CK(cudaMemsetAsync(a.attn_part, 0, size_t(m.n_heads) * ctx->plan.max_split * (m.head_dim + 2) * 8, st));
     if (s0 == 0) CK(cudaEventRecord(ctx->ev0, st));
     void *args[] = {&b};
     CK(cudaLaunchCooperativeKernel(monokernel_fn(ctx->m.dtype), dim3(ctx->plan.n_ctas),
@@ -849,8 +854,9 @@ static void set_act(const kie_ctx *ctx, KernelArgs &a, float *act) {
   a.xres = act + ctx->off_xres;
   // fp32 sums take [2][d] floats per accumulator, deterministic sums [2][d] hi + [2][d] lo
   a.acc_o = act + ctx->off_acc; a.acc_d = a.acc_o + (ctx->det_sum ? 4 : 2) * size_t(ctx->m.d_model);
-  a.qkv = act + ctx->off_qkv; a.dsum = act + ctx->off_dsum;
-  a.attn_part = act + ctx->off_part;
+  a.qkv = reinterpret_cast<unsigned long long *>(act + ctx->off_qkv);
+  a.dsum = act + ctx->off_dsum;
+  a.attn_part = reinterpret_cast<unsigned long long *>(act + ctx->off_part);
 }
 
 static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int first_token,
@@ -871,7 +877,7 @@ static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int fi
     CK(cudaMemsetAsync(ctx->trace, 0, 8, st));
   }
 
-  const size_t sync_bytes = size_t(SY_QG0 + 2 * m.n_kv_heads) * kSyncStride * 4;
+  const size_t sync_bytes = size_t(SY_COUNT) * kSyncStride * 4;
   if (forced_host)
     CK(cudaMemcpyAsync(ctx->tokens_in, forced_host, size_t(n) * 4, cudaMemcpyHostToDevice, st));
   ctx->host_tokens.resize(n);
@@ -1092,7 +1098,7 @@ extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t
   const kie_model_desc &m = ctx->m;
   // carve the scratch: counters | keys | forced tokens | out tokens | activations
   auto up = [](size_t b) { return (b + 255) / 256 * 256; };
-  const size_t sync_bytes = size_t(SY_QG0 + 2 * m.n_kv_heads) * kSyncStride * 4;
+  const size_t sync_bytes = size_t(SY_COUNT) * kSyncStride * 4;
   const size_t o_keys = up(sync_bytes);
   const size_t o_tin = o_keys + up(size_t(n_steps) * 8);
   const size_t o_tout = o_tin + up(size_t(n_steps) * 4);

@@ -27,8 +27,8 @@ enum SyncSlot : int {
   SY_ABORT = 4,  // nonzero: a CTA gave up; everyone leaves
   SY_STATUS = 5, // first device error code (0 = none)
   SY_GRID = 6,   // grid-barrier mode: signals made by all CTAs together
-  SY_QG0 = 8,    // SY_QG0 + g: CTAs of KV group g whose q/k/v rows are written;
-                 // SY_QG0 + n_kv_heads + g: ... whose attention partials are written
+  SY_COUNT = 8,  // counters in all (the KV group's q/k/v and attention partials are
+                 // exchanged as tagged words, without counters)
 };
 constexpr int kSyncStride = 32;  // uint32 words per counter (128 bytes)
 
@@ -178,9 +178,9 @@ struct KernelArgs {
   float *acc_o;  // [2, d] attention sublayer output of layer G (atomic sums; zero when reused);
                  // in deterministic mode followed by [2, d] sums of the lo parts
   float *acc_d;  // [2, d] MLP sublayer output of layer G (same storage as acc_o)
-  float *qkv;    // [(Hq + 2 Hkv) dh]
+  unsigned long long *qkv;  // [(Hq + 2 Hkv) dh] this step's q/k/v, tagged words (layer + 1)
   float *dsum;   // [delta, d] delayed cross-lane sums
-  float *attn_part;  // [Hq, max_split, dh + 2] per-split attention partials
+  unsigned long long *attn_part;  // [Hq, max_split, dh + 2] per-split attention partials, tagged
   int32_t max_split; // most CTAs sharing one KV head
   uint32_t *sync;
   unsigned long long *keys;  // [n_steps] packed argmax keys (zeroed by host)

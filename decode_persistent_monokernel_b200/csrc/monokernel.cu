@@ -102,6 +102,19 @@ __device__ __forceinline__ uint32_t ld_relaxed(const uint32_t *p) {
 __device__ __forceinline__ void red_release_add(uint32_t *p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// Tagged words: a float and the epoch it belongs to in one 64-bit word
+// (tag << 32 | float bits).  One aligned 64-bit access cannot tear, so a
+// reader that sees the tag it waits for has the value too: no fence and no
+// separate counter is needed.
+__device__ __forceinline__ void st_tagged(unsigned long long *p, float v, uint32_t tag) {
+  const unsigned long long w = (static_cast<unsigned long long>(tag) << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t *p, uint32_t v) {
   uint32_t old;
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
@@ -250,6 +263,33 @@ __device__ bool wait_counter(const KernelArgs &a, const uint32_t *ctr, uint32_t 
       }
     }
   }
+}
+
+// Bounded wait until the tagged word *p carries `tag`; its value goes to
+// out.  False on watchdog expiry or abort.
+__device__ bool wait_tagged(const KernelArgs &a, const unsigned long long *p, uint32_t tag,
+                            uint32_t where, float &out) {
+  unsigned long long w = ld_relaxed_u64(p);
+  if (uint32_t(w >> 32) != tag) {
+    const long long t0 = clock64(), limit = (long long)a.watchdog_ns * 2;
+    long long next_poll = kAbortPollCycles;
+    const uint32_t *abortp = sync_at(a, SY_ABORT);
+    for (;;) {
+      w = ld_relaxed_u64(p);
+      if (uint32_t(w >> 32) == tag) break;
+      const long long el = clock64() - t0;
+      if (el > next_poll) {
+        next_poll = el + kAbortPollCycles;
+        if (ld_relaxed(abortp)) return false;
+        if (el > limit) {
+          raise_error(a, DE_TIMEOUT_COUNTER | (where << 8));
+          return false;
+        }
+      }
+    }
+  }
+  out = __uint_as_float(uint32_t(w));
+  return true;
 }
 
 // Bounded wait on an mbarrier phase.
@@ -433,7 +473,6 @@ struct Consumer {
   uint32_t gl = 0;        // global layer index step * n_layers + l (parity of the buffers)
   uint32_t lm_count = 0;
   uint32_t nsig = 0;      // signals this CTA has made (grid-barrier mode)
-  uint32_t ag_rounds = 0; // split-KV attention rounds (partials exchanged in the group)
   bool tracing = false;   // profiling build: this SM records the current step
 #ifdef KIE_PROFILE
   __device__ void trace_put(int type, int arg) {
@@ -768,40 +807,45 @@ struct Consumer {
     float *qs = s.vbuf;
     float *kcur = qs + G * dh;
     float *vcur = kcur + dh;
-    const float *qkv = a.qkv;
     const float2 *cs = a.rope_cs + size_t(p) * half;
     const size_t cache_row = ((size_t(l) * Hkv + g) * a.max_seq + p) * dh;
+    // q/k/v of this layer are tagged gl + 1 by the SMs that computed them;
+    // every thread waits for the words it reads
+    const uint32_t tag = gl + 1;
+    bool ok = true;
     for (int idx = tid; idx < (G + 2) * dh; idx += kNC) {
       const int hh = idx / dh, d = idx - hh * dh;
       const int dd = d < half ? d : d - half;
       const float2 c = cs[dd];
+      // row of the fused q/k/v output: query head g G + hh, or the group's k or v
+      const size_t row = hh < G ? size_t(g * G + hh) * dh
+                                : (hh == G ? size_t(a.n_heads) * dh : size_t(a.n_heads + Hkv) * dh) +
+                                      size_t(g) * dh;
+      float v0 = 0.f, v1 = 0.f;
+      ok = ok && wait_tagged(a, a.qkv + row + d, tag, 0x20, v0);
+      if (hh <= G) ok = ok && wait_tagged(a, a.qkv + row + (d < half ? d + half : d - half), tag, 0x20, v1);
       if (hh < G) {
-        const float *q = qkv + size_t(g * G + hh) * dh;
-        const float v0 = __ldcg(q + d), v1 = __ldcg(q + (d < half ? d + half : d - half));
         const float r = d < half ? v0 * c.x - v1 * c.y : v0 * c.x + v1 * c.y;
         qs[idx] = r * a.attn_scale;
       } else if (hh == G) {
-        const float *k = qkv + size_t(a.n_heads) * dh + size_t(g) * dh;
-        const float v0 = __ldcg(k + d), v1 = __ldcg(k + (d < half ? d + half : d - half));
         const float r = d < half ? v0 * c.x - v1 * c.y : v0 * c.x + v1 * c.y;
         const uint16_t b = Store<T>::from_f(r);
         kcur[d] = Store<T>::to_f(b);
-        if (writer) a.kcache[cache_row + d] = b;
+        if (writer && ok) a.kcache[cache_row + d] = b;
       } else {
-        const float *vv = qkv + size_t(a.n_heads + Hkv) * dh + size_t(g) * dh;
-        const uint16_t b = Store<T>::from_f(__ldcg(vv + d));
+        const uint16_t b = Store<T>::from_f(v0);
         vcur[d] = Store<T>::to_f(b);
-        if (writer) a.vcache[cache_row + d] = b;
+        if (writer && ok) a.vcache[cache_row + d] = b;
       }
     }
+    if (!ok) s.misc->abort = 1;
     cbar();
   }
 
   __device__ void attention_body() {
-    const int dh = a.head_dim, half = dh >> 1;
+    const int dh = a.head_dim;
     const int Hkv = a.n_kv_heads, G = a.n_heads / a.n_kv_heads;
     const int g = cta % Hkv;
-    const int ngroup = (a.n_ctas - 1 - g) / Hkv + 1;      // CTAs of this KV group
     int j0, j1, split, nsplit;
     kv_range(j0, j1, split, nsplit);
     // the first cached rows (already pulled into L2 by the producer) are
@@ -810,11 +854,13 @@ struct Consumer {
     kv_load(kw, j0 + warp, j1);
     const bool active = split < nsplit;
     const bool writer = (split == nsplit - 1);  // its range holds position p
+    const uint32_t tag = gl + 1;                // this layer's tag of exchanged words
     float *qs = s.vbuf;              // [G][dh] roped, scaled queries
     float *kcur = qs + G * dh;       // [dh] roped, rounded key of position p
     float *vcur = kcur + dh;         // [dh] rounded value of position p
     float *wst = vcur + dh;          // [W][G][dh + 2] per-warp softmax states
     attn_prologue(writer);
+    if (aborted()) return;
     // Online softmax, kU positions per iteration: their score reductions are
     // independent and one rescale covers them.  The next iteration's rows are
     // requested before this one's arithmetic.
@@ -921,32 +967,40 @@ struct Consumer {
       float O = 0.f;
 #pragma unroll 4
       for (int w = 0; w < kConsumerWarps; ++w) O = fmaf(fac[i * 32 + w], wst[(size_t(w) * G + i) * st + d], O);
-      float *dst = a.attn_part + (size_t(g * G + i) * a.max_split + split) * st;
-      dst[d] = O;
-      if (d == 0) { dst[dh] = hs[2 * i]; dst[dh + 1] = hs[2 * i + 1]; }
+      unsigned long long *dst = a.attn_part + (size_t(g * G + i) * a.max_split + split) * st;
+      st_tagged(dst + d, O, tag);
+      if (d == 0) {
+        st_tagged(dst + dh, hs[2 * i], tag);
+        st_tagged(dst + dh + 1, hs[2 * i + 1], tag);
+      }
     }
-    // every split of the group publishes its partial, then each CTA of the
-    // group loads all of them into shared memory (one coalesced pass) and
-    // merges them (log-sum-exp) into the group's attention output
+    // every split of the group publishes its partial (tagged gl + 1), then
+    // each CTA of the group waits for and loads the words it needs into
+    // shared memory and merges them (log-sum-exp) into the group's output
     KT(TE_ATTN, 2);
-    ++ag_rounds;
-    signal(SY_QG0 + Hkv + g);
-    if (!gate(SY_QG0 + Hkv + g, ag_rounds * uint32_t(ngroup), 0x28, 5)) return;
+    if (a.grid_sync) {   // the ablation keeps a grid-wide barrier here
+      signal(SY_GRID);
+      if (!gate(SY_GRID, 0, 0x28, 5)) return;
+    }
     // This SM's O projection reads only the merged outputs [r0, r0 + nr) of
     // the group's G*dh: stage every split's (m, l) and those output columns.
     const int r0 = s.misc->sc[ST_O].row0, nr = s.misc->sc[ST_O].nout;
     float *pml = s.vbuf;                       // [G][nsplit][2]
     float *po = pml + 2 * G * kMaxSplit;       // [nsplit][nr]
+    bool ok = true;
     for (int q = tid; q < 2 * G * nsplit; q += kNC) {
       const int i = q / (2 * nsplit), r = q - i * 2 * nsplit;
-      pml[q] = __ldcg(a.attn_part + (size_t(g * G + i) * a.max_split + (r >> 1)) * st + dh + (r & 1));
+      ok = ok && wait_tagged(a, a.attn_part + (size_t(g * G + i) * a.max_split + (r >> 1)) * st + dh + (r & 1),
+                             tag, 0x28, pml[q]);
     }
     for (int q = tid; q < nsplit * nr; q += kNC) {
       const int sp = q / nr, idx = r0 + (q - sp * nr);
       const int i = idx / dh, d = idx - i * dh;
-      po[q] = __ldcg(a.attn_part + (size_t(g * G + i) * a.max_split + sp) * st + d);
+      ok = ok && wait_tagged(a, a.attn_part + (size_t(g * G + i) * a.max_split + sp) * st + d, tag, 0x28, po[q]);
     }
+    if (!ok) s.misc->abort = 1;
     cbar();
+    if (aborted()) return;
     // log-sum-exp merge of the splits: warp i computes head i's weights
     // exp(m_s - M) / sum_s l_s exp(m_s - M) once (lane = split), then every
     // needed output element is an nsplit-term weighted sum.  The split
@@ -1154,9 +1208,6 @@ struct Consumer {
     const bool lanes = a.n_lanes > 1;
     const int delta = a.lane_delay;
     const uint32_t nc = a.n_ctas;
-    const int Hkv = a.n_kv_heads;
-    const int g = cta % Hkv;                              // this CTA's KV-head group
-    const uint32_t ng = uint32_t((a.n_ctas - 1 - g) / Hkv + 1);
     const int own_lo = int(int64_t(d) * cta / a.n_ctas);  // residual rows this CTA owns
     const int own_hi = int(int64_t(d) * (cta + 1) / a.n_ctas);
     tok = a.forced ? a.forced[0] : a.first_token;
@@ -1184,11 +1235,15 @@ struct Consumer {
                     a.xres + size_t(cur) * d, own_lo, own_hi);
         {
           const StageCta &c = s.misc->sc[ST_QKV];
+          // q/k/v rows go out as words tagged gl + 1, which the group's SMs
+          // poll directly (the test hook withholds them once, so that the
+          // group's waits run out)
+          const bool publish = !(a.skip_signal_cta == cta && step == 0 && l == 0);
           auto to_qkv = [&](int i, float v) {
             for (int bi = 0; bi < c.nblk; ++bi) {
               const Block &o = s.misc->blk[c.blk_begin + bi];
               if (unsigned(i - o.lrow0) < unsigned(o.nrows)) {
-                a.qkv[o.out_off + (i - o.lrow0)] = v;
+                if (publish) st_tagged(a.qkv + o.out_off + (i - o.lrow0), v, gl + 1);
                 break;
               }
             }
@@ -1196,7 +1251,7 @@ struct Consumer {
           gemv_rows(ST_QKV, s.vbuf, to_qkv);
         }
         if (aborted()) goto done;
-        if (!(a.skip_signal_cta == cta && step == 0 && l == 0)) signal(SY_QG0 + g);
+        if (a.grid_sync) signal(SY_GRID);   // the ablation keeps a grid-wide barrier here
         // ---------------- delayed cross-lane sum of the previous layer
         if (lanes && l >= 1) {
           stage_input([=](int j) { return add4(acc4(a.acc_o, prev, j), acc4(a.acc_d, prev, j)); },
@@ -1208,7 +1263,7 @@ struct Consumer {
           if (aborted()) goto done;
         }
         // ---------------- attention of the group, merged in every group CTA
-        if (!gate(SY_QG0 + g, (gl + 1) * ng, 0x20, 4)) goto done;
+        if (a.grid_sync && !gate(SY_GRID, 0, 0x20, 4)) goto done;
         attention();
         if (aborted()) goto done;
         // ---------------- O projection over the group's attention outputs
