@@ -29,6 +29,8 @@ KIE_SYNC_DEPENDENCY = 0
 KIE_SYNC_GRID = 1
 KIE_SUM_FP32_ATOMIC = 0
 KIE_SUM_EXACT = 1
+KIE_PREFILL_STEPS = 0
+KIE_PREFILL_GEMM = 1
 KIE_F16 = 0
 KIE_BF16 = 1
 
@@ -50,7 +52,8 @@ class kie_stats(ctypes.Structure):
                 ("weight_bytes_per_step", ctypes.c_int64),
                 ("kv_bytes_per_position", ctypes.c_int64),
                 ("last_kernel_ms", ctypes.c_float), ("last_launch_steps", ctypes.c_int32),
-                ("pending_token", ctypes.c_int32)]
+                ("pending_token", ctypes.c_int32), ("last_prefill_ms", ctypes.c_float),
+                ("prefill_mode", ctypes.c_int32)]
 
 
 class KieError(RuntimeError):
@@ -85,6 +88,8 @@ def load(path: str = None) -> ctypes.CDLL:
         "kie_create": ([ctypes.POINTER(kie_model_desc), _P, _P, ctypes.POINTER(_P)], _I),
         "kie_weights_bytes": ([ctypes.POINTER(kie_model_desc), ctypes.POINTER(ctypes.c_int64)], _I),
         "kie_prefill": ([_P, _P, _I, ctypes.POINTER(_I)], _I),
+        "kie_prefill_ex": ([_P, _P, _I, ctypes.POINTER(_I), _P], _I),
+        "kie_set_prefill_mode": ([_P, _I], _I),
         "kie_decode": ([_P, _I, _P], _I),
         "kie_decode_ex": ([_P, _I, _P, _P, _P], _I),
         "kie_decode_ex_static": ([_P, _I, _P, _P, _P], _I),
@@ -173,6 +178,25 @@ class Decoder:
         nxt = _I()
         _check(load().kie_prefill(self._h, t.ctypes.data, len(t), ctypes.byref(nxt)))
         return nxt.value
+
+    def kie_prefill_ex(self, tokens, logits_out=None) -> int:
+        """kie_prefill; logits_out (float32 CUDA tensor of vocab elements, or
+        None) receives the logits of the last prompt position."""
+        import numpy as np
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        if logits_out is not None:
+            if not (hasattr(logits_out, "data_ptr") and logits_out.is_cuda
+                    and str(logits_out.dtype) == "torch.float32" and logits_out.is_contiguous()
+                    and logits_out.numel() >= self.desc.vocab):
+                raise ValueError(f"logits_out must be a contiguous float32 CUDA tensor of at "
+                                 f"least vocab = {self.desc.vocab} elements")
+        nxt = _I()
+        _check(load().kie_prefill_ex(self._h, t.ctypes.data, len(t), ctypes.byref(nxt),
+                                     _ptr(logits_out)))
+        return nxt.value
+
+    def kie_set_prefill_mode(self, mode: int) -> None:
+        _check(load().kie_set_prefill_mode(self._h, mode))
 
     def kie_decode(self, n_steps: int):
         import numpy as np

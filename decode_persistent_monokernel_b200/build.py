@@ -9,8 +9,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["kie_api.cu", "monokernel.cu"]
-HEADERS = ["kie_internal.h", os.path.join("..", "..", "include", "kie.h")]
+SOURCES = ["kie_api.cu", "monokernel.cu", "prefill_gemm.cu", "prefill.cu"]
+HEADERS = ["kie_internal.h", "prefill_internal.h", os.path.join("..", "..", "include", "kie.h")]
 LIB = os.path.join(HERE, "libkie.so")
 PROF_LIB = os.path.join(HERE, "libkie_prof.so")  # activity counters compiled in
 UBENCH_LIB = os.path.join(HERE, "libkie_ubench.so")  # micro-benchmarks (kie_ubench.h)

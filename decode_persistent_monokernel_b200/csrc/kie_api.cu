@@ -6,6 +6,8 @@
 // producer warp reads with bulk copies), and allocates the KV cache and
 // activation buffers.  kie_prefill / kie_decode launch the persistent kernel
 // once per call, cooperatively, with one CTA per SM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -20,6 +22,7 @@
 
 #include "../../include/kie.h"
 #include "kie_internal.h"
+#include "prefill_internal.h"
 
 namespace kie {
 size_t monokernel_smem_bytes(int ring_slots, int vbuf_floats, int part_floats);
@@ -484,6 +487,19 @@ struct kie_ctx {
   size_t off_xres, off_acc, off_qkv, off_dsum, off_part, act_floats;
   size_t kv_elems = 0;
   std::vector<int32_t> host_tokens;
+  // prompt pass on the tensor cores (dense models): the canonical weights as
+  // GEMM B operands, their tensor maps (per layer q/k/v, O, gate/up, down,
+  // then the LM head), and grow-only scratch for the prompt rows
+  int prefill_gemm = 0;           // 1: kie_prefill runs the GEMM prompt pass
+  int prefill_gemm_ok = 0;        // the prompt pass is available for this model
+  uint16_t *wcanon = nullptr;
+  std::vector<CUtensorMap> bmaps;
+  int pf_cap = 0, pf_rows_pad = 0;
+  float *pf_x = nullptr, *pf_qkv = nullptr, *pf_o = nullptr, *pf_gu = nullptr, *pf_logits = nullptr;
+  uint16_t *pf_a = nullptr;       // A parts [P][pf_rows_pad][kmax]
+  int32_t *pf_tok = nullptr;      // the prompt, then the greedy token
+  uint32_t *pf_status = nullptr;
+  float last_prefill_ms = 0.f;
 };
 
 static const char *validate(const kie_model_desc *m) {
@@ -530,7 +546,8 @@ static void free_ctx(kie_ctx *c) {
   if (!c) return;
   void *ptrs[] = {c->wstream, c->embed, c->gains, c->rope, c->kcache, c->vcache, c->act,
                   c->sync, c->keys, c->tokens_in, c->tokens_out, c->d_stage_cta, c->d_blocks,
-                  c->d_blk_begin, c->d_stream_off, c->prof, c->trace};
+                  c->d_blk_begin, c->d_stream_off, c->prof, c->trace, c->wcanon, c->pf_x,
+                  c->pf_qkv, c->pf_o, c->pf_gu, c->pf_logits, c->pf_a, c->pf_tok, c->pf_status};
   for (void *p : ptrs)
     if (p) cudaFree(p);
   if (c->ev0) cudaEventDestroy(c->ev0);
@@ -547,6 +564,39 @@ static int alloc(kie_ctx *ctx, void **p, size_t bytes, const char *what) {
   }
   if (e != cudaSuccess) return cuda_fail(ctx, what, e);
   return KIE_OK;
+}
+
+// ---------------------------------------------------------------- prompt pass (tensor cores)
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link-time
+// dependency on the driver library).
+static PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// Tensor map of a row-major [rows, K] matrix of 16-bit words with row pitch
+// ld elements, read as 64-column x 128-row boxes with 128-byte swizzle (the
+// GEMM's operand tiles); columns >= K and rows >= rows read as zero.
+static bool make_tmap(CUtensorMap *map, const void *base, int dtype, int64_t K, int64_t rows, int64_t ld) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tmap_encode_fn();
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 15) || ((ld * 2) & 15)) return false;
+  cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(ld) * 2};
+  cuuint32_t box[2] = {cuuint32_t(gemm_tile_k()), cuuint32_t(gemm_tile_m())};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, dtype == KIE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 extern "C" int kie_weights_bytes(const kie_model_desc *desc, int64_t *out) {
@@ -718,6 +768,35 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
        ck(cudaStreamSynchronize(st), "create sync");
   cudaFree(d_jobs);
   if (!ok) return fail(KIE_ERR_CUDA);
+  // the tensor-core prompt pass (dense models): a canonical copy of the
+  // weights for its GEMM operands; without room for it, prompts run through
+  // the persistent kernel one position per step
+  if (m.n_lanes == 1 && cudaMalloc((void **)&ctx->wcanon, size_t(Ly.total) * 2) == cudaSuccess) {
+    bool mk = ck(cudaMemcpyAsync(ctx->wcanon, w, size_t(Ly.total) * 2, cudaMemcpyDeviceToDevice, st),
+                 "weights copy") && ck(cudaStreamSynchronize(st), "create sync");
+    if (!mk) return fail(KIE_ERR_CUDA);
+    const int64_t nq = int64_t(m.n_heads + 2 * m.n_kv_heads) * dh, hd = int64_t(m.n_heads) * dh;
+    ctx->bmaps.resize(size_t(4) * L + 1);
+    for (int l = 0; l < L && mk; ++l) {
+      const uint16_t *lw = ctx->wcanon + Ly.layer0 + int64_t(l) * Ly.layer_stride;
+      mk = make_tmap(&ctx->bmaps[4 * l + 0], lw + Ly.wq, m.dtype, d, nq, d) &&
+           make_tmap(&ctx->bmaps[4 * l + 1], lw + Ly.wo, m.dtype, hd, d, hd) &&
+           make_tmap(&ctx->bmaps[4 * l + 2], lw + Ly.wg, m.dtype, d, 2 * int64_t(m.ffn_dim), d) &&
+           make_tmap(&ctx->bmaps[4 * l + 3], lw + Ly.wd, m.dtype, m.ffn_dim, d, m.ffn_dim);
+    }
+    mk = mk && make_tmap(&ctx->bmaps[4 * L], ctx->wcanon + Ly.lm_head, m.dtype, d, m.vocab, d);
+    // default: the tensor-core pass for fp16 models; bf16 models keep the
+    // decode path's own per-position prompt, whose cache matches the oracle's
+    // more closely (bf16 rounding turns fp32-level differences of the pass's
+    // tensor-core accumulation into one-ulp flips of cached K/V)
+    ctx->prefill_gemm_ok = mk ? 1 : 0;
+    ctx->prefill_gemm = mk && m.dtype == KIE_F16 ? 1 : 0;
+    if (!mk) {
+      cudaFree(ctx->wcanon);
+      ctx->wcanon = nullptr;
+    }
+  }
+  cudaGetLastError();
   *out = ctx;
   return KIE_OK;
 }
@@ -775,7 +854,13 @@ static int launch_steps(kie_ctx *ctx, const KernelArgs &a, size_t sync_bytes, in
     b.forced = a.forced ? a.forced + s0 : nullptr;
     b.out_tokens = a.out_tokens + s0;
     b.keys = a.keys + s0;
-    b.logits_out = a.logits_out ? a.logits_out + size_t(s0) * ctx->m.vocab : nullptr;
+    if (a.logits_every_step) {   // every step's logits, each launch at its own offset
+      b.logits_out = a.logits_out ? a.logits_out + size_t(s0) * ctx->m.vocab : nullptr;
+      b.logits_step0 = 0;
+    } else {                     // a prompt: the logits of its last position only
+      b.logits_out = s0 + c == n ? a.logits_out : nullptr;
+      b.logits_step0 = c - 1;
+    }
     b.skip_signal_cta = s0 == 0 ? a.skip_signal_cta : -1;
     if (a.trace && a.trace_step >= s0 && a.trace_step < s0 + c) b.trace_step = a.trace_step - s0;
     else b.trace = nullptr;
@@ -861,7 +946,6 @@ static void set_act(const kie_ctx *ctx, KernelArgs &a, float *act) {
 
 static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int first_token,
                bool logits_every_step, float *logits_out, int32_t *out_host) {
-  const kie_model_desc &m = ctx->m;
   cudaStream_t st = ctx->stream;
   KernelArgs a = fill_args(ctx, pos0, n, first_token, logits_every_step, logits_out);
   set_act(ctx, a, ctx->act);
@@ -886,7 +970,128 @@ static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int fi
   return KIE_OK;
 }
 
-extern "C" int kie_prefill(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_token) {
+// Grows the prompt pass's scratch to hold n prompt rows.
+static int prefill_scratch(kie_ctx *ctx, int n) {
+  if (n <= ctx->pf_cap) return KIE_OK;
+  const kie_model_desc &m = ctx->m;
+  const int d = m.d_model, dh = m.head_dim, F = m.ffn_dim;
+  const int P = m.dtype == KIE_F16 ? 2 : 3;
+  const size_t nq = size_t(m.n_heads + 2 * m.n_kv_heads) * dh, hd = size_t(m.n_heads) * dh;
+  const size_t kmax = std::max<size_t>({size_t(d), hd, size_t(F)});
+  const int rows_pad = (n + gemm_tile_m() - 1) / gemm_tile_m() * gemm_tile_m();
+  void *bufs[] = {ctx->pf_x, ctx->pf_qkv, ctx->pf_o, ctx->pf_gu, ctx->pf_logits, ctx->pf_a, ctx->pf_tok,
+                  ctx->pf_status};
+  for (void *b : bufs)
+    if (b) cudaFree(b);
+  ctx->pf_x = ctx->pf_qkv = ctx->pf_o = ctx->pf_gu = ctx->pf_logits = nullptr;
+  ctx->pf_a = nullptr;
+  ctx->pf_tok = nullptr;
+  ctx->pf_status = nullptr;
+  ctx->pf_cap = 0;
+  int rc;
+  if ((rc = alloc(ctx, (void **)&ctx->pf_x, size_t(n) * d * 4, "prompt scratch")) ||
+      (rc = alloc(ctx, (void **)&ctx->pf_qkv, size_t(n) * nq * 4, "prompt scratch")) ||
+      (rc = alloc(ctx, (void **)&ctx->pf_o, size_t(n) * hd * 4, "prompt scratch")) ||
+      (rc = alloc(ctx, (void **)&ctx->pf_gu, size_t(n) * 2 * F * 4, "prompt scratch")) ||
+      (rc = alloc(ctx, (void **)&ctx->pf_logits, size_t(m.vocab) * 4, "prompt scratch")) ||
+      (rc = alloc(ctx, (void **)&ctx->pf_a, size_t(P) * rows_pad * kmax * 2, "prompt scratch")) ||
+      (rc = alloc(ctx, (void **)&ctx->pf_tok, size_t(n + 1) * 4, "prompt scratch")) ||
+      (rc = alloc(ctx, (void **)&ctx->pf_status, 4, "prompt scratch")))
+    return rc;
+  ctx->pf_cap = n;
+  ctx->pf_rows_pad = rows_pad;
+  return KIE_OK;
+}
+
+// The prompt pass on the tensor cores: every layer for all n prompt rows at
+// once (RMSNorm -> q/k/v GEMM -> RoPE + K/V cache -> causal attention -> O
+// GEMM into the residual -> RMSNorm -> gate/up GEMM -> SwiGLU -> down GEMM
+// into the residual), then the final norm and LM head of the last row and
+// its greedy token.  logits_out (device [V] or null) receives that row's
+// logits.
+static int prefill_gemm_run(kie_ctx *ctx, const int32_t *tokens, int n, float *logits_out, int32_t *next) {
+  const kie_model_desc &m = ctx->m;
+  const int d = m.d_model, dh = m.head_dim, Hq = m.n_heads, Hkv = m.n_kv_heads, F = m.ffn_dim, L = m.n_layers;
+  const int V = m.vocab, P = m.dtype == KIE_F16 ? 2 : 3;
+  const int nq = (Hq + 2 * Hkv) * dh, hd = Hq * dh;
+  cudaStream_t st = ctx->stream;
+  if (int rc = prefill_scratch(ctx, n)) return rc;
+  const int64_t kmax = std::max({int64_t(d), int64_t(hd), int64_t(F)});
+  const int64_t pstride = int64_t(ctx->pf_rows_pad) * kmax;   // elements between A parts
+  CUtensorMap map_ad, map_af;   // the A parts read with K = d and with K = F
+  if (!make_tmap(&map_ad, ctx->pf_a, m.dtype, d, int64_t(P) * ctx->pf_rows_pad, kmax) ||
+      !make_tmap(&map_af, ctx->pf_a, m.dtype, F, int64_t(P) * ctx->pf_rows_pad, kmax)) {
+    g_last_error = "tensor map of the prompt pass could not be encoded";
+    ctx->poisoned = KIE_ERR_CUDA;
+    return KIE_ERR_CUDA;
+  }
+  GemmArgs g{};
+  g.parts = P;
+  g.stages = gemm_stages(P);
+  g.a_part_rows = ctx->pf_rows_pad;
+  g.dtype = m.dtype;
+  g.status = ctx->pf_status;
+  g.watchdog_ns = ctx->watchdog_ns;
+  auto gemm = [&](const CUtensorMap &ma, const CUtensorMap &mb, int M, int N, int K, float *C, int64_t ldc,
+                  int acc) {
+    GemmArgs a = g;
+    a.M = M; a.N = N; a.K = K; a.C = C; a.ldc = ldc; a.accumulate = acc;
+    return launch_gemm(ma, mb, a, st);
+  };
+  const float *gain_attn = ctx->gains, *gain_ffn = ctx->gains + size_t(L) * d;
+  const float *gain_final = ctx->gains + size_t(2 * L) * d;
+  const float scale = float(1.0 / sqrt(double(dh)));
+  CK(cudaEventRecord(ctx->ev0, st));
+  CK(cudaMemcpyAsync(ctx->pf_tok, tokens, size_t(n) * 4, cudaMemcpyHostToDevice, st));
+  CK(cudaMemsetAsync(ctx->pf_status, 0, 4, st));
+  CK(launch_embed_rows(ctx->embed, ctx->pf_tok, n, d, m.dtype, ctx->pf_x, st));
+  for (int l = 0; l < L; ++l) {
+    CK(launch_norm_split(ctx->pf_x, gain_attn + size_t(l) * d, n, d, m.rms_eps, P, m.dtype, ctx->pf_a, pstride,
+                         kmax, st));
+    CK(gemm(map_ad, ctx->bmaps[4 * l + 0], n, nq, d, ctx->pf_qkv, nq, 0));
+    CK(launch_rope_kv(ctx->pf_qkv, n, 0, Hq, Hkv, dh, ctx->rope, ctx->kcache, ctx->vcache, l, m.max_seq, m.dtype,
+                      scale, st));
+    CK(launch_prefill_attention(ctx->pf_qkv, n, 0, Hq, Hkv, dh, ctx->kcache, ctx->vcache, l, m.max_seq, m.dtype,
+                                ctx->pf_o, st));
+    CK(launch_split(ctx->pf_o, n, hd, hd, P, m.dtype, ctx->pf_a, pstride, kmax, st));
+    CK(gemm(map_ad, ctx->bmaps[4 * l + 1], n, d, hd, ctx->pf_x, d, 1));
+    CK(launch_norm_split(ctx->pf_x, gain_ffn + size_t(l) * d, n, d, m.rms_eps, P, m.dtype, ctx->pf_a, pstride,
+                         kmax, st));
+    CK(gemm(map_ad, ctx->bmaps[4 * l + 2], n, 2 * F, d, ctx->pf_gu, 2 * int64_t(F), 0));
+    CK(launch_swiglu_split(ctx->pf_gu, n, F, P, m.dtype, ctx->pf_a, pstride, kmax, st));
+    CK(gemm(map_af, ctx->bmaps[4 * l + 3], n, d, F, ctx->pf_x, d, 1));
+  }
+  CK(launch_norm_split(ctx->pf_x + size_t(n - 1) * d, gain_final, 1, d, m.rms_eps, P, m.dtype, ctx->pf_a, pstride,
+                       kmax, st));
+  CK(gemm(map_ad, ctx->bmaps[4 * L], 1, V, d, ctx->pf_logits, V, 0));
+  CK(launch_argmax_row(ctx->pf_logits, V, ctx->pf_tok + n, st));
+  if (logits_out)
+    CK(cudaMemcpyAsync(logits_out, ctx->pf_logits, size_t(V) * 4, cudaMemcpyDeviceToDevice, st));
+  CK(cudaEventRecord(ctx->ev1, st));
+  int32_t tok = -1;
+  uint32_t status = 0;
+  CK(cudaMemcpyAsync(&tok, ctx->pf_tok + n, 4, cudaMemcpyDeviceToHost, st));
+  CK(cudaMemcpyAsync(&status, ctx->pf_status, 4, cudaMemcpyDeviceToHost, st));
+  CK(cudaStreamSynchronize(st));
+  CK(cudaEventElapsedTime(&ctx->last_prefill_ms, ctx->ev0, ctx->ev1));
+  if (status != 0) {
+    char buf[160];
+    snprintf(buf, sizeof buf, "prompt pass: a bounded wait ran out (code 0x%x)", status);
+    g_last_error = buf;
+    ctx->poisoned = KIE_ERR_DEVICE_TIMEOUT;
+    return KIE_ERR_DEVICE_TIMEOUT;
+  }
+  if (tok < 0 || tok >= V) {
+    g_last_error = "non-finite logits at the last prompt position";
+    ctx->poisoned = KIE_ERR_NONFINITE;
+    return KIE_ERR_NONFINITE;
+  }
+  *next = tok;
+  return KIE_OK;
+}
+
+extern "C" int kie_prefill_ex(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_token,
+                              float *logits_out) {
   if (!ctx || !tokens || !next_token || n < 1) return KIE_ERR_INVALID;
   if (ctx->poisoned) return KIE_ERR_POISONED;
   if (n > ctx->m.max_seq) return KIE_ERR_CAPACITY;
@@ -896,12 +1101,33 @@ extern "C" int kie_prefill(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32
   CK(cudaMemsetAsync(ctx->vcache, 0xff, ctx->kv_elems * 2, ctx->stream));
   ctx->pos = 0;
   ctx->pending = -1;
-  std::vector<int32_t> out(n);
-  int rc = run(ctx, 0, n, tokens, 0, false, nullptr, out.data());
-  if (rc) return rc;
+  int32_t next = -1;
+  if (ctx->prefill_gemm) {
+    if (int rc = prefill_gemm_run(ctx, tokens, n, logits_out, &next)) return rc;
+  } else {
+    std::vector<int32_t> out(n);
+    if (int rc = run(ctx, 0, n, tokens, 0, false, logits_out, out.data())) return rc;
+    ctx->last_prefill_ms = ctx->last_ms;
+    next = out[n - 1];
+  }
   ctx->pos = n;
-  ctx->pending = out[n - 1];
-  *next_token = ctx->pending;
+  ctx->pending = next;
+  *next_token = next;
+  return KIE_OK;
+}
+
+extern "C" int kie_prefill(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_token) {
+  return kie_prefill_ex(ctx, tokens, n, next_token, nullptr);
+}
+
+extern "C" int kie_set_prefill_mode(kie_ctx *ctx, int32_t mode) {
+  if (!ctx || (mode != KIE_PREFILL_STEPS && mode != KIE_PREFILL_GEMM)) return KIE_ERR_INVALID;
+  if (mode == KIE_PREFILL_GEMM && !ctx->prefill_gemm_ok) {
+    g_last_error = "the tensor-core prompt pass is not available for this model (lane models, or no "
+                   "device memory for its weight copy)";
+    return KIE_ERR_INVALID;
+  }
+  ctx->prefill_gemm = mode == KIE_PREFILL_GEMM ? 1 : 0;
   return KIE_OK;
 }
 
@@ -966,6 +1192,8 @@ extern "C" int kie_get_stats(const kie_ctx *ctx, kie_stats *out) {
   out->last_kernel_ms = ctx->last_ms;
   out->last_launch_steps = ctx->last_steps;
   out->pending_token = ctx->pending;
+  out->last_prefill_ms = ctx->last_prefill_ms;
+  out->prefill_mode = ctx->prefill_gemm ? KIE_PREFILL_GEMM : KIE_PREFILL_STEPS;
   return KIE_OK;
 }
 
@@ -1095,7 +1323,6 @@ extern "C" int kie_decode_ex_static(kie_ctx *ctx, int32_t n_steps, const int32_t
   if (forced_tokens)
     for (int i = 0; i < n_steps; ++i)
       if (forced_tokens[i] < 0 || forced_tokens[i] >= ctx->m.vocab) return KIE_ERR_INVALID;
-  const kie_model_desc &m = ctx->m;
   // carve the scratch: counters | keys | forced tokens | out tokens | activations
   auto up = [](size_t b) { return (b + 255) / 256 * 256; };
   const size_t sync_bytes = size_t(SY_COUNT) * kSyncStride * 4;

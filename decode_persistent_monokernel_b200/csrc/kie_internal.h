@@ -190,7 +190,8 @@ struct KernelArgs {
   const int32_t *forced;        // device [n_steps] or nullptr
   int32_t logits_every_step;    // 1: LM head every step; 0: only at the last step
   int32_t *out_tokens;          // device [n_steps]
-  float *logits_out;            // device [n_steps, V] or nullptr
+  float *logits_out;            // device [n_steps, V] or nullptr; step s writes row s - logits_step0
+  int32_t logits_step0;
   uint64_t watchdog_ns;
   int32_t skip_signal_cta;      // test hook, -1 = off
   int32_t grid_sync;            // 1: every dependency wait is a grid-wide barrier

@@ -1170,7 +1170,7 @@ struct Consumer {
   // raises DE_NONFINITE.
   __device__ __forceinline__ void lm_row(int i, float v, float &best, int &bidx) {
     const int row = s.misc->sc[ST_LM].row0 + i;
-    if (a.logits_out) a.logits_out[size_t(step) * a.vocab + row] = v;
+    if (a.logits_out) a.logits_out[size_t(step - a.logits_step0) * a.vocab + row] = v;
     if (v != v) raise_error(a, DE_NONFINITE | (uint32_t(step & 0xffff) << 8));
     if (v > best || (v == best && row < bidx)) { best = v; bidx = row; }
   }

@@ -118,6 +118,35 @@ int kie_weights_bytes(const kie_model_desc *desc, int64_t *out);
  *   step, in the same persistent kernel. */
 int kie_prefill(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_token);
 
+/* kie_prefill that also returns the logits of the last prompt position:
+ *   logits_out: DEVICE fp32 array [vocab], or NULL. */
+int kie_prefill_ex(kie_ctx *ctx, const int32_t *tokens, int32_t n, int32_t *next_token,
+                   float *logits_out);
+
+/* How kie_prefill / kie_prefill_ex process a prompt (applies to later calls):
+ *   KIE_PREFILL_GEMM (default for dense fp16 models): the prompt pass on the
+ *     tensor cores.  Per layer, for all prompt rows at once: RMSNorm, the
+ *     q/k/v, O, gate/up and down projections as tcgen05 GEMMs (operands
+ *     staged by tensor-map bulk copies, fp32 accumulation in tensor memory;
+ *     the fp32 activations enter as a sum of two fp16 or three bf16 parts, so
+ *     the products keep fp32-level precision), RoPE and the K/V cache write,
+ *     causal attention on the CUDA cores; then the final norm, LM head and
+ *     greedy token of the last row.  Needs a second, canonical copy of the
+ *     weights in device memory, made by kie_create when there is room.
+ *   KIE_PREFILL_STEPS: the prompt runs through the persistent decode kernel
+ *     one position per step (the only mode for lane models, and the default
+ *     for bf16 models: bf16's 8-bit significand turns the fp32-level
+ *     differences of the tensor-core accumulation into one-ulp differences of
+ *     cached K/V, which the decode path's own arithmetic avoids).
+ * Both leave the same state: the KV cache of positions 0..n-1 and the greedy
+ * next token.  KIE_ERR_INVALID for another mode, or for KIE_PREFILL_GEMM
+ * when the prompt pass is not available for this context (lane model, or no
+ * room for its weight copy; kie_strerror says which).
+ * Passage: "Startup Kog dosahuje 3 000 tokenu/s..." page, section "Software
+ * versus kremik": prefill as part of the same engine's decode cycle. */
+enum { KIE_PREFILL_STEPS = 0, KIE_PREFILL_GEMM = 1 };
+int kie_set_prefill_mode(kie_ctx *ctx, int32_t mode);
+
 /* Greedy decode: step k feeds the pending token at position pos+k, appends
  * its K/V, and the argmax of its logits becomes out_tokens[k] and the next
  * pending token.  The first pending token is kie_prefill's next_token.
@@ -188,6 +217,8 @@ typedef struct {
                                  first one's start to the last one's end (CUDA events) */
   int32_t last_launch_steps;  /* steps run by that call */
   int32_t pending_token;
+  float last_prefill_ms;      /* device time of the most recent prompt (either mode) */
+  int32_t prefill_mode;       /* KIE_PREFILL_GEMM or KIE_PREFILL_STEPS */
 } kie_stats;
 
 int kie_get_stats(const kie_ctx *ctx, kie_stats *out);

@@ -18,7 +18,17 @@ def make_decoder(shape, bits, max_seq):
     return dec
 
 
-def check_logits(z_gpu, z_ora, label=""):
+# bf16 KV cache at full depth: a cached k or v is the bf16 rounding of an fp32
+# value on the GPU and of a float64 value in the oracle; bf16's 8-bit
+# significand turns differences of fp32 size into one-ulp flips of cached
+# values, and 32 layers compound them.  The float64 oracle against itself with
+# its k, v perturbed by 1e-6 relative before rounding differs by 1.9e-3
+# (max-abs 0.012) on the full 8B-class test case, above the 1e-3 that holds
+# everywhere else; that case is checked against this floor plus margin.
+REL_L2_BF16_FULL_DEPTH = 3e-3
+
+
+def check_logits(z_gpu, z_ora, label="", rel_l2=REL_L2):
     """Per-step acceptance: relative L2 and max-abs error of each step's logits."""
     z_gpu = np.asarray(z_gpu, dtype=np.float64)
     z_ora = np.asarray(z_ora, dtype=np.float64)
@@ -26,7 +36,7 @@ def check_logits(z_gpu, z_ora, label=""):
     assert np.isfinite(z_gpu).all(), f"{label}: non-finite logits"
     rel = np.linalg.norm(z_gpu - z_ora, axis=-1) / np.linalg.norm(z_ora, axis=-1)
     mab = np.abs(z_gpu - z_ora).max(axis=-1)
-    assert rel.max() <= REL_L2, f"{label}: rel-L2 {rel.max():.3g} at step {rel.argmax()}"
+    assert rel.max() <= rel_l2, f"{label}: rel-L2 {rel.max():.3g} at step {rel.argmax()}"
     assert mab.max() <= MAX_ABS, f"{label}: max-abs {mab.max():.3g} at step {mab.argmax()}"
     return float(rel.max()), float(mab.max())
 
@@ -59,3 +69,34 @@ def free_run_prefix(gpu_toks, ora_toks, ora_logits, label=""):
         assert gpu_toks[k] == ora_toks[k], f"{label}: step {k}: gpu {gpu_toks[k]} oracle {ora_toks[k]}"
         n += 1
     return n
+
+
+def storage_ulp(v, dtype):
+    """Spacing of the storage type (fp16: 10 fraction bits, bf16: 7) at |v|."""
+    frac = 10 if dtype == "f16" else 7
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    if dtype == "f16":
+        e = np.maximum(e, -14.0)          # subnormal spacing below 2^-14
+    return np.where(a > 0, 2.0 ** (e - frac), 2.0 ** (-14 - frac) if dtype == "f16" else 0.0)
+
+
+def check_kv(dec, orc, m, upto, max_seq, rel=0.0):
+    """Positions [0, upto) of every layer and KV head hold the oracle's rounded
+    K/V, the rest still hold the NaN poison.  A cached value is the storage-type
+    rounding of an fp32 value on the GPU and of a float64 value in the oracle,
+    so the two may round to neighbouring storage values (one ulp apart: up to
+    2^-7 of the value for bf16); each element must agree to that ulp plus
+    4e-3 of the head's largest value, plus `rel` of its own value where the
+    inputs themselves differ by that much (the bf16 cache at full depth)."""
+    from oracle.numerics import storage_to_f64
+    for l in range(m.n_layers):
+        for g in range(m.n_kv_heads):
+            k, v = dec.kie_copy_kv(l, g, 0, max_seq)
+            kf, vf = storage_to_f64(k, m.dtype), storage_to_f64(v, m.dtype)
+            assert np.isfinite(kf[:upto]).all() and np.isfinite(vf[:upto]).all()
+            assert np.isnan(kf[upto:]).all() and np.isnan(vf[upto:]).all()
+            for got, want in ((kf[:upto], orc.K[l, g, :upto]), (vf[:upto], orc.V[l, g, :upto])):
+                scale = np.abs(want).max() + 1e-30
+                tol = 4e-3 * scale + storage_ulp(want, m.dtype) + rel * np.abs(want)
+                assert (np.abs(got - want) <= tol).all(), (l, g, float(np.abs(got - want).max()))
