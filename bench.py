@@ -120,6 +120,27 @@ def dram_traffic(algorithmic_bytes, workload):
         return None, "no counter capture recorded"
 
 
+def prompt_gemm_flops(m, P):
+    """Algorithmic tensor-core work of the prompt pass over P tokens: 2 flops
+    per weight element per prompt row in the q/k/v, O, gate/up and down
+    projections of every layer, and the LM head for the last row (the
+    operand parts the pass splits activations into are not counted)."""
+    d, dh, F = m.d_model, m.head_dim, m.ffn_dim
+    per_layer = ((m.n_heads + 2 * m.n_kv_heads) * dh * d + d * m.n_heads * dh + 3 * F * d)
+    return 2.0 * P * m.n_layers * per_layer + 2.0 * m.vocab * d
+
+
+def peak_tensor():
+    """Measured dense bf16 tensor throughput (TFLOP/s, burst) of this machine's
+    B200s; fp16 has the same nominal rate."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def peak_hbm():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -348,6 +369,11 @@ def main():
     barrier()
     ms = ev0.elapsed_time(ev1)
     kernel_ms = dec.kie_get_stats().last_kernel_ms
+    # the prompt pass, timed on the device by the library (the prompt of the
+    # timed run above)
+    pf_ms = dec.kie_get_stats().last_prefill_ms
+    pf_mode = "tensor-core GEMM pass" if st.prefill_mode == kie.KIE_PREFILL_GEMM else \
+        "persistent kernel, one position per step"
     # end to end through the C ABI with host buffers: the prompt goes in from
     # host memory (timed on its own), then the decode call, whose wall time
     # includes the launch, the device-to-host copy of the K tokens and status,
@@ -406,6 +432,14 @@ def main():
         "kernel": {"ctas": st.n_ctas, "threads": st.threads_per_cta, "ring_slots": st.ring_slots,
                    "smem_bytes": st.smem_bytes},
     }
+    tpeak, tpeak_kind = peak_tensor()
+    gflop = prompt_gemm_flops(m, P) / 1e9
+    line["prefill"] = {"tokens": P, "mode": pf_mode, "device_ms": pf_ms,
+                       "tokens_per_s": P / (pf_ms * 1e-3) if pf_ms > 0 else None,
+                       "gemm_gflop": gflop,
+                       "gemm_tflops": gflop / pf_ms if pf_ms > 0 else None,
+                       "tensor_peak_tflops": tpeak, "peak_kind": tpeak_kind,
+                       "frac_of_tensor_peak": gflop / pf_ms / tpeak if pf_ms > 0 else None}
     if args.profile:
         mhz = line["clocks"]["sm_mhz"] or 1965
         line["profile"] = profile_summary(dec.kie_get_profile(), K, mhz)

@@ -72,6 +72,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=4)
     ap.add_argument("--prompt", type=int, default=0, help="prompt length (0: the workload's)")
     ap.add_argument("--launches", type=int, default=1, help="timed kie_decode launches")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the prompt (twice: a warm-up and the captured one)")
     ap.add_argument("--record-traffic", metavar="NCU_REPORT",
                     help="no GPU run: record DRAM traffic / algorithmic bytes from a report of "
                          "this case (read with ncu -i) for bench.py")
@@ -97,6 +99,14 @@ def main(argv=None):
     dec = kie.Decoder(kie.make_desc(m, P + args.steps * (args.launches + 1) + 8), dev)
     del dev
     torch.cuda.synchronize()
+    if args.prefill_only:
+        for _ in range(2):
+            dec.kie_prefill(prompt)
+        st = dec.kie_get_stats()
+        print(json.dumps({"workload": w.name, "layers": m.n_layers, "prompt": P,
+                          "prefill_mode": st.prefill_mode, "prefill_ms": st.last_prefill_ms}))
+        dec.kie_destroy()
+        return
     dec.kie_prefill(prompt)
     dec.kie_decode(args.steps)                 # warm-up launch
     ms = []
