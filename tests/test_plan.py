@@ -6,7 +6,7 @@ producer's tile walk and the consumers' lane and thread mappings on the
 streamed bytes in double precision: every weight element is copied exactly
 once, every (row, column chunk) is read exactly once, and one layer's
 q/k/v, gate/up, O, down and lane-mix products equal the canonical
-matrix-vector products.  The kernel file is compiled to PTX only (nothing
+matrix-vector products.  The kernel files are compiled to PTX only (nothing
 runs on a GPU).
 """
 import os
@@ -22,7 +22,8 @@ def test_plan_mappings_cover_every_weight_once(tmp_path):
     exe = str(tmp_path / "plan_check")
     cmd = [kbuild.nvcc(), "-gencode", "arch=compute_100a,code=compute_100a", "-O1", "-std=c++17",
            "-I", os.path.join(ROOT, "include"), os.path.join(HERE, "plan_check.cu"),
-           os.path.join(ROOT, "decode_persistent_monokernel_b200", "csrc", "monokernel.cu"),
+           *[os.path.join(ROOT, "decode_persistent_monokernel_b200", "csrc", f)
+             for f in ("monokernel.cu", "prefill_gemm.cu", "prefill.cu")],
            "-o", exe]
     subprocess.run(cmd, check=True, capture_output=True, text=True)
     res = subprocess.run([exe], capture_output=True, text=True, timeout=600)
