@@ -23,3 +23,4 @@ pure-Python no-cache brute force; none is "parity unpinned".
 """
 from .numerics import round_to_storage, storage_to_f64  # noqa: F401
 from .decoder import Oracle, argmax_lowest, rmsnorm, rope, silu, top2_margin  # noqa: F401
+from .sampling import sample_token, sampling_margins  # noqa: F401
