@@ -33,6 +33,7 @@ KIE_PREFILL_STEPS = 0
 KIE_PREFILL_GEMM = 1
 KIE_F16 = 0
 KIE_BF16 = 1
+KIE_MAX_TOP_K = 64
 
 
 class kie_model_desc(ctypes.Structure):
@@ -54,6 +55,11 @@ class kie_stats(ctypes.Structure):
                 ("last_kernel_ms", ctypes.c_float), ("last_launch_steps", ctypes.c_int32),
                 ("pending_token", ctypes.c_int32), ("last_prefill_ms", ctypes.c_float),
                 ("prefill_mode", ctypes.c_int32)]
+
+
+class kie_sampling(ctypes.Structure):
+    _fields_ = [("temperature", ctypes.c_float), ("top_k", ctypes.c_int32),
+                ("top_p", ctypes.c_float)]
 
 
 class KieError(RuntimeError):
@@ -93,6 +99,7 @@ def load(path: str = None) -> ctypes.CDLL:
         "kie_decode": ([_P, _I, _P], _I),
         "kie_decode_ex": ([_P, _I, _P, _P, _P], _I),
         "kie_decode_ex_static": ([_P, _I, _P, _P, _P], _I),
+        "kie_decode_sample": ([_P, _I, ctypes.POINTER(kie_sampling), _P, _P, _P, _P], _I),
         "kie_destroy": ([_P], _I),
         "kie_strerror": ([_I], ctypes.c_char_p),
         "kie_get_stats": ([_P, ctypes.POINTER(kie_stats)], _I),
@@ -227,6 +234,24 @@ class Decoder:
         out = np.empty(n_steps, dtype=np.int32)
         fp, lp, _keep = self._decode_args(n_steps, forced, logits_out)
         _check(load().kie_decode_ex(self._h, n_steps, fp, out.ctypes.data, lp))
+        return out
+
+    def kie_decode_sample(self, n_steps: int, temperature: float, top_k: int = 0,
+                          top_p: float = 1.0, uniforms=None, forced=None, logits_out=None):
+        """kie_decode_ex with each step's token drawn (temperature, top-k,
+        top-p, inverse CDF at uniforms[k]) instead of the argmax."""
+        import numpy as np
+        out = np.empty(n_steps, dtype=np.int32)
+        fp, lp, _keep = self._decode_args(n_steps, forced, logits_out)
+        u = None
+        if uniforms is not None:
+            u = np.ascontiguousarray(uniforms, dtype=np.float32)
+            if u.ndim != 1 or u.size != n_steps:
+                raise ValueError(f"uniforms must hold exactly n_steps = {n_steps} values")
+        prm = kie_sampling(float(temperature), int(top_k), float(top_p))
+        _check(load().kie_decode_sample(self._h, n_steps, ctypes.byref(prm),
+                                        None if u is None else u.ctypes.data, fp,
+                                        out.ctypes.data, lp))
         return out
 
     def kie_decode_ex_static(self, n_steps: int, forced=None, logits_out=None):

@@ -16,6 +16,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -500,6 +501,11 @@ struct kie_ctx {
   int32_t *pf_tok = nullptr;      // the prompt, then the greedy token
   uint32_t *pf_status = nullptr;
   float last_prefill_ms = 0.f;
+  // sampling at the LM head: the uniforms of a call, the step's logits, each
+  // CTA's top-k candidates and its tagged probability sum
+  float *uniforms = nullptr, *zbuf = nullptr;
+  unsigned long long *cand = nullptr, *psum = nullptr;
+  int max_lm_rows = 0;   // LM-head rows of the largest CTA slice
 };
 
 static const char *validate(const kie_model_desc *m) {
@@ -547,7 +553,8 @@ static void free_ctx(kie_ctx *c) {
   void *ptrs[] = {c->wstream, c->embed, c->gains, c->rope, c->kcache, c->vcache, c->act,
                   c->sync, c->keys, c->tokens_in, c->tokens_out, c->d_stage_cta, c->d_blocks,
                   c->d_blk_begin, c->d_stream_off, c->prof, c->trace, c->wcanon, c->pf_x,
-                  c->pf_qkv, c->pf_o, c->pf_gu, c->pf_logits, c->pf_a, c->pf_tok, c->pf_status};
+                  c->pf_qkv, c->pf_o, c->pf_gu, c->pf_logits, c->pf_a, c->pf_tok, c->pf_status,
+                  c->uniforms, c->zbuf, c->cand, c->psum};
   for (void *p : ptrs)
     if (p) cudaFree(p);
   if (c->ev0) cudaEventDestroy(c->ev0);
@@ -700,6 +707,12 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
   if ((rc = alloc(ctx, (void **)&ctx->keys, size_t(m.max_seq) * 8, "keys"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->tokens_in, size_t(m.max_seq) * 4, "tokens"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->tokens_out, size_t(m.max_seq) * 4, "tokens"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->uniforms, size_t(m.max_seq) * 4, "sampling"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->zbuf, size_t(m.vocab) * 4, "sampling"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->cand, size_t(P.n_ctas) * kMaxTopK * 8, "sampling"))) return fail(rc);
+  if ((rc = alloc(ctx, (void **)&ctx->psum, size_t(P.n_ctas) * 8, "sampling"))) return fail(rc);
+  for (int c = 0; c < P.n_ctas; ++c)
+    ctx->max_lm_rows = std::max(ctx->max_lm_rows, P.stage_cta[size_t(ST_LM) * P.n_ctas + c].nout);
   if ((rc = alloc(ctx, (void **)&ctx->d_stage_cta, P.stage_cta.size() * sizeof(StageCta), "plan"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->d_blocks, std::max<size_t>(1, P.blocks.size()) * sizeof(Block), "plan"))) return fail(rc);
   if ((rc = alloc(ctx, (void **)&ctx->d_blk_begin, P.cta_blk_begin.size() * 4, "plan"))) return fail(rc);
@@ -854,6 +867,7 @@ static int launch_steps(kie_ctx *ctx, const KernelArgs &a, size_t sync_bytes, in
     b.forced = a.forced ? a.forced + s0 : nullptr;
     b.out_tokens = a.out_tokens + s0;
     b.keys = a.keys + s0;
+    b.uniforms = a.uniforms ? a.uniforms + s0 : nullptr;
     if (a.logits_every_step) {   // every step's logits, each launch at its own offset
       b.logits_out = a.logits_out ? a.logits_out + size_t(s0) * ctx->m.vocab : nullptr;
       b.logits_step0 = 0;
@@ -871,6 +885,7 @@ static int launch_steps(kie_ctx *ctx, const KernelArgs &a, size_t sync_bytes, in
     const kie_model_desc &m = ctx->m;
     CK(cudaMemsetAsync(a.qkv, 0, size_t(m.n_heads + 2 * m.n_kv_heads) * m.head_dim * 8, st));
     CK(cudaMemsetAsync(a.attn_part, 0, size_t(m.n_heads) * ctx->plan.max_split * (m.head_dim + 2) * 8, st));
+    if (a.sample_t > 0.f) CK(cudaMemsetAsync(a.psum, 0, size_t(ctx->plan.n_ctas) * 8, st));
     if (s0 == 0) CK(cudaEventRecord(ctx->ev0, st));
     void *args[] = {&b};
     CK(cudaLaunchCooperativeKernel(monokernel_fn(ctx->m.dtype), dim3(ctx->plan.n_ctas),
@@ -930,6 +945,8 @@ static KernelArgs fill_args(kie_ctx *ctx, int pos0, int n, int first_token,
   a.grid_sync = ctx->grid_sync;
   a.det_sum = ctx->det_sum;
   a.l2pf_tiles = ctx->l2pf_tiles; a.l2pf_delay = ctx->l2pf_delay; a.l2pf_pace = ctx->l2pf_pace;
+  a.sample_t = 0.f; a.sample_k = 0; a.sample_p = 1.f;   // greedy unless a sampling call says otherwise
+  a.zbuf = ctx->zbuf; a.cand = ctx->cand; a.psum = ctx->psum;
   return a;
 }
 
@@ -945,9 +962,17 @@ static void set_act(const kie_ctx *ctx, KernelArgs &a, float *act) {
 }
 
 static int run(kie_ctx *ctx, int pos0, int n, const int32_t *forced_host, int first_token,
-               bool logits_every_step, float *logits_out, int32_t *out_host) {
+               bool logits_every_step, float *logits_out, int32_t *out_host,
+               const kie_sampling *smp = nullptr, const float *uniforms_host = nullptr) {
   cudaStream_t st = ctx->stream;
   KernelArgs a = fill_args(ctx, pos0, n, first_token, logits_every_step, logits_out);
+  if (smp && smp->temperature > 0.f) {
+    a.sample_t = smp->temperature;
+    a.sample_k = smp->top_k;
+    a.sample_p = smp->top_p;
+    a.uniforms = ctx->uniforms;
+    CK(cudaMemcpyAsync(ctx->uniforms, uniforms_host, size_t(n) * 4, cudaMemcpyHostToDevice, st));
+  }
   set_act(ctx, a, ctx->act);
   a.sync = ctx->sync; a.keys = ctx->keys;
   a.forced = forced_host ? ctx->tokens_in : nullptr;
@@ -1149,6 +1174,49 @@ extern "C" int kie_decode_ex(kie_ctx *ctx, int32_t n_steps, const int32_t *force
 
 extern "C" int kie_decode(kie_ctx *ctx, int32_t n_steps, int32_t *out_tokens) {
   return kie_decode_ex(ctx, n_steps, nullptr, out_tokens, nullptr);
+}
+
+extern "C" int kie_decode_sample(kie_ctx *ctx, int32_t n_steps, const kie_sampling *params,
+                                 const float *uniforms, const int32_t *forced_tokens,
+                                 int32_t *out_tokens, float *logits_out) {
+  if (!ctx || !out_tokens || !params || n_steps < 1) return KIE_ERR_INVALID;
+  if (ctx->poisoned) return KIE_ERR_POISONED;
+  const float T = params->temperature;
+  if (!(T >= 0.f) || !std::isfinite(T)) {
+    g_last_error = "temperature must be finite and >= 0";
+    return KIE_ERR_INVALID;
+  }
+  if (T == 0.f) return kie_decode_ex(ctx, n_steps, forced_tokens, out_tokens, logits_out);
+  if (params->top_k < 0 || params->top_k > KIE_MAX_TOP_K || !(params->top_p > 0.f) ||
+      !(params->top_p <= 1.f) || (params->top_k == 0 && params->top_p != 1.f)) {
+    g_last_error = "top_k must lie in [0, KIE_MAX_TOP_K] and top_p in (0, 1], with top_p 1 when top_k is 0";
+    return KIE_ERR_INVALID;
+  }
+  if (params->top_k > 0 && ctx->max_lm_rows > kMaxSampleRows) {
+    g_last_error = "vocabulary slice per SM too large for a top-k cut";
+    return KIE_ERR_INVALID;
+  }
+  if (params->top_k == 0 && ctx->plan.vbuf_floats < ctx->plan.n_ctas + 1) {
+    g_last_error = "too many SMs for sampling without a top-k cut";
+    return KIE_ERR_INVALID;
+  }
+  if (!uniforms) return KIE_ERR_INVALID;
+  for (int i = 0; i < n_steps; ++i)
+    if (!(uniforms[i] >= 0.f && uniforms[i] < 1.f)) {
+      g_last_error = "uniforms must lie in [0, 1)";
+      return KIE_ERR_INVALID;
+    }
+  if (!forced_tokens && ctx->pending < 0) return KIE_ERR_INVALID;
+  if (int64_t(ctx->pos) + n_steps > ctx->m.max_seq) return KIE_ERR_CAPACITY;
+  if (forced_tokens)
+    for (int i = 0; i < n_steps; ++i)
+      if (forced_tokens[i] < 0 || forced_tokens[i] >= ctx->m.vocab) return KIE_ERR_INVALID;
+  int rc = run(ctx, ctx->pos, n_steps, forced_tokens, ctx->pending, true, logits_out, out_tokens,
+               params, uniforms);
+  if (rc) return rc;
+  ctx->pos += n_steps;
+  ctx->pending = out_tokens[n_steps - 1];
+  return KIE_OK;
 }
 
 extern "C" int kie_destroy(kie_ctx *ctx) {

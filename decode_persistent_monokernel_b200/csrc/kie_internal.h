@@ -149,6 +149,8 @@ constexpr int kMaxRowBlock = 128;  // rows of a row block (lane l: rows l + 32 j
 constexpr int kPartialFloats = 2 * kConsumerWarps * kMaxRowBlock;  // double-buffered warp partials
 constexpr int kMaxRowSums = 1024;  // row sums a non-LM row stage keeps per CTA
 constexpr int kMaxSplit = 32;      // CTAs that share one KV head's positions (others only merge)
+constexpr int kMaxTopK = 64;       // largest top-k of the sampler (candidates kept per CTA)
+constexpr int kMaxSampleRows = 2048;  // LM-head rows per CTA that a top-k cut can sort in shared memory
 
 struct KernelArgs {
   // model
@@ -192,6 +194,14 @@ struct KernelArgs {
   int32_t *out_tokens;          // device [n_steps]
   float *logits_out;            // device [n_steps, V] or nullptr; step s writes row s - logits_step0
   int32_t logits_step0;
+  // sampling at the LM head (greedy argmax when sample_t == 0)
+  float sample_t;               // temperature
+  int32_t sample_k;             // top-k: 0 = no cut (sample_p is then 1), else 1 .. kMaxTopK
+  float sample_p;               // top-p within the top-k tokens, in (0, 1]
+  const float *uniforms;        // device [n_steps]: each step's uniform in [0, 1)
+  float *zbuf;                  // device [V]: the step's logits
+  unsigned long long *cand;     // device [n_ctas][kMaxTopK]: each CTA's largest logit keys
+  unsigned long long *psum;     // device [n_ctas]: tagged per-CTA probability sums (no top-k cut)
   uint64_t watchdog_ns;
   int32_t skip_signal_cta;      // test hook, -1 = off
   int32_t grid_sync;            // 1: every dependency wait is a grid-wide barrier

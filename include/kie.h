@@ -175,6 +175,43 @@ int kie_decode(kie_ctx *ctx, int32_t n_steps, int32_t *out_tokens);
 int kie_decode_ex(kie_ctx *ctx, int32_t n_steps, const int32_t *forced_tokens,
                   int32_t *out_tokens, float *logits_out);
 
+/* Sampling beyond greedy at the LM head, inside the same persistent kernel.
+ * Passage: the "Software versus kremik" section of the "Startup Kog dosahuje
+ * 3 000 tokenu/s..." page names LM-head sampling among the work done in one
+ * go on the device; the pages report greedy decoding only and define no
+ * sampler, so the plain one is taken, in this order:
+ *   1. temperature T > 0 scales the logits, y = z / T;
+ *   2. top_k > 0 keeps the top_k largest logits (equal logits: the lower id
+ *      first, as the argmax); top_k == 0 keeps every token;
+ *   3. top_p keeps, of those and most probable first, the smallest leading
+ *      set whose softmax(y) probability within the top-k set reaches top_p;
+ *   4. the token is drawn by inverse CDF: walking the kept tokens in
+ *      increasing id, the first whose cumulative probability, renormalised
+ *      over the kept set, exceeds that step's uniform.
+ * The random numbers are inputs: uniforms[k], in [0, 1), is step k's.  The
+ * arithmetic is fp32 (expf, sequential sums); every SM draws the same token
+ * from the same data, so the token is fed back with no extra exchange. */
+#define KIE_MAX_TOP_K 64
+typedef struct {
+  float temperature;  /* 0: greedy (the uniforms are then unused); else > 0 and finite */
+  int32_t top_k;      /* 0 .. KIE_MAX_TOP_K; 0 = no top-k cut */
+  float top_p;        /* (0, 1]; must be 1 when top_k is 0 */
+} kie_sampling;
+
+/* kie_decode_ex with the token of each step drawn per kie_sampling instead
+ * of the argmax.
+ *   params: HOST, not NULL.  temperature 0 makes this call kie_decode_ex.
+ *   uniforms: HOST array of n_steps floats in [0, 1) (not read when greedy).
+ *   forced_tokens, out_tokens, logits_out: as for kie_decode_ex; out_tokens
+ *     receives the sampled tokens, and the last becomes the pending token.
+ * KIE_ERR_INVALID, before any device work: a parameter outside the ranges
+ * above, a uniform outside [0, 1) or NaN, or a top-k cut on a model whose
+ * LM-head slice per SM exceeds 2048 rows (vocab above about 300,000 on 148
+ * SMs).  The prompt's own next token (kie_prefill) stays greedy. */
+int kie_decode_sample(kie_ctx *ctx, int32_t n_steps, const kie_sampling *params,
+                      const float *uniforms, const int32_t *forced_tokens, int32_t *out_tokens,
+                      float *logits_out);
+
 /* kie_decode_ex without any allocation.  The pages have no counterpart to
  * this call; it exists for callers that may not allocate device memory at the
  * time they decode (for example a serving thread under a fixed device-memory
