@@ -29,7 +29,7 @@ namespace kie {
 size_t monokernel_smem_bytes(int ring_slots, int vbuf_floats, int part_floats);
 int monokernel_threads();
 bool monokernel_profiled();
-const void *monokernel_fn(int dtype);
+const void *monokernel_fn(int dtype, bool sample);
 cudaError_t launch_repack(const uint16_t *src, uint8_t *dst, const RepackJob *jobs, int njobs,
                           cudaStream_t st);
 }  // namespace kie
@@ -671,15 +671,17 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
     return fail(KIE_ERR_INVALID);
   }
   Plan &P = ctx->plan;
-  const void *fn = monokernel_fn(m.dtype);
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(P.smem));
-  if (e != cudaSuccess) return fail(cuda_fail(nullptr, "cudaFuncSetAttribute", e));
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, monokernel_threads(), P.smem);
-  if (e != cudaSuccess) return fail(cuda_fail(nullptr, "occupancy query", e));
-  if (per_sm < 1) {
-    g_last_error = "persistent CTA does not fit on an SM";
-    return fail(KIE_ERR_NOT_RESIDENT);
+  for (bool sample : {false, true}) {   // the greedy and the sampling instance
+    const void *fn = monokernel_fn(m.dtype, sample);
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(P.smem));
+    if (e != cudaSuccess) return fail(cuda_fail(nullptr, "cudaFuncSetAttribute", e));
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, monokernel_threads(), P.smem);
+    if (e != cudaSuccess) return fail(cuda_fail(nullptr, "occupancy query", e));
+    if (per_sm < 1) {
+      g_last_error = "persistent CTA does not fit on an SM";
+      return fail(KIE_ERR_NOT_RESIDENT);
+    }
   }
 
   const Layout Ly = make_layout(m);
@@ -888,7 +890,7 @@ static int launch_steps(kie_ctx *ctx, const KernelArgs &a, size_t sync_bytes, in
     if (a.sample_t > 0.f) CK(cudaMemsetAsync(a.psum, 0, size_t(ctx->plan.n_ctas) * 8, st));
     if (s0 == 0) CK(cudaEventRecord(ctx->ev0, st));
     void *args[] = {&b};
-    CK(cudaLaunchCooperativeKernel(monokernel_fn(ctx->m.dtype), dim3(ctx->plan.n_ctas),
+    CK(cudaLaunchCooperativeKernel(monokernel_fn(ctx->m.dtype, a.sample_t > 0.f), dim3(ctx->plan.n_ctas),
                                    dim3(monokernel_threads()), args, ctx->plan.smem, st));
     if (s0 + c < n) {   // the next launch needs this one's last token
       CK(cudaMemcpyAsync(&status, a.sync + SY_STATUS * kSyncStride, 4, cudaMemcpyDeviceToHost, st));

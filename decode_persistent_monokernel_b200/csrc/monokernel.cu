@@ -233,10 +233,11 @@ __device__ __forceinline__ uint32_t *sync_at(const KernelArgs &a, int slot) {
   return a.sync + slot * kSyncStride;
 }
 
-__device__ void raise_error(const KernelArgs &a, uint32_t code) {
-  atomicCAS(sync_at(a, SY_STATUS), 0u, code);
-  atomicExch(sync_at(a, SY_ABORT), 1u);
+__device__ __forceinline__ void raise_error_at(uint32_t *sync, uint32_t code) {
+  atomicCAS(sync + SY_STATUS * kSyncStride, 0u, code);
+  atomicExch(sync + SY_ABORT * kSyncStride, 1u);
 }
+__device__ __forceinline__ void raise_error(const KernelArgs &a, uint32_t code) { raise_error_at(a.sync, code); }
 
 // Watchdog arithmetic uses the SM cycle counter (cheap to read); the limit in
 // cycles assumes at most 2 GHz, so a wait gives up after at least watchdog_ns.
@@ -268,14 +269,15 @@ __device__ bool wait_counter(const KernelArgs &a, const uint32_t *ctr, uint32_t 
 }
 
 // Bounded wait until the tagged word *p carries `tag`; its value goes to
-// out.  False on watchdog expiry or abort.
-__device__ bool wait_tagged(const KernelArgs &a, const unsigned long long *p, uint32_t tag,
-                            uint32_t where, float &out) {
+// out.  False on watchdog expiry or abort (sync: the counters' base).
+__device__ __forceinline__ bool wait_tagged_at(uint32_t *sync, uint64_t watchdog_ns,
+                                               const unsigned long long *p, uint32_t tag,
+                                               uint32_t where, float &out) {
   unsigned long long w = ld_relaxed_u64(p);
   if (uint32_t(w >> 32) != tag) {
-    const long long t0 = clock64(), limit = (long long)a.watchdog_ns * 2;
+    const long long t0 = clock64(), limit = (long long)watchdog_ns * 2;
     long long next_poll = kAbortPollCycles;
-    const uint32_t *abortp = sync_at(a, SY_ABORT);
+    const uint32_t *abortp = sync + SY_ABORT * kSyncStride;
     for (;;) {
       w = ld_relaxed_u64(p);
       if (uint32_t(w >> 32) == tag) break;
@@ -284,7 +286,7 @@ __device__ bool wait_tagged(const KernelArgs &a, const unsigned long long *p, ui
         next_poll = el + kAbortPollCycles;
         if (ld_relaxed(abortp)) return false;
         if (el > limit) {
-          raise_error(a, DE_TIMEOUT_COUNTER | (where << 8));
+          raise_error_at(sync, DE_TIMEOUT_COUNTER | (where << 8));
           return false;
         }
       }
@@ -292,6 +294,10 @@ __device__ bool wait_tagged(const KernelArgs &a, const unsigned long long *p, ui
   }
   out = __uint_as_float(uint32_t(w));
   return true;
+}
+__device__ __forceinline__ bool wait_tagged(const KernelArgs &a, const unsigned long long *p, uint32_t tag,
+                                            uint32_t where, float &out) {
+  return wait_tagged_at(a.sync, a.watchdog_ns, p, tag, where, out);
 }
 
 // Bounded wait on an mbarrier phase.
@@ -463,8 +469,274 @@ struct Producer {
   }
 };
 
+// ---- logit keys: (order-preserving bits of the value) << 32 | (~row), so
+// that a larger key is a larger logit, and among equal logits the lower
+// row; every finite or infinite logit's key is above 0
+__device__ __forceinline__ unsigned long long logit_key(float v, int row) {
+  const uint32_t fb = __float_as_uint(v);
+  const uint32_t ord = (fb & 0x80000000u) ? ~fb : (fb | 0x80000000u);
+  return (static_cast<unsigned long long>(ord) << 32) | (0xffffffffu - uint32_t(row));
+}
+__device__ __forceinline__ float key_value(unsigned long long key) {
+  const uint32_t ord = uint32_t(key >> 32);
+  return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord);
+}
+__device__ __forceinline__ int key_row(unsigned long long key) {
+  return int(0xffffffffu - uint32_t(key & 0xffffffffull));
+}
+
+// ------------------------------------------------------------------ sampling
+// Sampling beyond greedy (temperature, top-k, top-p; the uniform of each step
+// is an input).  Every CTA computes the same token from the same global data,
+// so no further exchange is needed once it is drawn.  These run once per
+// token and exist only in the sampling instance of the kernel.
+
+// What the sampler reads.
+struct SampleArgs {
+  const float *zbuf;
+  unsigned long long *cand, *psum;
+  const unsigned long long *keys;
+  const float *uniforms;
+  const StageCta *stage_cta;
+  uint32_t *sync;
+  uint64_t watchdog_ns;
+  float t, p;                // temperature, top-p
+  int32_t k, vocab, n_ctas;  // top-k
+};
+
+// Before the token barrier, top-k mode: this CTA's sample_k largest logit
+// keys, largest first, into cand[cta] (its LM-head rows' keys, read back
+// from zbuf and sorted in shared memory by a descending bitonic sort; 0
+// pads a slice shorter than k).
+__device__ __forceinline__ void local_topk(const SampleArgs g, const Smem s, int tid, int cta) {
+  const StageCta &c = s.misc->sc[ST_LM];
+  const int n = c.nout;
+  int np = 2;
+  while (np < n) np <<= 1;   // n <= kMaxSampleRows (checked on the host): fits `part`
+  unsigned long long *kp = reinterpret_cast<unsigned long long *>(s.part);
+  for (int i = tid; i < np; i += kNC)
+    kp[i] = i < n ? logit_key(__ldcg(g.zbuf + c.row0 + i), c.row0 + i) : 0ull;
+  cbar();
+  for (int size = 2; size <= np; size <<= 1)
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < np; i += kNC) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const unsigned long long x = kp[i], y = kp[j];
+          if ((i & size) == 0 ? x < y : x > y) { kp[i] = y; kp[j] = x; }
+        }
+      }
+      cbar();
+    }
+  for (int j = tid; j < g.k; j += kNC)
+    g.cand[size_t(cta) * kMaxTopK + j] = j < n ? kp[j] : 0ull;
+}
+
+// After the token barrier, top-k mode.  The k = min(sample_k, V) largest
+// keys of all CTAs' candidates: a radix select over 8-bit digits from the
+// top keeps a prefix and the number of keys still needed below it, and
+// stops once the keys sharing the prefix are exactly those; the kept keys
+// are gathered and ranked (largest first) in shared memory.  Thread 0 then
+// weighs them exp((z - z_max) / T), cuts the most probable leading set
+// reaching top_p of their sum, and draws by inverse CDF in token order.
+__device__ __forceinline__ int sample_topk(const SampleArgs g, const Smem s, int tid, int step) {
+  const int warp = tid >> 5, lane = tid & 31;
+  const int kc = g.k, k = min(kc, g.vocab), total = g.n_ctas * kc;
+  uint32_t *hist = reinterpret_cast<uint32_t *>(s.part);                 // [256]
+  unsigned long long *sel = reinterpret_cast<unsigned long long *>(s.part + 256);  // [kMaxTopK]
+  unsigned long long *srt = sel + kMaxTopK;                              // [kMaxTopK]
+  float *ev = reinterpret_cast<float *>(srt + kMaxTopK);                 // [kMaxTopK]
+  int *byrow = reinterpret_cast<int *>(ev + kMaxTopK);                   // [kMaxTopK]
+  auto cand_at = [&](int q) { return __ldcg(g.cand + size_t(q / kc) * kMaxTopK + q % kc); };
+  unsigned long long prefix = 0, mask = 0;
+  int need = k;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kNC) hist[i] = 0;
+    cbar();
+    for (int q = tid; q < total; q += kNC) {
+      const unsigned long long key = cand_at(q);
+      if (key != 0ull && (key & mask) == prefix) atomicAdd(&hist[uint32_t(key >> shift) & 255u], 1u);
+    }
+    cbar();
+    if (warp == 0) {
+      // lane l holds bins 255 - 8 l - e (e < 8): lane 0 the highest digits
+      uint32_t h[8], tot = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { h[e] = hist[255 - 8 * lane - e]; tot += h[e]; }
+      uint32_t incl = tot;
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const uint32_t above = incl - tot;
+      if (above < uint32_t(need) && uint32_t(need) <= incl) {   // exactly one lane
+        uint32_t acc = above;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (acc + h[e] >= uint32_t(need)) {
+            s.misc->sel[0] = 255 - 8 * lane - e;
+            s.misc->sel[1] = need - int(acc);
+            s.misc->sel[2] = int(h[e]);
+            break;
+          }
+          acc += h[e];
+        }
+      }
+    }
+    cbar();
+    prefix |= static_cast<unsigned long long>(s.misc->sel[0]) << shift;
+    mask |= 0xffull << shift;
+    need = s.misc->sel[1];
+    const bool done = s.misc->sel[2] == need;   // every key with this prefix is taken
+    cbar();
+    if (done) break;
+  }
+  if (tid == 0) s.misc->sel[3] = 0;
+  cbar();
+  for (int q = tid; q < total; q += kNC) {
+    const unsigned long long key = cand_at(q);
+    if (key != 0ull && (key & mask) >= prefix) {
+      const int slot = atomicAdd(&s.misc->sel[3], 1);
+      if (slot < kMaxTopK) sel[slot] = key;
+    }
+  }
+  cbar();
+  const int m = min(s.misc->sel[3], kMaxTopK);   // k, the keys being distinct
+  if (tid < m) {
+    const unsigned long long x = sel[tid];
+    int r = 0;
+    for (int i = 0; i < m; ++i) r += sel[i] > x;
+    srt[r] = x;
+  }
+  cbar();
+  if (tid == 0) {
+    const float zmax = key_value(srt[0]), temp = g.t;
+    float S = 0.f;
+    for (int j = 0; j < m; ++j) {
+      ev[j] = expf((key_value(srt[j]) - zmax) / temp);
+      S += ev[j];
+    }
+    int mm = m;
+    if (g.p < 1.f) {   // most probable first, until top_p of the mass
+      const float lim = g.p * S;
+      float c = 0.f;
+      mm = 0;
+      do { c += ev[mm]; ++mm; } while (mm < m && c < lim);
+    }
+    s.misc->sel[3] = mm;
+  }
+  cbar();
+  const int mm = s.misc->sel[3];
+  if (tid < mm) {
+    const int row = key_row(srt[tid]);
+    int r = 0;
+    for (int i = 0; i < mm; ++i) r += key_row(srt[i]) < row;
+    byrow[r] = tid;
+  }
+  cbar();
+  if (tid == 0) {
+    float S = 0.f;
+    for (int r = 0; r < mm; ++r) S += ev[byrow[r]];
+    const float target = __ldg(g.uniforms + step) * S;
+    int tk = key_row(srt[byrow[mm - 1]]);
+    float c = 0.f;
+    for (int r = 0; r < mm; ++r) {
+      c += ev[byrow[r]];
+      if (c > target) { tk = key_row(srt[byrow[r]]); break; }
+    }
+    s.misc->sel[0] = tk;
+  }
+  cbar();
+  return s.misc->sel[0];
+}
+
+// After the token barrier, no top-k cut (top_p 1): every token, in token
+// order.  With z_max from the argmax key, each CTA adds exp((z - z_max) / T)
+// over its LM-head rows (a fixed order) and publishes the sum as a tagged
+// word; every CTA walks the CTAs' sums in order (their row slices are
+// consecutive) to the slice that holds the draw, and warp 0 walks that
+// slice's rows: each lane a run of rows, a scan of the runs' sums, then the
+// lane whose run crosses walks it.  A crossing lost to rounding falls back
+// to the slice's last row.  Returns -1 if a wait gave up.
+__device__ __forceinline__ int sample_full(const SampleArgs g, const Smem s, int tid, int cta, int step,
+                                        uint32_t lm_count) {
+  const int warp = tid >> 5, lane = tid & 31;
+  const float zmax = key_value(__ldcg(g.keys + step)), temp = g.t;
+  const StageCta &c = s.misc->sc[ST_LM];
+  float e = 0.f;
+  for (int i = tid; i < c.nout; i += kNC) e += expf((__ldcg(g.zbuf + c.row0 + i) - zmax) / temp);
+  for (int o = 16; o; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+  if (lane == 0) s.misc->red_v[warp] = e;
+  cbar();
+  const uint32_t tag = lm_count;
+  if (tid == 0) {
+    float t = 0.f;
+    for (int w = 0; w < kConsumerWarps; ++w) t += s.misc->red_v[w];
+    st_tagged(g.psum + cta, t, tag);
+  }
+  float *ps = s.vbuf;
+  bool ok = true;
+  for (int q = tid; q < g.n_ctas; q += kNC) ok = ok && wait_tagged_at(g.sync, g.watchdog_ns, g.psum + q, tag, 0x90, ps[q]);
+  if (!ok) s.misc->abort = 1;
+  cbar();
+  if (s.misc->abort != 0) return -1;
+  if (tid == 0) {
+    float S = 0.f;
+    for (int q = 0; q < g.n_ctas; ++q) S += ps[q];
+    const float target = __ldg(g.uniforms + step) * S;
+    int cs = -1;
+    float before = 0.f;
+    for (int q = 0; q < g.n_ctas; ++q) {
+      if (ps[q] > 0.f) cs = q;
+      if (before + ps[q] > target) { cs = q; break; }
+      before += ps[q];
+    }
+    if (cs < 0) cs = g.n_ctas - 1;
+    before = 0.f;
+    for (int q = 0; q < cs; ++q) before += ps[q];
+    s.misc->sel[0] = cs;
+    s.misc->self = before;
+    ps[g.n_ctas] = target;
+  }
+  cbar();
+  if (warp == 0) {
+    const int cs = s.misc->sel[0];
+    const float target = ps[g.n_ctas];
+    const StageCta sc = g.stage_cta[size_t(ST_LM) * g.n_ctas + cs];
+    const int ch = (sc.nout + 31) / 32, i0 = min(lane * ch, sc.nout), i1 = min(i0 + ch, sc.nout);
+    float run = 0.f;
+    for (int i = i0; i < i1; ++i) run += expf((__ldcg(g.zbuf + sc.row0 + i) - zmax) / temp);
+    float incl = run;
+    for (int o = 1; o < 32; o <<= 1) {
+      const float t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const float base = s.misc->self + (incl - run);
+    const unsigned ball = __ballot_sync(0xffffffffu, i1 > i0 && base + run > target);
+    int tk = sc.row0 + sc.nout - 1;
+    if (ball) {
+      const int src = __ffs(ball) - 1;
+      int found = sc.row0 + i1 - 1;
+      if (lane == src) {
+        float cum = base;
+        for (int i = i0; i < i1; ++i) {
+          cum += expf((__ldcg(g.zbuf + sc.row0 + i) - zmax) / temp);
+          if (cum > target) { found = sc.row0 + i; break; }
+        }
+      }
+      tk = __shfl_sync(0xffffffffu, found, src);
+    }
+    if (lane == 0) s.misc->sel[1] = tk;
+  }
+  cbar();
+  return s.misc->sel[1];
+}
+
 // ------------------------------------------------------------------ consumer
-template <typename T>
+// SAMPLE: the kernel instance that draws tokens (temperature > 0).  The greedy
+// instance holds none of the sampling code: code that never runs still changed
+// the persistent loop's register allocation and cost the greedy path ~2 %.
+template <typename T, bool SAMPLE>
 struct Consumer {
   const KernelArgs &a;
   Smem s;
@@ -1164,22 +1436,6 @@ struct Consumer {
     KP_END(t_gemv, PF_GEMV_K + k);
   }
 
-  // ---- logit keys: (order-preserving bits of the value) << 32 | (~row), so
-  // that a larger key is a larger logit, and among equal logits the lower
-  // row; every finite or infinite logit's key is above 0
-  static __device__ __forceinline__ unsigned long long logit_key(float v, int row) {
-    const uint32_t fb = __float_as_uint(v);
-    const uint32_t ord = (fb & 0x80000000u) ? ~fb : (fb | 0x80000000u);
-    return (static_cast<unsigned long long>(ord) << 32) | (0xffffffffu - uint32_t(row));
-  }
-  static __device__ __forceinline__ float key_value(unsigned long long key) {
-    const uint32_t ord = uint32_t(key >> 32);
-    return __uint_as_float((ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord);
-  }
-  static __device__ __forceinline__ int key_row(unsigned long long key) {
-    return int(0xffffffffu - uint32_t(key & 0xffffffffull));
-  }
-
   // ---- LM head epilogue: logits and the CTA's share of the argmax
   // lm_row() takes each logit as its row block is reduced (thread `row` of the
   // block); lm_fold() then folds the threads' (value, index) pairs into one
@@ -1189,7 +1445,7 @@ struct Consumer {
   __device__ __forceinline__ void lm_row(int i, float v, float &best, int &bidx) {
     const int row = s.misc->sc[ST_LM].row0 + i;
     if (a.logits_out) a.logits_out[size_t(step - a.logits_step0) * a.vocab + row] = v;
-    if (a.sample_t > 0.f) a.zbuf[row] = v;
+    if (SAMPLE) a.zbuf[row] = v;
     if (v != v) raise_error(a, DE_NONFINITE | (uint32_t(step & 0xffff) << 8));
     if (v > best || (v == best && row < bidx)) { best = v; bidx = row; }
   }
@@ -1212,233 +1468,9 @@ struct Consumer {
     }
   }
 
-  // ---- sampling beyond greedy (temperature, top-k, top-p; the uniform of
-  // each step is an input).  Every CTA computes the same token from the same
-  // global data, so no further exchange is needed once it is drawn.
-
-  // Before the token barrier, top-k mode: this CTA's sample_k largest logit
-  // keys, largest first, into cand[cta] (its LM-head rows' keys, read back
-  // from zbuf and sorted in shared memory by a descending bitonic sort; 0
-  // pads a slice shorter than k).
-  __device__ void local_topk() {
-    const StageCta &c = s.misc->sc[ST_LM];
-    const int n = c.nout;
-    int np = 2;
-    while (np < n) np <<= 1;   // n <= kMaxSampleRows (checked on the host): fits `part`
-    unsigned long long *kp = reinterpret_cast<unsigned long long *>(s.part);
-    for (int i = tid; i < np; i += kNC)
-      kp[i] = i < n ? logit_key(__ldcg(a.zbuf + c.row0 + i), c.row0 + i) : 0ull;
-    cbar();
-    for (int size = 2; size <= np; size <<= 1)
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < np; i += kNC) {
-          const int j = i ^ stride;
-          if (j > i) {
-            const unsigned long long x = kp[i], y = kp[j];
-            if ((i & size) == 0 ? x < y : x > y) { kp[i] = y; kp[j] = x; }
-          }
-        }
-        cbar();
-      }
-    for (int j = tid; j < a.sample_k; j += kNC)
-      a.cand[size_t(cta) * kMaxTopK + j] = j < n ? kp[j] : 0ull;
-  }
-
-  // After the token barrier, top-k mode.  The k = min(sample_k, V) largest
-  // keys of all CTAs' candidates: a radix select over 8-bit digits from the
-  // top keeps a prefix and the number of keys still needed below it, and
-  // stops once the keys sharing the prefix are exactly those; the kept keys
-  // are gathered and ranked (largest first) in shared memory.  Thread 0 then
-  // weighs them exp((z - z_max) / T), cuts the most probable leading set
-  // reaching top_p of their sum, and draws by inverse CDF in token order.
-  __device__ int sample_topk() {
-    const int kc = a.sample_k, k = min(kc, a.vocab), total = a.n_ctas * kc;
-    uint32_t *hist = reinterpret_cast<uint32_t *>(s.part);                 // [256]
-    unsigned long long *sel = reinterpret_cast<unsigned long long *>(s.part + 256);  // [kMaxTopK]
-    unsigned long long *srt = sel + kMaxTopK;                              // [kMaxTopK]
-    float *ev = reinterpret_cast<float *>(srt + kMaxTopK);                 // [kMaxTopK]
-    int *byrow = reinterpret_cast<int *>(ev + kMaxTopK);                   // [kMaxTopK]
-    auto cand_at = [&](int q) { return __ldcg(a.cand + size_t(q / kc) * kMaxTopK + q % kc); };
-    unsigned long long prefix = 0, mask = 0;
-    int need = k;
-    for (int shift = 56; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += kNC) hist[i] = 0;
-      cbar();
-      for (int q = tid; q < total; q += kNC) {
-        const unsigned long long key = cand_at(q);
-        if (key != 0ull && (key & mask) == prefix) atomicAdd(&hist[uint32_t(key >> shift) & 255u], 1u);
-      }
-      cbar();
-      if (warp == 0) {
-        // lane l holds bins 255 - 8 l - e (e < 8): lane 0 the highest digits
-        uint32_t h[8], tot = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) { h[e] = hist[255 - 8 * lane - e]; tot += h[e]; }
-        uint32_t incl = tot;
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t;
-        }
-        const uint32_t above = incl - tot;
-        if (above < uint32_t(need) && uint32_t(need) <= incl) {   // exactly one lane
-          uint32_t acc = above;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if (acc + h[e] >= uint32_t(need)) {
-              s.misc->sel[0] = 255 - 8 * lane - e;
-              s.misc->sel[1] = need - int(acc);
-              s.misc->sel[2] = int(h[e]);
-              break;
-            }
-            acc += h[e];
-          }
-        }
-      }
-      cbar();
-      prefix |= static_cast<unsigned long long>(s.misc->sel[0]) << shift;
-      mask |= 0xffull << shift;
-      need = s.misc->sel[1];
-      const bool done = s.misc->sel[2] == need;   // every key with this prefix is taken
-      cbar();
-      if (done) break;
-    }
-    if (tid == 0) s.misc->sel[3] = 0;
-    cbar();
-    for (int q = tid; q < total; q += kNC) {
-      const unsigned long long key = cand_at(q);
-      if (key != 0ull && (key & mask) >= prefix) {
-        const int slot = atomicAdd(&s.misc->sel[3], 1);
-        if (slot < kMaxTopK) sel[slot] = key;
-      }
-    }
-    cbar();
-    const int m = min(s.misc->sel[3], kMaxTopK);   // k, the keys being distinct
-    if (tid < m) {
-      const unsigned long long x = sel[tid];
-      int r = 0;
-      for (int i = 0; i < m; ++i) r += sel[i] > x;
-      srt[r] = x;
-    }
-    cbar();
-    if (tid == 0) {
-      const float zmax = key_value(srt[0]), temp = a.sample_t;
-      float S = 0.f;
-      for (int j = 0; j < m; ++j) {
-        ev[j] = expf((key_value(srt[j]) - zmax) / temp);
-        S += ev[j];
-      }
-      int mm = m;
-      if (a.sample_p < 1.f) {   // most probable first, until top_p of the mass
-        const float lim = a.sample_p * S;
-        float c = 0.f;
-        mm = 0;
-        do { c += ev[mm]; ++mm; } while (mm < m && c < lim);
-      }
-      s.misc->sel[3] = mm;
-    }
-    cbar();
-    const int mm = s.misc->sel[3];
-    if (tid < mm) {
-      const int row = key_row(srt[tid]);
-      int r = 0;
-      for (int i = 0; i < mm; ++i) r += key_row(srt[i]) < row;
-      byrow[r] = tid;
-    }
-    cbar();
-    if (tid == 0) {
-      float S = 0.f;
-      for (int r = 0; r < mm; ++r) S += ev[byrow[r]];
-      const float target = __ldg(a.uniforms + step) * S;
-      int tk = key_row(srt[byrow[mm - 1]]);
-      float c = 0.f;
-      for (int r = 0; r < mm; ++r) {
-        c += ev[byrow[r]];
-        if (c > target) { tk = key_row(srt[byrow[r]]); break; }
-      }
-      s.misc->sel[0] = tk;
-    }
-    cbar();
-    return s.misc->sel[0];
-  }
-
-  // After the token barrier, no top-k cut (top_p 1): every token, in token
-  // order.  With z_max from the argmax key, each CTA adds exp((z - z_max) / T)
-  // over its LM-head rows (a fixed order) and publishes the sum as a tagged
-  // word; every CTA walks the CTAs' sums in order (their row slices are
-  // consecutive) to the slice that holds the draw, and warp 0 walks that
-  // slice's rows: each lane a run of rows, a scan of the runs' sums, then the
-  // lane whose run crosses walks it.  A crossing lost to rounding falls back
-  // to the slice's last row.  Returns -1 if a wait gave up.
-  __device__ int sample_full() {
-    const float zmax = key_value(__ldcg(a.keys + step)), temp = a.sample_t;
-    const StageCta &c = s.misc->sc[ST_LM];
-    float e = 0.f;
-    for (int i = tid; i < c.nout; i += kNC) e += expf((__ldcg(a.zbuf + c.row0 + i) - zmax) / temp);
-    for (int o = 16; o; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-    if (lane == 0) s.misc->red_v[warp] = e;
-    cbar();
-    const uint32_t tag = lm_count;
-    if (tid == 0) {
-      float t = 0.f;
-      for (int w = 0; w < kConsumerWarps; ++w) t += s.misc->red_v[w];
-      st_tagged(a.psum + cta, t, tag);
-    }
-    float *ps = s.vbuf;
-    bool ok = true;
-    for (int q = tid; q < a.n_ctas; q += kNC) ok = ok && wait_tagged(a, a.psum + q, tag, 0x90, ps[q]);
-    if (!ok) s.misc->abort = 1;
-    cbar();
-    if (aborted()) return -1;
-    if (tid == 0) {
-      float S = 0.f;
-      for (int q = 0; q < a.n_ctas; ++q) S += ps[q];
-      const float target = __ldg(a.uniforms + step) * S;
-      int cs = -1;
-      float before = 0.f;
-      for (int q = 0; q < a.n_ctas; ++q) {
-        if (ps[q] > 0.f) cs = q;
-        if (before + ps[q] > target) { cs = q; break; }
-        before += ps[q];
-      }
-      if (cs < 0) cs = a.n_ctas - 1;
-      before = 0.f;
-      for (int q = 0; q < cs; ++q) before += ps[q];
-      s.misc->sel[0] = cs;
-      s.misc->self = before;
-      ps[a.n_ctas] = target;
-    }
-    cbar();
-    if (warp == 0) {
-      const int cs = s.misc->sel[0];
-      const float target = ps[a.n_ctas];
-      const StageCta sc = a.stage_cta[size_t(ST_LM) * a.n_ctas + cs];
-      const int ch = (sc.nout + 31) / 32, i0 = min(lane * ch, sc.nout), i1 = min(i0 + ch, sc.nout);
-      float run = 0.f;
-      for (int i = i0; i < i1; ++i) run += expf((__ldcg(a.zbuf + sc.row0 + i) - zmax) / temp);
-      float incl = run;
-      for (int o = 1; o < 32; o <<= 1) {
-        const float t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      const float base = s.misc->self + (incl - run);
-      const unsigned ball = __ballot_sync(0xffffffffu, i1 > i0 && base + run > target);
-      int tk = sc.row0 + sc.nout - 1;
-      if (ball) {
-        const int src = __ffs(ball) - 1;
-        int found = sc.row0 + i1 - 1;
-        if (lane == src) {
-          float cum = base;
-          for (int i = i0; i < i1; ++i) {
-            cum += expf((__ldcg(a.zbuf + sc.row0 + i) - zmax) / temp);
-            if (cum > target) { found = sc.row0 + i; break; }
-          }
-        }
-        tk = __shfl_sync(0xffffffffu, found, src);
-      }
-      if (lane == 0) s.misc->sel[1] = tk;
-    }
-    cbar();
-    return s.misc->sel[1];
+  __device__ __forceinline__ SampleArgs sample_args() const {
+    return SampleArgs{a.zbuf,      a.cand, a.psum,        a.keys,     a.uniforms, a.stage_cta, a.sync,
+                      a.watchdog_ns, a.sample_t, a.sample_p, a.sample_k, a.vocab,    a.n_ctas};
   }
 
   __device__ void run() {
@@ -1586,13 +1618,16 @@ struct Consumer {
           gemv_rows(ST_LM, s.vbuf, to_lm);
           if (aborted()) goto done;
           lm_fold(best, bidx);
-          if (a.sample_t > 0.f && a.sample_k > 0) local_topk();
+          if constexpr (SAMPLE) {
+            if (a.sample_k > 0) local_topk(sample_args(), s, tid, cta);
+          }
         }
         signal(SY_TOK);
         if (!gate(SY_TOK, lm_count * nc, 0x80, 3)) goto done;
         int next;
-        if (a.sample_t > 0.f) {
-          next = a.sample_k > 0 ? sample_topk() : sample_full();
+        if constexpr (SAMPLE) {
+          next = a.sample_k > 0 ? sample_topk(sample_args(), s, tid, step)
+                                : sample_full(sample_args(), s, tid, cta, step, lm_count);
           if (next < 0) goto done;
         } else {
           next = key_row(__ldcg(a.keys + step));
@@ -1607,7 +1642,7 @@ struct Consumer {
   }
 };
 
-template <typename T>
+template <typename T, bool SAMPLE>
 __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int tid = threadIdx.x;
@@ -1654,7 +1689,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
     }
     __syncwarp();
   } else {
-    Consumer<T> c(a, s, tid, cta);
+    Consumer<T, SAMPLE> c(a, s, tid, cta);
     c.run();
     // a CTA that gave up makes every other CTA (and its own producer) leave
     if (tid == 0 && c.aborted()) atomicExch(sync_at(a, SY_ABORT), 1u);
@@ -1743,9 +1778,12 @@ bool monokernel_profiled() {
 #endif
 }
 
-const void *monokernel_fn(int dtype) {
-  return dtype == 0 ? reinterpret_cast<const void *>(&monokernel<__half>)
-                    : reinterpret_cast<const void *>(&monokernel<__nv_bfloat16>);
+const void *monokernel_fn(int dtype, bool sample) {
+  if (sample)
+    return dtype == 0 ? reinterpret_cast<const void *>(&monokernel<__half, true>)
+                      : reinterpret_cast<const void *>(&monokernel<__nv_bfloat16, true>);
+  return dtype == 0 ? reinterpret_cast<const void *>(&monokernel<__half, false>)
+                    : reinterpret_cast<const void *>(&monokernel<__nv_bfloat16, false>);
 }
 
 cudaError_t launch_repack(const uint16_t *src, uint8_t *dst, const RepackJob *jobs, int njobs,
