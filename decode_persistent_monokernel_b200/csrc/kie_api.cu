@@ -29,7 +29,9 @@ namespace kie {
 size_t monokernel_smem_bytes(int ring_slots, int vbuf_floats, int part_floats);
 int monokernel_threads();
 bool monokernel_profiled();
-const void *monokernel_fn(int dtype, bool sample);
+// variant bits: 1 = the general instance (lane models, grid-barrier and
+// exact-sum ablations, L2 look-ahead), 2 = the sampler compiled in
+const void *monokernel_fn(int dtype, int variant);
 cudaError_t launch_repack(const uint16_t *src, uint8_t *dst, const RepackJob *jobs, int njobs,
                           cudaStream_t st);
 }  // namespace kie
@@ -671,8 +673,8 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
     return fail(KIE_ERR_INVALID);
   }
   Plan &P = ctx->plan;
-  for (bool sample : {false, true}) {   // the greedy and the sampling instance
-    const void *fn = monokernel_fn(m.dtype, sample);
+  for (int variant = 0; variant < 4; ++variant) {   // every kernel instance
+    const void *fn = monokernel_fn(m.dtype, variant);
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(P.smem));
     if (e != cudaSuccess) return fail(cuda_fail(nullptr, "cudaFuncSetAttribute", e));
     int per_sm = 0;
@@ -847,6 +849,14 @@ static int steps_per_launch(const kie_ctx *ctx) {
   return int(std::max<int64_t>(n, 1));
 }
 
+// The kernel instance for these arguments: the dense one unless a lane
+// model, an ablation switch or the L2 look-ahead needs the general one; the
+// sampler's when a temperature is set.
+static int kernel_variant(const KernelArgs &a) {
+  const bool general = a.n_lanes > 1 || a.grid_sync || a.det_sum || a.l2pf_tiles > 0;
+  return (general ? 1 : 0) | (a.sample_t > 0.f ? 2 : 0);
+}
+
 // Runs the n steps described by `a` (forced tokens, output tokens, argmax
 // keys and logits of the whole call) as one or more launches.  Each launch
 // takes the next run of steps and starts from the previous launch's last
@@ -890,7 +900,7 @@ static int launch_steps(kie_ctx *ctx, const KernelArgs &a, size_t sync_bytes, in
     if (a.sample_t > 0.f) CK(cudaMemsetAsync(a.psum, 0, size_t(ctx->plan.n_ctas) * 8, st));
     if (s0 == 0) CK(cudaEventRecord(ctx->ev0, st));
     void *args[] = {&b};
-    CK(cudaLaunchCooperativeKernel(monokernel_fn(ctx->m.dtype, a.sample_t > 0.f), dim3(ctx->plan.n_ctas),
+    CK(cudaLaunchCooperativeKernel(monokernel_fn(ctx->m.dtype, kernel_variant(a)), dim3(ctx->plan.n_ctas),
                                    dim3(monokernel_threads()), args, ctx->plan.smem, st));
     if (s0 + c < n) {   // the next launch needs this one's last token
       CK(cudaMemcpyAsync(&status, a.sync + SY_STATUS * kSyncStride, 4, cudaMemcpyDeviceToHost, st));
