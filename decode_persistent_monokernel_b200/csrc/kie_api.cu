@@ -30,8 +30,10 @@ size_t monokernel_smem_bytes(int ring_slots, int vbuf_floats, int part_floats);
 int monokernel_threads();
 bool monokernel_profiled();
 // variant bits: 1 = the general instance (lane models, grid-barrier and
-// exact-sum ablations, L2 look-ahead), 2 = the sampler compiled in
-const void *monokernel_fn(int dtype, int variant);
+// exact-sum ablations, L2 look-ahead), 2 = the sampler compiled in; G, dh:
+// the attention shape (query heads per KV head, head size), for which the
+// dense greedy instance may be specialised
+const void *monokernel_fn(int dtype, int variant, int G, int dh);
 cudaError_t launch_repack(const uint16_t *src, uint8_t *dst, const RepackJob *jobs, int njobs,
                           cudaStream_t st);
 }  // namespace kie
@@ -673,8 +675,8 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
     return fail(KIE_ERR_INVALID);
   }
   Plan &P = ctx->plan;
-  for (int variant = 0; variant < 4; ++variant) {   // every kernel instance
-    const void *fn = monokernel_fn(m.dtype, variant);
+  for (int variant = 0; variant < 4; ++variant) {   // every kernel instance this model can launch
+    const void *fn = monokernel_fn(m.dtype, variant, m.n_heads / m.n_kv_heads, m.head_dim);
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(P.smem));
     if (e != cudaSuccess) return fail(cuda_fail(nullptr, "cudaFuncSetAttribute", e));
     int per_sm = 0;
@@ -900,7 +902,9 @@ static int launch_steps(kie_ctx *ctx, const KernelArgs &a, size_t sync_bytes, in
     if (a.sample_t > 0.f) CK(cudaMemsetAsync(a.psum, 0, size_t(ctx->plan.n_ctas) * 8, st));
     if (s0 == 0) CK(cudaEventRecord(ctx->ev0, st));
     void *args[] = {&b};
-    CK(cudaLaunchCooperativeKernel(monokernel_fn(ctx->m.dtype, kernel_variant(a)), dim3(ctx->plan.n_ctas),
+    CK(cudaLaunchCooperativeKernel(monokernel_fn(ctx->m.dtype, kernel_variant(a), m.n_heads / m.n_kv_heads,
+                                                 m.head_dim),
+                                   dim3(ctx->plan.n_ctas),
                                    dim3(monokernel_threads()), args, ctx->plan.smem, st));
     if (s0 + c < n) {   // the next launch needs this one's last token
       CK(cudaMemcpyAsync(&status, a.sync + SY_STATUS * kSyncStride, 4, cudaMemcpyDeviceToHost, st));
