@@ -30,10 +30,10 @@ size_t monokernel_smem_bytes(int ring_slots, int vbuf_floats, int part_floats);
 int monokernel_threads();
 bool monokernel_profiled();
 // variant bits: 1 = the general instance (lane models, grid-barrier and
-// exact-sum ablations, L2 look-ahead), 2 = the sampler compiled in; G, dh:
-// the attention shape (query heads per KV head, head size), for which the
-// dense greedy instance may be specialised
-const void *monokernel_fn(int dtype, int variant, int G, int dh);
+// exact-sum ablations, L2 look-ahead), 2 = the sampler compiled in; shape:
+// the model's attention shape and its plan's GEMV widths, for which the dense
+// greedy instance may be specialised
+const void *monokernel_fn(int dtype, int variant, const InstShape &shape);
 cudaError_t launch_repack(const uint16_t *src, uint8_t *dst, const RepackJob *jobs, int njobs,
                           cudaStream_t st);
 }  // namespace kie
@@ -620,6 +620,8 @@ extern "C" int kie_weights_bytes(const kie_model_desc *desc, int64_t *out) {
   return KIE_OK;
 }
 
+static InstShape inst_shape(const kie_model_desc &m, const Plan &P);
+
 extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void *stream,
                           kie_ctx **out) {
   if (!out) return KIE_ERR_INVALID;
@@ -676,7 +678,7 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
   }
   Plan &P = ctx->plan;
   for (int variant = 0; variant < 4; ++variant) {   // every kernel instance this model can launch
-    const void *fn = monokernel_fn(m.dtype, variant, m.n_heads / m.n_kv_heads, m.head_dim);
+    const void *fn = monokernel_fn(m.dtype, variant, inst_shape(m, P));
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(P.smem));
     if (e != cudaSuccess) return fail(cuda_fail(nullptr, "cudaFuncSetAttribute", e));
     int per_sm = 0;
@@ -851,6 +853,18 @@ static int steps_per_launch(const kie_ctx *ctx) {
   return int(std::max<int64_t>(n, 1));
 }
 
+// The model's attention shape and its plan's GEMV widths, as a kernel
+// instance may fix them.
+static InstShape inst_shape(const kie_model_desc &m, const Plan &P) {
+  InstShape k{};
+  k.G = m.n_heads / m.n_kv_heads;
+  k.dh = m.head_dim;
+  k.cq = P.shape[ST_QKV].cps;
+  k.cr = P.shape[ST_GU].cps == P.shape[ST_LM].cps ? P.shape[ST_GU].cps : 0;
+  k.cc = P.shape[ST_O].cps == P.shape[ST_D].cps ? P.shape[ST_O].cps : 0;
+  return k;
+}
+
 // The kernel instance for these arguments: the dense one unless a lane
 // model, an ablation switch or the L2 look-ahead needs the general one; the
 // sampler's when a temperature is set.
@@ -902,8 +916,7 @@ static int launch_steps(kie_ctx *ctx, const KernelArgs &a, size_t sync_bytes, in
     if (a.sample_t > 0.f) CK(cudaMemsetAsync(a.psum, 0, size_t(ctx->plan.n_ctas) * 8, st));
     if (s0 == 0) CK(cudaEventRecord(ctx->ev0, st));
     void *args[] = {&b};
-    CK(cudaLaunchCooperativeKernel(monokernel_fn(ctx->m.dtype, kernel_variant(a), m.n_heads / m.n_kv_heads,
-                                                 m.head_dim),
+    CK(cudaLaunchCooperativeKernel(monokernel_fn(ctx->m.dtype, kernel_variant(a), inst_shape(m, ctx->plan)),
                                    dim3(ctx->plan.n_ctas),
                                    dim3(monokernel_threads()), args, ctx->plan.smem, st));
     if (s0 + c < n) {   // the next launch needs this one's last token

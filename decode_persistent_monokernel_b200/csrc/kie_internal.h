@@ -152,6 +152,15 @@ constexpr int kMaxSplit = 32;      // CTAs that share one KV head's positions (o
 constexpr int kMaxTopK = 64;       // largest top-k of the sampler (candidates kept per CTA)
 constexpr int kMaxSampleRows = 2048;  // LM-head rows per CTA that a top-k cut can sort in shared memory
 
+// What a kernel instance may fix at compile time (see monokernel.cu, "kernel
+// instances"): attention shape and GEMV tile widths; a launch compares the
+// model's and its plan's values with an instance's before using it.
+struct InstShape {
+  int32_t G, dh;   // query heads per KV head, head size
+  int32_t cq, cr;  // row-stage widths (cps): q/k/v; gate/up and LM head (0: they differ)
+  int32_t cc;      // column-stage width (cps) of O and down (0: they differ)
+};
+
 struct KernelArgs {
   // model
   int32_t n_layers, d_model, n_heads, n_kv_heads, head_dim, ffn_dim, vocab;

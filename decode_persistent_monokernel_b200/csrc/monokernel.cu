@@ -335,17 +335,24 @@ __device__ bool wait_mbar(const KernelArgs &a, uint64_t *bar, uint32_t parity, u
 //   general (KV_GENERAL): lane models, the grid-barrier and exact-sum
 //           ablations and the L2 look-ahead as runtime switches;
 // each with the sampler (KV_SAMPLE) or without it.
-// The dense greedy instance is also built for fixed attention shapes (query
-// heads per KV head, head size): with them constant the attention's per-head
-// loops fold and its registers shrink (workload 1: 935 vs 891 tok/s).  A
-// shape of 0 reads the model's at run time.
+// The dense greedy instance is also built for fixed shapes: the attention's
+// (query heads per KV head, head size) and the GEMV tile widths of the q/k/v
+// stage, of the other row stages and of the column stages.  With them
+// constant the attention's per-head loops fold and only the GEMV variants in
+// use are compiled, so registers shrink (workload 1, same-GPU A/B: 891 tok/s
+// with runtime shapes, 935 with a constant attention shape, 955 with the
+// widths constant too).  A launch uses such an instance only when every
+// field matches the model and its plan; 0 means "read at run time".
 enum : int { KV_GENERAL = 1, KV_SAMPLE = 2 };
-template <int V, int GS = 0, int DHS = 0>
+template <int V, int GS = 0, int DHS = 0, int CQ = 0, int CR = 0, int CC = 0>
 struct Inst {
   static constexpr bool general = (V & KV_GENERAL) != 0;
   static constexpr bool sample = (V & KV_SAMPLE) != 0;
-  static constexpr int g = GS;    // query heads per KV head, 0 = the model's
-  static constexpr int dh = DHS;  // head size, 0 = the model's
+  static constexpr int g = GS;    // query heads per KV head
+  static constexpr int dh = DHS;  // head size
+  static constexpr int cq = CQ;   // 16-byte chunks per lane and row of a q/k/v tile
+  static constexpr int cr = CR;   // the same for the other row stages (gate/up, LM head)
+  static constexpr int cc = CC;   // output groups per thread of the column stages (O, down)
 };
 
 // ------------------------------------------------------------------ weight producer
@@ -760,9 +767,9 @@ __device__ __forceinline__ int sample_full(const SampleArgs g, const Smem s, int
 }
 
 // ------------------------------------------------------------------ consumer
-template <typename T, int V, int GS, int DHS>
+template <typename T, int V, int GS, int DHS, int CQ, int CR, int CC>
 struct Consumer {
-  using I = Inst<V, GS, DHS>;
+  using I = Inst<V, GS, DHS, CQ, CR, CC>;
   const KernelArgs &a;
   Smem s;
   const int tid, warp, lane, cta;
@@ -1037,7 +1044,8 @@ struct Consumer {
   __device__ void gemv_rows(int k, const float *vin, OutF &&out) {
     KP_BEGIN(t_gemv);
     KT(TE_STAGE_BEGIN, k);
-    switch (a.shape[k].cps) {
+    const int fixed = k == ST_QKV ? I::cq : I::cr;   // call sites pass a constant k
+    switch (fixed ? fixed : a.shape[k].cps) {
       case 4: gemv_rows_c<4>(k, vin, out); break;
       case 2: gemv_rows_c<2>(k, vin, out); break;
       default: gemv_rows_c<1>(k, vin, out); break;
@@ -1362,7 +1370,7 @@ struct Consumer {
 
   // acc: the accumulator (acc_o or acc_d); parity: the layer's half of it
   __device__ void gemv_cols(int k, const float *svals, float *acc, uint32_t parity) {
-    if (a.shape[k].cps == 1) gemv_cols_impl<1>(k, svals, acc, parity);
+    if ((I::cc ? I::cc : a.shape[k].cps) == 1) gemv_cols_impl<1>(k, svals, acc, parity);
     else gemv_cols_impl<2>(k, svals, acc, parity);
   }
 
@@ -1670,7 +1678,7 @@ struct Consumer {
   }
 };
 
-template <typename T, int V, int GS, int DHS>
+template <typename T, int V, int GS, int DHS, int CQ, int CR, int CC>
 __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int tid = threadIdx.x;
@@ -1717,7 +1725,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
     }
     __syncwarp();
   } else {
-    Consumer<T, V, GS, DHS> c(a, s, tid, cta);
+    Consumer<T, V, GS, DHS, CQ, CR, CC> c(a, s, tid, cta);
     c.run();
     // a CTA that gave up makes every other CTA (and its own producer) leave
     if (tid == 0 && c.aborted()) atomicExch(sync_at(a, SY_ABORT), 1u);
@@ -1806,21 +1814,26 @@ bool monokernel_profiled() {
 #endif
 }
 
-// variant: KV_GENERAL and KV_SAMPLE bits (see "kernel instances"); the dense
-// greedy variant comes shape-specialised for (G, dh) = (2, 128) and (4, 128)
+// variant: KV_GENERAL and KV_SAMPLE bits (see "kernel instances").  The
+// dense greedy variant comes specialised for the shapes of the 2.3B-class
+// models (G 2, dh 128, widths q/k/v 4, rows 1, columns 1) and of the
+// 8B-class one (G 4, dh 128, widths 2, 1, 2); any other shape runs the
+// runtime-shape instance.
 template <typename T>
-static const void *pick(int variant, int G, int dh) {
-  if (variant == 0 && dh == 128 && G == 2) return reinterpret_cast<const void *>(&monokernel<T, 0, 2, 128>);
-  if (variant == 0 && dh == 128 && G == 4) return reinterpret_cast<const void *>(&monokernel<T, 0, 4, 128>);
+static const void *pick(int variant, const InstShape &k) {
+  if (variant == 0 && k.G == 2 && k.dh == 128 && k.cq == 4 && k.cr == 1 && k.cc == 1)
+    return reinterpret_cast<const void *>(&monokernel<T, 0, 2, 128, 4, 1, 1>);
+  if (variant == 0 && k.G == 4 && k.dh == 128 && k.cq == 2 && k.cr == 1 && k.cc == 2)
+    return reinterpret_cast<const void *>(&monokernel<T, 0, 4, 128, 2, 1, 2>);
   switch (variant & 3) {
-    case 0: return reinterpret_cast<const void *>(&monokernel<T, 0, 0, 0>);
-    case 1: return reinterpret_cast<const void *>(&monokernel<T, 1, 0, 0>);
-    case 2: return reinterpret_cast<const void *>(&monokernel<T, 2, 0, 0>);
-    default: return reinterpret_cast<const void *>(&monokernel<T, 3, 0, 0>);
+    case 0: return reinterpret_cast<const void *>(&monokernel<T, 0, 0, 0, 0, 0, 0>);
+    case 1: return reinterpret_cast<const void *>(&monokernel<T, 1, 0, 0, 0, 0, 0>);
+    case 2: return reinterpret_cast<const void *>(&monokernel<T, 2, 0, 0, 0, 0, 0>);
+    default: return reinterpret_cast<const void *>(&monokernel<T, 3, 0, 0, 0, 0, 0>);
   }
 }
-const void *monokernel_fn(int dtype, int variant, int G, int dh) {
-  return dtype == 0 ? pick<__half>(variant, G, dh) : pick<__nv_bfloat16>(variant, G, dh);
+const void *monokernel_fn(int dtype, int variant, const InstShape &shape) {
+  return dtype == 0 ? pick<__half>(variant, shape) : pick<__nv_bfloat16>(variant, shape);
 }
 
 cudaError_t launch_repack(const uint16_t *src, uint8_t *dst, const RepackJob *jobs, int njobs,
