@@ -30,7 +30,8 @@ size_t monokernel_smem_bytes(int ring_slots, int vbuf_floats, int part_floats);
 int monokernel_threads();
 bool monokernel_profiled();
 // variant bits: 1 = the general instance (lane models, grid-barrier and
-// exact-sum ablations, L2 look-ahead), 2 = the sampler compiled in; shape:
+// exact-sum ablations, L2 look-ahead), 2 = the sampler compiled in, 4 = the
+// lanes instance (lane models without ablations); shape:
 // the model's attention shape and its plan's GEMV widths, for which the dense
 // greedy instance may be specialised
 const void *monokernel_fn(int dtype, int variant, const InstShape &shape);
@@ -677,7 +678,7 @@ extern "C" int kie_create(const kie_model_desc *desc, const void *weights, void 
     return fail(KIE_ERR_INVALID);
   }
   Plan &P = ctx->plan;
-  for (int variant = 0; variant < 4; ++variant) {   // every kernel instance this model can launch
+  for (int variant = 0; variant < 5; ++variant) {   // every kernel instance this model can launch
     const void *fn = monokernel_fn(m.dtype, variant, inst_shape(m, P));
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(P.smem));
     if (e != cudaSuccess) return fail(cuda_fail(nullptr, "cudaFuncSetAttribute", e));
@@ -862,15 +863,20 @@ static InstShape inst_shape(const kie_model_desc &m, const Plan &P) {
   k.cq = P.shape[ST_QKV].cps;
   k.cr = P.shape[ST_GU].cps == P.shape[ST_LM].cps ? P.shape[ST_GU].cps : 0;
   k.cc = P.shape[ST_O].cps == P.shape[ST_D].cps ? P.shape[ST_O].cps : 0;
+  k.cm = m.n_lanes > 1 ? P.shape[ST_MIX].cps : 0;
   return k;
 }
 
-// The kernel instance for these arguments: the dense one unless a lane
-// model, an ablation switch or the L2 look-ahead needs the general one; the
-// sampler's when a temperature is set.
+// The kernel instance for these arguments: the general one when an
+// ablation switch or the L2 look-ahead is on, or a lane model samples; the
+// lanes one for other lane-model calls; else the dense one; with the
+// sampler compiled in when a temperature is set.
 static int kernel_variant(const KernelArgs &a) {
-  const bool general = a.n_lanes > 1 || a.grid_sync || a.det_sum || a.l2pf_tiles > 0;
-  return (general ? 1 : 0) | (a.sample_t > 0.f ? 2 : 0);
+  const bool ablations = a.grid_sync || a.det_sum || a.l2pf_tiles > 0;
+  const bool lanes = a.n_lanes > 1, sample = a.sample_t > 0.f;
+  if (ablations || (lanes && sample)) return 1 | (sample ? 2 : 0);
+  if (lanes) return 4;
+  return sample ? 2 : 0;
 }
 
 // Runs the n steps described by `a` (forced tokens, output tokens, argmax

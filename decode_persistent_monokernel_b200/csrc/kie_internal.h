@@ -159,6 +159,7 @@ struct InstShape {
   int32_t G, dh;   // query heads per KV head, head size
   int32_t cq, cr;  // row-stage widths (cps): q/k/v; gate/up and LM head (0: they differ)
   int32_t cc;      // column-stage width (cps) of O and down (0: they differ)
+  int32_t cm;      // lane models: row-stage width of the lane mix (0: dense)
 };
 
 struct KernelArgs {

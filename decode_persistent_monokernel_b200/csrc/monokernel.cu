@@ -328,31 +328,35 @@ __device__ bool wait_mbar(const KernelArgs &a, uint64_t *bar, uint32_t parity, u
 // and code layout.  Measured on workload 1 (2.3B-class, 128 steps, three
 // repeats on one GPU): with the lane-model and ablation branches compiled out
 // the dense greedy loop ran 3.0 % faster (892 vs 866 tok/s), and it ran 1.7 %
-// faster without the sampler compiled in.  So a launch picks one of four
+// faster without the sampler compiled in.  So a launch picks one of these
 // instances:
-//   dense   (V without KV_GENERAL): one lane, dependency counters, fp32 atomic
-//           sums, no L2 look-ahead -- the decode every dense model runs;
+//   dense   (V 0): one lane, dependency counters, fp32 atomic sums, no L2
+//           look-ahead -- the decode every dense model runs;
+//   lanes   (KV_LANES): the same for lane models (delayed cross-lane mix);
 //   general (KV_GENERAL): lane models, the grid-barrier and exact-sum
 //           ablations and the L2 look-ahead as runtime switches;
-// each with the sampler (KV_SAMPLE) or without it.
+// dense and general with the sampler (KV_SAMPLE) or without it.
 // The dense greedy instance is also built for fixed shapes: the attention's
 // (query heads per KV head, head size) and the GEMV tile widths of the q/k/v
 // stage, of the other row stages and of the column stages.  With them
 // constant the attention's per-head loops fold and only the GEMV variants in
 // use are compiled, so registers shrink (workload 1, same-GPU A/B: 891 tok/s
 // with runtime shapes, 935 with a constant attention shape, 955 with the
-// widths constant too).  A launch uses such an instance only when every
-// field matches the model and its plan; 0 means "read at run time".
-enum : int { KV_GENERAL = 1, KV_SAMPLE = 2 };
-template <int V, int GS = 0, int DHS = 0, int CQ = 0, int CR = 0, int CC = 0>
+// widths constant too).  The lanes instance exists only in a fixed shape.  A
+// launch uses a fixed-shape instance only when every field matches the model
+// and its plan; 0 means "read at run time".
+enum : int { KV_GENERAL = 1, KV_SAMPLE = 2, KV_LANES = 4 };
+template <int V, int GS = 0, int DHS = 0, int CQ = 0, int CR = 0, int CC = 0, int CM = 0>
 struct Inst {
-  static constexpr bool general = (V & KV_GENERAL) != 0;
+  static constexpr bool ablations = (V & KV_GENERAL) != 0;   // grid barrier, exact sums, L2 look-ahead
+  static constexpr bool lanes = (V & (KV_GENERAL | KV_LANES)) != 0;
   static constexpr bool sample = (V & KV_SAMPLE) != 0;
   static constexpr int g = GS;    // query heads per KV head
   static constexpr int dh = DHS;  // head size
   static constexpr int cq = CQ;   // 16-byte chunks per lane and row of a q/k/v tile
   static constexpr int cr = CR;   // the same for the other row stages (gate/up, LM head)
   static constexpr int cc = CC;   // output groups per thread of the column stages (O, down)
+  static constexpr int cm = CM;   // the row width of the lane-mix stage
 };
 
 // ------------------------------------------------------------------ weight producer
@@ -436,7 +440,7 @@ struct Producer {
           // the slot's previous tile (T - NS) was released by every consumer warp
           uint32_t nthis = 0;
           const uint8_t *c0 = cur;
-          const bool pf = I::general && a.l2pf_tiles > 0;
+          const bool pf = I::ablations && a.l2pf_tiles > 0;
           if (!wait_mbar(a, &s.empty[slot], phase ^ 1u, DE_TIMEOUT_EMPTY, [&](long long el) {
                 if (pf) l2_lookahead(el, nthis, c0);
               }))
@@ -460,7 +464,7 @@ struct Producer {
 
   __device__ void run() {
     base = a.wstream + a.cta_stream_off[cta];
-    const bool lanes = I::general && a.n_lanes > 1;
+    const bool lanes = I::lanes && a.n_lanes > 1;
     // bytes of one step's stream: every layer's stages, then the final lane
     // mix and the LM head (when the step computes logits)
     const StageCta *sc = s.misc->sc;
@@ -767,9 +771,9 @@ __device__ __forceinline__ int sample_full(const SampleArgs g, const Smem s, int
 }
 
 // ------------------------------------------------------------------ consumer
-template <typename T, int V, int GS, int DHS, int CQ, int CR, int CC>
+template <typename T, int V, int GS, int DHS, int CQ, int CR, int CC, int CM>
 struct Consumer {
-  using I = Inst<V, GS, DHS, CQ, CR, CC>;
+  using I = Inst<V, GS, DHS, CQ, CR, CC, CM>;
   const KernelArgs &a;
   Smem s;
   const int tid, warp, lane, cta;
@@ -806,7 +810,7 @@ struct Consumer {
 #ifdef KIE_PROFILE
       const long long t0 = clock64();
 #endif
-      if (I::general && a.grid_sync) {
+      if (I::ablations && a.grid_sync) {
         slot = SY_GRID;
         target = nsig * a.n_ctas;
       }
@@ -829,7 +833,7 @@ struct Consumer {
     cbar();
     KT(TE_SIGNAL_END, 0);
     ++nsig;
-    if (tid == 0) red_release_add(sync_at(a, (I::general && a.grid_sync) ? int(SY_GRID) : slot), 1u);
+    if (tid == 0) red_release_add(sync_at(a, (I::ablations && a.grid_sync) ? int(SY_GRID) : slot), 1u);
     KP_END(t_sig, PF_SIGNAL);
   }
 
@@ -845,14 +849,14 @@ struct Consumer {
   // sums (stored 2 d floats further on).
   __device__ float4 acc4(const float *base, uint32_t parity, int j) const {
     const float4 h = __ldcg(vec4(base, parity) + j);
-    if (!(I::general && a.det_sum)) return h;
+    if (!(I::ablations && a.det_sum)) return h;
     const float4 l = __ldcg(vec4(base + 2 * size_t(a.d_model), parity) + j);
     return make_float4(h.x + l.x, h.y + l.y, h.z + l.z, h.w + l.w);
   }
   // Adds outputs e .. e+3 into a layer accumulator of the given parity.
   __device__ __forceinline__ void acc_add4(float *base, uint32_t parity, int e, float4 v) const {
     float *p = base + size_t(parity & 1u) * a.d_model + e;
-    if (!(I::general && a.det_sum)) {
+    if (!(I::ablations && a.det_sum)) {
       red_add_v4(p, v);
       return;
     }
@@ -876,7 +880,7 @@ struct Consumer {
       const uint32_t q = gl - 1;
       v = add4(add4(__ldcg(vec4(a.xres, q) + j), acc4(a.acc_o, q, j)), acc4(a.acc_d, q, j));
     }
-    if (I::general && a.n_lanes > 1 && l >= a.lane_delay)
+    if (I::lanes && a.n_lanes > 1 && l >= a.lane_delay)
       v = add4(v, __ldcg(reinterpret_cast<const float4 *>(
                              a.dsum + size_t((l - a.lane_delay) % a.lane_delay) * a.d_model) + j));
     return v;
@@ -1044,7 +1048,8 @@ struct Consumer {
   __device__ void gemv_rows(int k, const float *vin, OutF &&out) {
     KP_BEGIN(t_gemv);
     KT(TE_STAGE_BEGIN, k);
-    const int fixed = k == ST_QKV ? I::cq : I::cr;   // call sites pass a constant k
+    // call sites pass a constant k
+    const int fixed = k == ST_QKV ? I::cq : k == ST_MIX ? I::cm : I::cr;
     switch (fixed ? fixed : a.shape[k].cps) {
       case 4: gemv_rows_c<4>(k, vin, out); break;
       case 2: gemv_rows_c<2>(k, vin, out); break;
@@ -1288,7 +1293,7 @@ struct Consumer {
     // each CTA of the group waits for and loads the words it needs into
     // shared memory and merges them (log-sum-exp) into the group's output
     KT(TE_ATTN, 2);
-    if (I::general && a.grid_sync) {   // the ablation keeps a grid-wide barrier here
+    if (I::ablations && a.grid_sync) {   // the ablation keeps a grid-wide barrier here
       signal(SY_GRID);
       if (!gate(SY_GRID, 0, 0x28, 5)) return;
     }
@@ -1517,7 +1522,7 @@ struct Consumer {
 
   __device__ void run_body() {
     const int L = a.n_layers, d = a.d_model;
-    const bool lanes = I::general && a.n_lanes > 1;
+    const bool lanes = I::lanes && a.n_lanes > 1;
     const int delta = a.lane_delay;
     const uint32_t nc = a.n_ctas;
     const int own_lo = int(int64_t(d) * cta / a.n_ctas);  // residual rows this CTA owns
@@ -1563,7 +1568,7 @@ struct Consumer {
           gemv_rows(ST_QKV, s.vbuf, to_qkv);
         }
         if (aborted()) goto done;
-        if (I::general && a.grid_sync) signal(SY_GRID);   // the ablation keeps a grid-wide barrier here
+        if (I::ablations && a.grid_sync) signal(SY_GRID);   // the ablation keeps a grid-wide barrier here
         // ---------------- delayed cross-lane sum of the previous layer
         if (lanes && l >= 1) {
           stage_input([=](int j) { return add4(acc4(a.acc_o, prev, j), acc4(a.acc_d, prev, j)); },
@@ -1575,7 +1580,7 @@ struct Consumer {
           if (aborted()) goto done;
         }
         // ---------------- attention of the group, merged in every group CTA
-        if (I::general && a.grid_sync && !gate(SY_GRID, 0, 0x20, 4)) goto done;
+        if (I::ablations && a.grid_sync && !gate(SY_GRID, 0, 0x20, 4)) goto done;
         attention();
         if (aborted()) goto done;
         // ---------------- O projection over the group's attention outputs
@@ -1590,7 +1595,7 @@ struct Consumer {
           for (int r = own_lo + tid; r < own_hi; r += kNC) {
             a.acc_o[size_t(prev) * d + r] = 0.f;
             a.acc_d[size_t(prev) * d + r] = 0.f;
-            if (I::general && a.det_sum) {   // the lo sums, 2 d further on
+            if (I::ablations && a.det_sum) {   // the lo sums, 2 d further on
               a.acc_o[size_t(2 + prev) * d + r] = 0.f;
               a.acc_d[size_t(2 + prev) * d + r] = 0.f;
             }
@@ -1678,7 +1683,7 @@ struct Consumer {
   }
 };
 
-template <typename T, int V, int GS, int DHS, int CQ, int CR, int CC>
+template <typename T, int V, int GS, int DHS, int CQ, int CR, int CC, int CM>
 __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int tid = threadIdx.x;
@@ -1725,7 +1730,7 @@ __global__ void __launch_bounds__(kThreads, 1) monokernel(const KernelArgs a) {
     }
     __syncwarp();
   } else {
-    Consumer<T, V, GS, DHS, CQ, CR, CC> c(a, s, tid, cta);
+    Consumer<T, V, GS, DHS, CQ, CR, CC, CM> c(a, s, tid, cta);
     c.run();
     // a CTA that gave up makes every other CTA (and its own producer) leave
     if (tid == 0 && c.aborted()) atomicExch(sync_at(a, SY_ABORT), 1u);
@@ -1814,22 +1819,29 @@ bool monokernel_profiled() {
 #endif
 }
 
-// variant: KV_GENERAL and KV_SAMPLE bits (see "kernel instances").  The
-// dense greedy variant comes specialised for the shapes of the 2.3B-class
-// models (G 2, dh 128, widths q/k/v 4, rows 1, columns 1) and of the
-// 8B-class one (G 4, dh 128, widths 2, 1, 2); any other shape runs the
-// runtime-shape instance.
+// variant: KV_GENERAL, KV_SAMPLE and KV_LANES bits (see "kernel instances").
+// The dense greedy variant comes specialised for the shapes of the
+// 2.3B-class models (G 2, dh 128, widths q/k/v 4, rows 1, columns 1) and of
+// the 8B-class one (G 4, dh 128, widths 2, 1, 2), other shapes running the
+// runtime-shape instance; the lanes variant exists for the lane-structured
+// model's shape (G 1, dh 128, widths 2, 1, 1, lane mix 4), other lane
+// models running the general instance.
 template <typename T>
 static const void *pick(int variant, const InstShape &k) {
   if (variant == 0 && k.G == 2 && k.dh == 128 && k.cq == 4 && k.cr == 1 && k.cc == 1)
-    return reinterpret_cast<const void *>(&monokernel<T, 0, 2, 128, 4, 1, 1>);
+    return reinterpret_cast<const void *>(&monokernel<T, 0, 2, 128, 4, 1, 1, 0>);
   if (variant == 0 && k.G == 4 && k.dh == 128 && k.cq == 2 && k.cr == 1 && k.cc == 2)
-    return reinterpret_cast<const void *>(&monokernel<T, 0, 4, 128, 2, 1, 2>);
+    return reinterpret_cast<const void *>(&monokernel<T, 0, 4, 128, 2, 1, 2, 0>);
+  if (variant == KV_LANES) {
+    if (k.G == 1 && k.dh == 128 && k.cq == 2 && k.cr == 1 && k.cc == 1 && k.cm == 4)
+      return reinterpret_cast<const void *>(&monokernel<T, KV_LANES, 1, 128, 2, 1, 1, 4>);
+    variant = KV_GENERAL;
+  }
   switch (variant & 3) {
-    case 0: return reinterpret_cast<const void *>(&monokernel<T, 0, 0, 0, 0, 0, 0>);
-    case 1: return reinterpret_cast<const void *>(&monokernel<T, 1, 0, 0, 0, 0, 0>);
-    case 2: return reinterpret_cast<const void *>(&monokernel<T, 2, 0, 0, 0, 0, 0>);
-    default: return reinterpret_cast<const void *>(&monokernel<T, 3, 0, 0, 0, 0, 0>);
+    case 0: return reinterpret_cast<const void *>(&monokernel<T, 0, 0, 0, 0, 0, 0, 0>);
+    case 1: return reinterpret_cast<const void *>(&monokernel<T, 1, 0, 0, 0, 0, 0, 0>);
+    case 2: return reinterpret_cast<const void *>(&monokernel<T, 2, 0, 0, 0, 0, 0, 0>);
+    default: return reinterpret_cast<const void *>(&monokernel<T, 3, 0, 0, 0, 0, 0, 0>);
   }
 }
 const void *monokernel_fn(int dtype, int variant, const InstShape &shape) {
