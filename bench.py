@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--sum", choices=["fp32_atomic", "exact"], default=None,
                     help="how the O / down projections are added over SMs (default: the "
                          "library's default mode)")
+    ap.add_argument("--sample", metavar="T,K,P", default=None,
+                    help="decode by sampling (kie_decode_sample) with temperature T, top-k K "
+                         "and top-p P, one seeded uniform per step, instead of greedy")
     ap.add_argument("--profile", action="store_true",
                     help="run the profiling build (libkie_prof.so) and report where each "
                          "SM's time goes; its timings are not the benchmark value")
@@ -267,13 +270,25 @@ def cpu_baseline_obj(rate, n, el, cores, prefill_s, P):
             "prefill_s": prefill_s, "cpu": host_cpu_model(), "host_cpus": os.cpu_count()}
 
 
-def run_config(w, P, K, world, sync, weight_bytes_per_step):
+def run_config(w, P, K, world, sync, weight_bytes_per_step, sample=None):
     """The `config` object of the bench line, the same for both arms."""
-    return {"workload": w.name, "prompt": P, "decode_steps": K, "batch": 1,
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-            "sync": sync,
-            "l2": "inputs larger than L2: %.2f GB of weights streamed per step"
-                  % (weight_bytes_per_step / 1e9)}
+    cfg = {"workload": w.name, "prompt": P, "decode_steps": K, "batch": 1,
+           "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+           "sync": sync,
+           "l2": "inputs larger than L2: %.2f GB of weights streamed per step"
+                 % (weight_bytes_per_step / 1e9)}
+    if sample is not None:
+        cfg["sampling"] = {"temperature": sample[0], "top_k": sample[1], "top_p": sample[2],
+                           "uniforms": "seeded, one per step"}
+    return cfg
+
+
+def parse_sample(text):
+    """(temperature, top_k, top_p) from "T,K,P", or None."""
+    if not text:
+        return None
+    t, k, p = text.split(",")
+    return float(t), int(k), float(p)
 
 
 def reduce_max_over_ranks(values, world, device):
@@ -305,6 +320,7 @@ def main():
     w = synth.WORKLOADS[args.workload]
     m = w.model
     P, K, W = w.prompt_len, args.steps, max(3, args.warmup)
+    smp = parse_sample(args.sample)
 
     if args.impl == "reference":
         # the oracle as it stands, on this host's cores, rank 0 only
@@ -353,9 +369,19 @@ def main():
     torch.cuda.empty_cache()
     st = dec.kie_get_stats()
 
+    # greedy, or sampling with uniforms drawn before any timed region
+    urng = np.random.default_rng(2024)
+    u_warm = urng.random(W).astype(np.float32)
+    u_timed = urng.random(K).astype(np.float32)
+
+    def decode(n, u):
+        if smp is None:
+            return dec.kie_decode(n)
+        return dec.kie_decode_sample(n, smp[0], smp[1], smp[2], u)
+
     # warm-up: prompt + W steps, untimed
     dec.kie_prefill(prompt)
-    dec.kie_decode(W)
+    decode(W, u_warm)
     # timed: K steps from the workload's own starting point (position P)
     dec.kie_prefill(prompt)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -363,7 +389,7 @@ def main():
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         ev0.record(stream)
-        toks = dec.kie_decode(K)
+        toks = decode(K, u_timed)
         ev1.record(stream)
         torch.cuda.synchronize()
     barrier()
@@ -386,7 +412,7 @@ def main():
     barrier()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    toks2 = dec.kie_decode(K)
+    toks2 = decode(K, u_timed)
     e2e_s = time.perf_counter() - t0
     barrier()
     # With fp32 atomic O/down sums the last bits of the logits vary between
@@ -412,7 +438,7 @@ def main():
         "warmup": W, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 (fp16 weights/KV)" if m.dtype == "f16"
         else "f32 (bf16 weights/KV)", "data": "synthetic (seeded weights and prompt)",
-        "config": run_config(w, P, K, world, args.sync, st.weight_bytes_per_step),
+        "config": run_config(w, P, K, world, args.sync, st.weight_bytes_per_step, smp),
         "us_per_token": 1e3 * ms / K,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
@@ -426,8 +452,9 @@ def main():
         "sum_mode": args.sum or "library default",
         "e2e": {"value": job_tokens_per_s(world, K, e2e_s * 1e3), "unit": "tokens/s",
                 "what": "decode tokens / wall time of one kie_decode(K) call into a host "
-                        "array (launch, K steps, token and status copies, synchronisation)",
-                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": (4 * K + 4) / K,
+                        "array (launch, K steps, token and status copies, synchronisation)"
+                        + ("; kie_decode_sample with the K uniforms copied in" if smp else ""),
+                "h2d_bytes_per_step": 4 if smp else 0, "d2h_bytes_per_step": (4 * K + 4) / K,
                 "prefill_wall_s": prefill_s, "prefill_tokens": P},
         "kernel": {"ctas": st.n_ctas, "threads": st.threads_per_cta, "ring_slots": st.ring_slots,
                    "smem_bytes": st.smem_bytes},

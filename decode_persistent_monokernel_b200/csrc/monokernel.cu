@@ -1820,7 +1820,7 @@ bool monokernel_profiled() {
 }
 
 // variant: KV_GENERAL, KV_SAMPLE and KV_LANES bits (see "kernel instances").
-// The dense greedy variant comes specialised for the shapes of the
+// The dense variants, greedy and sampling, come specialised for the shapes of the
 // 2.3B-class models (G 2, dh 128, widths q/k/v 4, rows 1, columns 1) and of
 // the 8B-class one (G 4, dh 128, widths 2, 1, 2), other shapes running the
 // runtime-shape instance; the lanes variant exists for the lane-structured
@@ -1828,10 +1828,16 @@ bool monokernel_profiled() {
 // models running the general instance.
 template <typename T>
 static const void *pick(int variant, const InstShape &k) {
-  if (variant == 0 && k.G == 2 && k.dh == 128 && k.cq == 4 && k.cr == 1 && k.cc == 1)
-    return reinterpret_cast<const void *>(&monokernel<T, 0, 2, 128, 4, 1, 1, 0>);
-  if (variant == 0 && k.G == 4 && k.dh == 128 && k.cq == 2 && k.cr == 1 && k.cc == 2)
-    return reinterpret_cast<const void *>(&monokernel<T, 0, 4, 128, 2, 1, 2, 0>);
+  if (k.G == 2 && k.dh == 128 && k.cq == 4 && k.cr == 1 && k.cc == 1) {
+    if (variant == 0) return reinterpret_cast<const void *>(&monokernel<T, 0, 2, 128, 4, 1, 1, 0>);
+    if (variant == KV_SAMPLE)
+      return reinterpret_cast<const void *>(&monokernel<T, KV_SAMPLE, 2, 128, 4, 1, 1, 0>);
+  }
+  if (k.G == 4 && k.dh == 128 && k.cq == 2 && k.cr == 1 && k.cc == 2) {
+    if (variant == 0) return reinterpret_cast<const void *>(&monokernel<T, 0, 4, 128, 2, 1, 2, 0>);
+    if (variant == KV_SAMPLE)
+      return reinterpret_cast<const void *>(&monokernel<T, KV_SAMPLE, 4, 128, 2, 1, 2, 0>);
+  }
   if (variant == KV_LANES) {
     if (k.G == 1 && k.dh == 128 && k.cq == 2 && k.cr == 1 && k.cc == 1 && k.cm == 4)
       return reinterpret_cast<const void *>(&monokernel<T, KV_LANES, 1, 128, 2, 1, 1, 4>);
