@@ -326,6 +326,16 @@ int main() {
     const char *why = build_plan(m, 148, 232448, P);
     printf("%s: %s slots %d smem %zu stream %.3f GB wbytes %lld\n", nm, why ? why : "ok", P.ring_slots, P.smem,
            P.stream_bytes / 1e9, (long long)P.weight_bytes_per_step);
+    // the named workloads run on shape-specialised kernel instances: their
+    // model and plan must match an instance's key (else they would silently
+    // fall back to the slower runtime-shape instance)
+    const InstShape k = inst_shape(m, P), none{};
+    if (m.n_lanes == 1) {
+      REQ(monokernel_fn(m.dtype, 0, k) != monokernel_fn(m.dtype, 0, none), "%s: no shape-specialised dense instance", nm);
+      REQ(monokernel_fn(m.dtype, 2, k) != monokernel_fn(m.dtype, 2, none), "%s: no shape-specialised sampling instance", nm);
+    } else {
+      REQ(monokernel_fn(m.dtype, 4, k) != monokernel_fn(m.dtype, 1, k), "%s: no lanes instance for its shape", nm);
+    }
   }
   // row lengths: K / 128 lanes share a row, so only 128 x a power of two
   for (int K = 128; K <= 4096; K += 128) {

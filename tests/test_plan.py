@@ -6,8 +6,9 @@ producer's tile walk and the consumers' lane and thread mappings on the
 streamed bytes in double precision: every weight element is copied exactly
 once, every (row, column chunk) is read exactly once, and one layer's
 q/k/v, gate/up, O, down and lane-mix products equal the canonical
-matrix-vector products.  The kernel files are compiled to PTX only (nothing
-runs on a GPU).
+matrix-vector products; and the named workloads' models and plans match the
+keys of the shape-specialised kernel instances.  The kernel files are compiled
+to PTX only (nothing runs on a GPU).
 """
 import os
 import subprocess
