@@ -356,6 +356,21 @@ int main() {
     kie_model_desc m3{2, 384, 6, 3, 64, 768, 4096, 1e-5f, 1e4f, 0, 3, 2, 64};
     REQ(build_plan(m3, 148, 232448, P) != nullptr, "3-lane d_model 384 accepted");
   }
+  {
+    // which kernel instance each kind of call launches: the dense one unless an
+    // ablation switch, the L2 look-ahead or a lane model needs another; the
+    // sampler's when a temperature is set (lane models sample on the general one)
+    struct Case { int lanes, grid, det, l2pf; float t; int want; };
+    const Case cases[] = {{1, 0, 0, 0, 0.f, 0}, {1, 0, 0, 0, 0.7f, 2}, {8, 0, 0, 0, 0.f, 4},
+                          {8, 0, 0, 0, 0.7f, 3}, {1, 1, 0, 0, 0.f, 1}, {1, 0, 1, 0, 0.f, 1},
+                          {1, 0, 0, 4, 0.f, 1}, {1, 0, 1, 0, 0.7f, 3}, {8, 1, 0, 0, 0.f, 1}};
+    for (const Case &c : cases) {
+      KernelArgs a{};
+      a.n_lanes = c.lanes; a.grid_sync = c.grid; a.det_sum = c.det; a.l2pf_tiles = c.l2pf; a.sample_t = c.t;
+      REQ(kernel_variant(a) == c.want, "kernel_variant(lanes %d grid %d det %d l2pf %d T %g) = %d, want %d",
+          c.lanes, c.grid, c.det, c.l2pf, c.t, kernel_variant(a), c.want);
+    }
+  }
   printf(fails ? "FAILED (%d)\n" : "ALL OK\n", fails);
   return fails != 0;
 }
