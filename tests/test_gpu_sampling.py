@@ -173,6 +173,25 @@ def test_full_size_sampling(mode, dense_2b):
     dec.kie_destroy()
 
 
+def test_8b_class_shapes_sampling():
+    """The 8B-class workload's shapes (bf16, 4 query heads per KV head,
+    V 128,256: 867 LM-head rows per SM) on two layers, 24 sampled steps
+    after a 64-token prompt, in both sampling modes."""
+    w = synth.WORKLOADS[4]
+    m = w.model.replace(n_layers=2)
+    bits = synth.generate_weights(m, w.weight_seed)
+    prompt = synth.prompt(w)[:64]
+    N = 24
+    dec = make_decoder(m, bits, len(prompt) + N + 4)
+    for mode, seed in (("top_k_top_p", 41), ("full_vocab", 42)):
+        T, k, p = MODES[mode]
+        u = np.random.default_rng(seed).random(N).astype(np.float32)
+        dec.kie_prefill(prompt)
+        toks, z = _sample_run(dec, N, m.vocab, T, k, p, u)
+        check_sampled(toks, z, u, T, k, p, f"8b-2L {mode}")
+    dec.kie_destroy()
+
+
 @pytest.fixture(scope="module")
 def dense_2b():
     w = synth.WORKLOADS[1]
