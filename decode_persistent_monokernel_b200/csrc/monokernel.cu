@@ -509,9 +509,10 @@ struct Producer {
 
 // ---- logit keys: (order-preserving bits of the value) << 32 | (~row), so
 // that a larger key is a larger logit, and among equal logits the lower
-// row; every finite or infinite logit's key is above 0
+// row; every finite or infinite logit's key is above 0.  -0 and +0 are
+// equal logits, so both take +0's bits (else +0 would outrank -0).
 __device__ __forceinline__ unsigned long long logit_key(float v, int row) {
-  const uint32_t fb = __float_as_uint(v);
+  const uint32_t fb = __float_as_uint(v == 0.f ? 0.f : v);
   const uint32_t ord = (fb & 0x80000000u) ? ~fb : (fb | 0x80000000u);
   return (static_cast<unsigned long long>(ord) << 32) | (0xffffffffu - uint32_t(row));
 }

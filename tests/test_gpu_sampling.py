@@ -192,6 +192,30 @@ def test_8b_class_shapes_sampling():
     dec.kie_destroy()
 
 
+def test_all_logits_equal():
+    """A zeroed LM head makes every logit a signed zero (+0 or -0 by the sign of
+    the last products): all tie.  Greedy must take token 0 at every step (the
+    lowest index of the largest value, g11), and top-k 5 must keep ids 0..4,
+    each drawn with probability 1/5: the uniform u picks id floor(5 u)."""
+    w = synth.WORKLOADS[0]
+    m = w.model
+    bits = synth.generate_weights(m, w.weight_seed).copy()
+    lm = {t.name: t for t in synth.tensor_table(m)}["lm_head"]
+    bits[lm.offset:lm.offset + lm.numel] = 0
+    prompt = synth.prompt(w)
+    N = 16
+    dec = make_decoder(m, bits, len(prompt) + 2 * N + 8)
+    assert dec.kie_prefill(prompt) == 0
+    assert np.all(dec.kie_decode(N) == 0)
+    u = np.random.default_rng(3).random(N).astype(np.float32)
+    dec.kie_prefill(prompt)
+    toks, z = _sample_run(dec, N, m.vocab, 1.0, 5, 1.0, u)
+    assert np.all(z == 0.0)
+    check_sampled(toks, z, u, 1.0, 5, 1.0, "all logits equal", max_near=0)
+    assert np.array_equal(toks, np.floor(5 * u.astype(np.float64)).astype(np.int32))
+    dec.kie_destroy()
+
+
 @pytest.fixture(scope="module")
 def dense_2b():
     w = synth.WORKLOADS[1]
