@@ -130,3 +130,20 @@ def test_algorithmic_bytes_agree_between_bench_and_the_counter_case():
         # the counter case times the launch after a warm-up launch of `steps`
         got = bench.workload_bytes(m, P + steps, steps, synth.streamed_weight_bytes(m), kvpp)
         assert got == profile_case.algorithmic_bytes(m, P, steps), wid
+
+
+def test_sampling_option_reaches_the_config():
+    """`--sample T,K,P` is parsed into (temperature, top-k, top-p) and named in
+    the bench line's config; greedy runs carry no sampling key."""
+    import bench
+    import synth
+    w = synth.WORKLOADS[1]
+    assert bench.parse_sample(None) is None and bench.parse_sample("") is None
+    smp = bench.parse_sample("0.8,40,0.9")
+    assert smp == (0.8, 40, 0.9) and isinstance(smp[1], int)
+    cfg = bench.run_config(w, 128, 512, 1, "dependency", 4.4e9, smp)
+    assert cfg["sampling"] == {"temperature": 0.8, "top_k": 40, "top_p": 0.9,
+                               "uniforms": "seeded, one per step"}
+    assert "sampling" not in bench.run_config(w, 128, 512, 1, "dependency", 4.4e9)
+    with pytest.raises(ValueError):
+        bench.parse_sample("0.8,40")
